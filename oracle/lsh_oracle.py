@@ -1,0 +1,243 @@
+"""Float64 CPU oracle of shared-QK LSH attention, forward pass.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).  Slow on purpose: plain
+NumPy in float64 on the exact input values, one step of the method at a time,
+no blocking, fusion or reordering beyond what the method itself states.
+
+Sources (the pages this follows, by title and section):
+
+* [GLOSSARY] Ultralytics glossary page "Reformer" (pt), section "Atenção LSH":
+  one shared projection for queries and keys; angular LSH: multiply by a random
+  matrix R and take as bucket the position of the largest value of [xR, -xR];
+  sort tokens by bucket, split the sorted sequence into equal blocks, each
+  token attends to its own block and the previous one; several hashing rounds
+  run in parallel.  Its worked example (d=64, 16 buckets, 1000 rounds, seed 0:
+  72% / 9% shared buckets at cosine 0.96 / 0.04) pins ``oracle_hash``.
+* [ZH-ICLR] twgreatdaily.com article on the ICLR 2020 oral "Reformer: The
+  Efficient Transformer", section "1 LSH Attention": attention of query i as a
+  sum over an admissible key set P_i normalised by a partition function; keys
+  outside the set are masked; Q = K with keys length-normalised; two-level
+  sort by (bucket, position inside the bucket); consecutive equal chunks where
+  a later chunk looks back one chunk; several hash rounds combined.
+* [JA-SCHOLAR] ai-scholar.tech article "計算時間とメモリの壁を打破！
+  Transformerの次世代モデルReformer", sections "Transformerの問題点とは"
+  (scaled dot product, 1/sqrt(d_k)) and "LSH Attention" (bucket, sort, equal
+  chunks, attend to own and previous chunk).
+* [RU-VIDEO] rdly.ru summary "Как уместить 64 000 токенов в одну видеокарту",
+  section "Разделение на блоки (Chunking)": fixed-size blocks of the sorted
+  sequence, each element attends inside its block and the neighbouring one.
+
+Readings where the pages are silent or garbled (each also listed in the design doc):
+
+* chunk 0 has no previous chunk (no wrap-around); the window is a *set* of
+  sorted slots, so a single chunk covering the sequence is not duplicated;
+* no bucket-equality mask inside the window: every key of the two chunks is
+  admissible;
+* queries stay raw, keys are unit-normalised, logit scale defaults to
+  1/sqrt(D);
+* a token does not attend to itself unless it is the only key in its window;
+* rounds are merged by their per-query log-sum-exp weights;
+* argmax ties go to the lowest index; a hash is "near-tie" when the top two
+  values of [p, -p] differ by less than ``TIE_REL`` relative to the top.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+TIE_REL = 1e-5  # relative top-1 / top-2 gap below which a hash counts as a near tie
+
+
+def _f64(a) -> np.ndarray:
+    """Exact float64 copy of an array (bf16 / f32 values are representable)."""
+    if hasattr(a, "detach"):  # a torch tensor: widen on the CPU, exactly
+        import torch
+
+        a = a.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------
+# a1  hash  [GLOSSARY "Atenção LSH"]; [ZH-ICLR §1]; [JA-SCHOLAR "LSH Attention"]
+# ----------------------------------------------------------------------------
+def oracle_hash(qk, R, n_buckets: int, tie_rel: float = TIE_REL, row_block: int = 8192):
+    """Angular LSH bucket of every shared query/key row, for every round.
+
+    qk: [B, H, L, D]; R: [n_rounds, D, n_buckets // 2] (one random projection
+    per round, shared by all batches and heads).
+
+    For each row x and round r: x_hat = x / ||x||, p = x_hat @ R[r]
+    (n_buckets/2 values), u = [p, -p] (n_buckets values, first half from p),
+    bucket = index of the largest entry of u (lowest index on exact ties).
+    near_tie = (u1 - u2) / |u1| < tie_rel with u1 >= u2 the two largest
+    entries of u counted as a multiset.
+
+    Returns (buckets int32 [B, H, n_rounds, L], near_tie bool [B, H, n_rounds, L]).
+    """
+    x = _f64(qk)
+    Rm = _f64(R)
+    B, H, L, D = x.shape
+    n_rounds, D2, half = Rm.shape
+    if D2 != D or 2 * half != n_buckets:
+        raise ValueError("R must be [n_rounds, D, n_buckets // 2]")
+    rows = x.reshape(B * H * L, D)
+    norms = np.sqrt(np.sum(rows * rows, axis=1, keepdims=True))
+    x_hat = rows / np.maximum(norms, 1e-12)
+    buckets = np.empty((B * H * L, n_rounds), dtype=np.int32)
+    near = np.empty((B * H * L, n_rounds), dtype=bool)
+    for r in range(n_rounds):
+        for lo in range(0, B * H * L, row_block):
+            p = x_hat[lo:lo + row_block] @ Rm[r]
+            u = np.concatenate([p, -p], axis=1)
+            buckets[lo:lo + row_block, r] = np.argmax(u, axis=1)  # first maximum
+            top2 = np.partition(u, n_buckets - 2, axis=1)[:, n_buckets - 2:]
+            u2, u1 = top2[:, 0], top2[:, 1]
+            near[lo:lo + row_block, r] = (u1 - u2) / np.maximum(np.abs(u1), 1e-30) < tie_rel
+    buckets = buckets.reshape(B, H, L, n_rounds).transpose(0, 1, 3, 2).copy()
+    near = near.reshape(B, H, L, n_rounds).transpose(0, 1, 3, 2).copy()
+    return buckets, near
+
+
+# ----------------------------------------------------------------------------
+# a2  sort  [ZH-ICLR §1: two-level sort by bucket, then position in bucket];
+#           [JA-SCHOLAR "LSH Attention"]; [GLOSSARY "Atenção LSH"]
+# ----------------------------------------------------------------------------
+def oracle_sort(buckets):
+    """perm[..., s] = original position of sorted slot s, per (b, h, round).
+
+    Tokens are ordered by the key (bucket, position): np.lexsort with the
+    position as the minor key and the bucket as the major key.
+    """
+    b = np.asarray(buckets)
+    L = b.shape[-1]
+    flat = b.reshape(-1, L)
+    pos = np.arange(L)
+    perm = np.empty(flat.shape, dtype=np.int32)
+    for seg in range(flat.shape[0]):
+        perm[seg] = np.lexsort((pos, flat[seg]))
+    return perm.reshape(b.shape)
+
+
+# ----------------------------------------------------------------------------
+# a3 + a4  gather and chunk attention
+#   [ZH-ICLR §1: per-query sum over the admissible set with its partition
+#    function, masked keys, Q = K with normalised keys, later chunk looks back
+#    one chunk]; [JA-SCHOLAR "Transformerの問題点とは": 1/sqrt(d_k)];
+#   [RU-VIDEO "Разделение на блоки"]; [GLOSSARY "Atenção LSH"]
+# ----------------------------------------------------------------------------
+def _window_slots(k: int, chunk: int) -> np.ndarray:
+    """Sorted slots visible to chunk k: chunk k-1 (if it exists) and chunk k."""
+    return np.arange(max(k - 1, 0) * chunk, (k + 1) * chunk)
+
+
+def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale):
+    """Outputs of the queries of sorted chunk k of one (b, h, round) segment.
+
+    Returns (orig positions [c], o [c, D], lse [c]).
+    """
+    q_slots = np.arange(k * chunk, (k + 1) * chunk)
+    w_slots = _window_slots(k, chunk)
+    qi = perm_seg[q_slots]
+    kj = perm_seg[w_slots]
+    logits = (x[qi] @ k_hat[kj].T) * scale  # [c, |W|]
+    if self_mask and len(w_slots) > 1:
+        logits[q_slots[:, None] == w_slots[None, :]] = -np.inf
+    m = np.max(logits, axis=1, keepdims=True)
+    lse = m[:, 0] + np.log(np.sum(np.exp(logits - m), axis=1))
+    weights = np.exp(logits - lse[:, None])
+    return qi, weights @ v[kj], lse
+
+
+def _prep_slice(qk_bh, v_bh):
+    x = _f64(qk_bh)
+    vv = _f64(v_bh)
+    norms = np.sqrt(np.sum(x * x, axis=1, keepdims=True))
+    return x, x / np.maximum(norms, 1e-12), vv
+
+
+def oracle_attend(qk, v, perm, chunk: int, self_mask: bool = True, scale: float | None = None):
+    """Per-round LSH attention outputs in original token order.
+
+    qk, v: [B, H, L, D]; perm: [B, H, n_rounds, L].
+    Returns (o [B, H, n_rounds, L, D] float64, lse [B, H, n_rounds, L] float64).
+    """
+    B, H, L, D = qk.shape
+    perm = np.asarray(perm)
+    n_rounds = perm.shape[2]
+    if L % chunk:
+        raise ValueError("L must be a multiple of chunk")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = np.empty((B, H, n_rounds, L, D))
+    lse = np.empty((B, H, n_rounds, L))
+    for b in range(B):
+        for h in range(H):
+            x, k_hat, vv = _prep_slice(qk[b, h], v[b, h])
+            for r in range(n_rounds):
+                for k in range(L // chunk):
+                    qi, ob, lb = _attend_chunk(x, k_hat, vv, perm[b, h, r], k, chunk, self_mask, scale)
+                    o[b, h, r, qi] = ob
+                    lse[b, h, r, qi] = lb
+    return o, lse
+
+
+def oracle_attend_slots(qk_bh, v_bh, perm_seg, chunk: int, slots, self_mask: bool = True,
+                        scale: float | None = None):
+    """Outputs of selected sorted slots of ONE (b, h, round) segment.
+
+    For checks at sizes where a whole segment is too slow: qk_bh, v_bh are
+    [L, D]; perm_seg is [L]; slots are sorted-slot indices.  The chunk of each
+    slot is evaluated in full and the requested rows are returned.
+
+    Returns (orig positions [n], o [n, D], lse [n]).
+    """
+    L, D = qk_bh.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    x, k_hat, vv = _prep_slice(qk_bh, v_bh)
+    slots = np.asarray(slots)
+    out_pos = np.empty(len(slots), dtype=np.int64)
+    out_o = np.empty((len(slots), D))
+    out_l = np.empty(len(slots))
+    cache = {}
+    for n, s in enumerate(slots):
+        k = int(s) // chunk
+        if k not in cache:
+            cache[k] = _attend_chunk(x, k_hat, vv, np.asarray(perm_seg), k, chunk, self_mask, scale)
+        qi, ob, lb = cache[k]
+        j = int(s) - k * chunk
+        out_pos[n], out_o[n], out_l[n] = qi[j], ob[j], lb[j]
+    return out_pos, out_o, out_l
+
+
+# ----------------------------------------------------------------------------
+# a5  combine rounds  [ZH-ICLR §1: several hash rounds, each with its own
+#      admissible set]; [GLOSSARY "Atenção LSH": rounds run in parallel];
+#      merged by per-query log-sum-exp weights
+# ----------------------------------------------------------------------------
+def oracle_combine(o, lse):
+    """out = sum_r w_r * o_r with w_r = exp(lse_r - LSE), LSE = log sum_r exp(lse_r).
+
+    o: [B, H, n_rounds, L, D]; lse: [B, H, n_rounds, L].
+    Returns (out [B, H, L, D], LSE [B, H, L]).
+    """
+    o = _f64(o)
+    lse = _f64(lse)
+    m = np.max(lse, axis=2, keepdims=True)
+    big = m[:, :, 0] + np.log(np.sum(np.exp(lse - m), axis=2))
+    w = np.exp(lse - big[:, :, None, :])
+    out = np.sum(w[..., None] * o, axis=2)
+    return out, big
+
+
+def oracle_lsh_attention(qk, v, R, n_buckets: int, chunk: int, self_mask: bool = True,
+                         scale: float | None = None):
+    """All four steps end to end.  Returns a dict of every intermediate."""
+    buckets, near = oracle_hash(qk, R, n_buckets)
+    perm = oracle_sort(buckets)
+    o, lse = oracle_attend(_f64(qk), _f64(v), perm, chunk, self_mask, scale)
+    out, lse_out = oracle_combine(o, lse)
+    return {"buckets": buckets, "near_tie": near, "perm": perm, "o_rounds": o,
+            "lse_rounds": lse, "out": out, "lse": lse_out}

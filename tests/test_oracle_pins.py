@@ -1,0 +1,359 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+Runs on the CPU (``-m "not gpu"``).  Each test ties an oracle function to
+something other than itself: the pages' worked example, a closed form, an
+invariant, a textbook library routine, or a pure-Python brute force
+(``tests/brute.py``).
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import (
+    TIE_REL,
+    oracle_attend,
+    oracle_attend_slots,
+    oracle_combine,
+    oracle_hash,
+    oracle_lsh_attention,
+    oracle_sort,
+)
+from tests import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _pct_half_up(frac):
+    return int(math.floor(100.0 * frac + 0.5))
+
+
+# ---------------------------------------------------------------------------
+# hash
+# ---------------------------------------------------------------------------
+def test_hash_collision_demo_matches_glossary_example():
+    """Ultralytics glossary "Reformer", section "Atenção LSH": 72% / 9%."""
+    with open(os.path.join(GOLDEN, "collision_demo.json")) as f:
+        g = json.load(f)
+    dim, nb, rounds = g["dim"], g["n_buckets"], g["rounds"]
+    gen = torch.Generator().manual_seed(g["seed"])
+    query = torch.randn(dim, generator=gen)
+    near = query + 0.3 * torch.randn(dim, generator=gen)
+    far = torch.randn(dim, generator=gen)
+    R = torch.randn(rounds, dim, nb // 2, generator=gen)
+    qk = torch.stack([query, near, far]).reshape(1, 1, 3, dim)
+    buckets, _ = oracle_hash(qk, R, nb)
+    b = buckets[0, 0]  # [rounds, 3]
+    for col, name in ((1, "near"), (2, "far")):
+        shared = float(np.mean(b[:, col] == b[:, 0]))
+        assert _pct_half_up(shared) == g["printed"][name]["shared_bucket_pct"], (name, shared)
+        cos = float(torch.nn.functional.cosine_similarity(query, qk[0, 0, col], dim=0))
+        assert f"{cos:.2f}" == g["printed"][name]["cosine"]
+
+
+def _orthonormal(D, n, seed):
+    q, _ = np.linalg.qr(np.random.default_rng(seed).standard_normal((D, D)))
+    return q[:, :n]
+
+
+@pytest.mark.parametrize("D,nb", [(8, 8), (8, 16), (16, 8), (6, 12)])
+def test_hash_orthonormal_columns_closed_form(D, nb):
+    """x along column k of an orthonormal R gives p = e_k: bucket k; -x gives k + nb/2.
+
+    With D == nb/2 the projection is square, so a transposed R fails here.
+    """
+    half = nb // 2
+    Rr = _orthonormal(D, half, seed=D * 100 + nb)
+    R = Rr[None]
+    rows = []
+    for k in range(half):
+        rows.append(2.5 * Rr[:, k])
+        rows.append(-0.7 * Rr[:, k])
+    qk = np.array(rows)[None, None]
+    buckets, near = oracle_hash(qk, R, nb)
+    want = []
+    for k in range(half):
+        want += [k, k + half]
+    assert buckets[0, 0, 0].tolist() == want
+    assert not near.any()
+
+
+def test_hash_near_tie_flag_threshold():
+    """Two equal projections tie (flagged, lowest index wins); a gap just above 1e-5 is not flagged."""
+    D, nb = 8, 8
+    Rr = _orthonormal(D, nb // 2, seed=3)
+    R = Rr[None]
+    a, b = 1, 3
+    rows = [Rr[:, a] + Rr[:, b],                         # exact tie
+            Rr[:, a] + (1 - 2 * TIE_REL) * Rr[:, b],     # gap 2e-5: not a near tie
+            Rr[:, a] + (1 - 0.5 * TIE_REL) * Rr[:, b],   # gap 5e-6: near tie
+            -(Rr[:, b] + Rr[:, a])]                      # tie on the negative side
+    buckets, near = oracle_hash(np.array(rows)[None, None], R, nb)
+    assert buckets[0, 0, 0].tolist() == [a, a, a, a + nb // 2]
+    assert near[0, 0, 0].tolist() == [True, False, True, True]
+
+
+def test_hash_zero_vector_is_bucket0_and_flagged():
+    R = np.random.default_rng(0).standard_normal((2, 4, 4))
+    buckets, near = oracle_hash(np.zeros((1, 1, 1, 4)), R, 8)
+    assert buckets.ravel().tolist() == [0, 0]
+    assert near.all()
+
+
+def test_hash_invariants_scale_negation_projection_scale():
+    """h(a x) = h(x) (a > 0), h(-x) = (h(x) + nb/2) mod nb, h unchanged by R -> b R (b > 0)."""
+    rng = np.random.default_rng(11)
+    B, H, L, D, nb, nr = 2, 2, 64, 16, 32, 3
+    x = rng.standard_normal((B, H, L, D))
+    R = rng.standard_normal((nr, D, nb // 2))
+    h0, f0 = oracle_hash(x, R, nb)
+    alpha = rng.uniform(0.01, 100.0, size=(B, H, L, 1))
+    h1, f1 = oracle_hash(alpha * x, R, nb)
+    h2, f2 = oracle_hash(-x, R, nb)
+    h3, f3 = oracle_hash(x, 7.25 * R, nb)
+    ok = ~(f0 | f1 | f2 | f3)
+    assert ok.mean() > 0.95
+    assert np.array_equal(h1[ok], h0[ok])
+    assert np.array_equal(h2[ok], ((h0 + nb // 2) % nb)[ok])
+    assert np.array_equal(h3[ok], h0[ok])
+
+
+def test_hash_matches_pure_python_enumeration():
+    rng = np.random.default_rng(5)
+    L, D, nb, nr = 20, 6, 10, 2
+    x = rng.standard_normal((1, 1, L, D))
+    R = rng.standard_normal((nr, D, nb // 2))
+    h, f = oracle_hash(x, R, nb)
+    for r in range(nr):
+        Rl = R[r].tolist()
+        for i in range(L):
+            bk, u1, u2 = brute.brute_hash_row(x[0, 0, i].tolist(), Rl)
+            assert h[0, 0, r, i] == bk
+            assert f[0, 0, r, i] == ((u1 - u2) / max(abs(u1), 1e-30) < TIE_REL)
+
+
+def test_hash_gaussian_marginal_is_uniform():
+    """For any fixed x and R ~ N(0,1), x_hat @ R has iid N(0,1) entries, so every bucket is equally likely.
+
+    One row hashed under many independent rounds gives iid bucket draws (chi-square against uniform).
+    """
+    from scipy import stats
+
+    rng = np.random.default_rng(1)
+    nb, D, rounds = 16, 32, 20000
+    x = rng.standard_normal((1, 1, 1, D))
+    R = rng.standard_normal((rounds, D, nb // 2))
+    h, _ = oracle_hash(x, R, nb)
+    counts = np.bincount(h.ravel(), minlength=nb)
+    assert stats.chisquare(counts).pvalue > 1e-4, counts
+
+
+def test_hash_collision_rate_rises_with_cosine():
+    rng = np.random.default_rng(2)
+    D, nb, rounds = 32, 16, 400
+    q = rng.standard_normal(D)
+    q /= np.linalg.norm(q)
+    w = rng.standard_normal(D)
+    w -= (w @ q) * q
+    w /= np.linalg.norm(w)
+    cosines = [0.0, 0.5, 0.8, 0.95, 0.99]
+    vecs = [q] + [c * q + math.sqrt(1 - c * c) * w for c in cosines]
+    R = rng.standard_normal((rounds, D, nb // 2))
+    h, _ = oracle_hash(np.array(vecs)[None, None], R, nb)
+    rates = [(h[0, 0, :, j + 1] == h[0, 0, :, 0]).mean() for j in range(len(cosines))]
+    assert all(a < b for a, b in zip(rates, rates[1:])), rates
+
+
+# ---------------------------------------------------------------------------
+# sort
+# ---------------------------------------------------------------------------
+def test_sort_matches_tuple_sort_and_invariants():
+    rng = np.random.default_rng(3)
+    buckets = rng.integers(0, 7, size=(2, 3, 2, 50)).astype(np.int32)
+    perm = oracle_sort(buckets)
+    for idx in np.ndindex(*buckets.shape[:-1]):
+        row = buckets[idx].tolist()
+        p = perm[idx].tolist()
+        assert p == brute.brute_sort(row)
+        assert sorted(p) == list(range(50))
+        keys = [(row[i], i) for i in p]
+        assert keys == sorted(keys)
+
+
+def test_sort_skewed_single_bucket_is_identity():
+    b = np.full((1, 1, 1, 300), 5, dtype=np.int32)
+    assert oracle_sort(b)[0, 0, 0].tolist() == list(range(300))
+
+
+# ---------------------------------------------------------------------------
+# attend
+# ---------------------------------------------------------------------------
+def _random_perm(rng, L, nr):
+    return np.stack([rng.permutation(L) for _ in range(nr)]).astype(np.int32)
+
+
+@pytest.mark.parametrize("L,chunk,self_mask", [
+    (24, 4, True), (24, 4, False), (16, 1, True), (16, 16, True), (16, 8, True),
+    (12, 3, False), (8, 1, False),
+])
+def test_attend_matches_admissible_set_enumeration(L, chunk, self_mask):
+    rng = np.random.default_rng(L * 31 + chunk)
+    D, nr = 5, 2
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, nr)[None, None]
+    scale = 0.37
+    o, lse = oracle_attend(qk, v, perm, chunk, self_mask, scale)
+    for r in range(nr):
+        bo, bl = brute.brute_attend_round(qk[0, 0].tolist(), v[0, 0].tolist(),
+                                          perm[0, 0, r].tolist(), chunk, self_mask, scale)
+        for i in range(L):
+            assert np.allclose(o[0, 0, r, i], bo[i], rtol=0, atol=1e-12)
+            assert abs(lse[0, 0, r, i] - bl[i]) < 1e-12
+
+
+@pytest.mark.parametrize("self_mask", [True, False])
+def test_attend_single_chunk_equals_dense_softmax(self_mask):
+    """chunk == L: every round is full softmax attention with normalised keys (and the self mask)."""
+    rng = np.random.default_rng(9)
+    B, H, L, D, nr = 2, 2, 32, 8, 3
+    qk = rng.standard_normal((B, H, L, D))
+    v = rng.standard_normal((B, H, L, D))
+    perm = np.stack([np.stack([_random_perm(rng, L, nr) for _ in range(H)]) for _ in range(B)])
+    o, lse = oracle_attend(qk, v, perm, L, self_mask)
+    scale = 1 / math.sqrt(D)
+    for b in range(B):
+        for h in range(H):
+            x = qk[b, h]
+            kh = x / np.linalg.norm(x, axis=1, keepdims=True)
+            S = (x @ kh.T) * scale
+            if self_mask:
+                np.fill_diagonal(S, -np.inf)
+            Z = np.exp(S).sum(1)
+            dense = (np.exp(S) / Z[:, None]) @ v[b, h]
+            for r in range(nr):
+                assert np.allclose(o[b, h, r], dense, atol=1e-12)
+                assert np.allclose(lse[b, h, r], np.log(Z), atol=1e-12)
+    out, big = oracle_combine(o, lse)
+    assert np.allclose(out, o[:, :, 0], atol=1e-12)
+    assert np.allclose(big, lse[:, :, 0] + math.log(nr), atol=1e-12)
+
+
+def test_attend_convexity_and_constant_values():
+    rng = np.random.default_rng(4)
+    L, D, chunk = 64, 6, 8
+    qk = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, 1)[None, None]
+    o1, _ = oracle_attend(qk, np.ones((1, 1, L, D)), perm, chunk)
+    assert np.allclose(o1, 1.0, atol=1e-12)
+    v = rng.standard_normal((1, 1, L, D))
+    o, _ = oracle_attend(qk, v, perm, chunk)
+    p = perm[0, 0, 0]
+    for s in range(L):
+        W = brute.admissible_slots(s, L, chunk, True)
+        vals = v[0, 0, p[W]]
+        assert np.all(o[0, 0, 0, p[s]] <= vals.max(0) + 1e-12)
+        assert np.all(o[0, 0, 0, p[s]] >= vals.min(0) - 1e-12)
+
+
+def test_attend_chunk1_self_only_fallback():
+    """chunk 1: slot 0 has only itself (o = v_i, lse = |q_i| * scale); slot s > 0 sees only slot s-1."""
+    rng = np.random.default_rng(6)
+    L, D = 6, 4
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, 1)[None, None]
+    scale = 0.5
+    o, lse = oracle_attend(qk, v, perm, 1, True, scale)
+    p = perm[0, 0, 0]
+    i0 = p[0]
+    assert np.allclose(o[0, 0, 0, i0], v[0, 0, i0])
+    assert abs(lse[0, 0, 0, i0] - np.linalg.norm(qk[0, 0, i0]) * scale) < 1e-12
+    for s in range(1, L):
+        i, j = p[s], p[s - 1]
+        assert np.allclose(o[0, 0, 0, i], v[0, 0, j])
+        want = qk[0, 0, i] @ qk[0, 0, j] / np.linalg.norm(qk[0, 0, j]) * scale
+        assert abs(lse[0, 0, 0, i] - want) < 1e-12
+
+
+def test_attend_two_chunks_first_chunk_self_contained():
+    """L / chunk == 2: chunk 0 does not wrap around to chunk 1."""
+    rng = np.random.default_rng(8)
+    L, D, chunk = 8, 3, 4
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, 1)[None, None]
+    o, _ = oracle_attend(qk, v, perm, chunk)
+    v2 = v.copy()
+    v2[0, 0, perm[0, 0, 0, chunk:]] += 100.0  # change every value of chunk 1
+    o2, _ = oracle_attend(qk, v2, perm, chunk)
+    first = perm[0, 0, 0, :chunk]
+    assert np.allclose(o[0, 0, 0, first], o2[0, 0, 0, first], atol=1e-12)
+
+
+def test_attend_slots_matches_full():
+    rng = np.random.default_rng(12)
+    L, D, chunk = 64, 5, 8
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, 1)[None, None]
+    o, lse = oracle_attend(qk, v, perm, chunk)
+    slots = [0, 7, 8, 33, 63]
+    pos, os_, ls = oracle_attend_slots(qk[0, 0], v[0, 0], perm[0, 0, 0], chunk, slots)
+    assert pos.tolist() == perm[0, 0, 0, slots].tolist()
+    assert np.allclose(os_, o[0, 0, 0, pos], atol=0)
+    assert np.allclose(ls, lse[0, 0, 0, pos], atol=0)
+
+
+# ---------------------------------------------------------------------------
+# combine and end to end
+# ---------------------------------------------------------------------------
+def test_combine_equals_softmax_over_multiset_union():
+    rng = np.random.default_rng(13)
+    L, D, chunk, nr = 16, 4, 4, 3
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, nr)[None, None]
+    scale = 0.8
+    o, lse = oracle_attend(qk, v, perm, chunk, True, scale)
+    out, big = oracle_combine(o, lse)
+    bo, bl = brute.brute_multiset_union(qk[0, 0].tolist(), v[0, 0].tolist(),
+                                        [perm[0, 0, r].tolist() for r in range(nr)], chunk, True, scale)
+    for i in range(L):
+        assert np.allclose(out[0, 0, i], bo[i], atol=1e-12)
+        assert abs(big[0, 0, i] - bl[i]) < 1e-12
+
+
+def test_combine_identical_rounds_collapse():
+    rng = np.random.default_rng(14)
+    o1 = rng.standard_normal((2, 1, 1, 10, 3))
+    l1 = rng.standard_normal((2, 1, 1, 10))
+    o = np.repeat(o1, 4, axis=2)
+    l = np.repeat(l1, 4, axis=2)
+    out, big = oracle_combine(o, l)
+    assert np.allclose(out, o1[:, :, 0], atol=1e-12)
+    assert np.allclose(big, l1[:, :, 0] + math.log(4), atol=1e-12)
+
+
+def test_end_to_end_matches_brute_force_pipeline():
+    rng = np.random.default_rng(21)
+    L, D, nb, chunk, nr = 24, 4, 6, 4, 2
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    R = rng.standard_normal((nr, D, nb // 2))
+    res = oracle_lsh_attention(qk, v, R, nb, chunk)
+    X = qk[0, 0].tolist()
+    perms = []
+    for r in range(nr):
+        bk = [brute.brute_hash_row(X[i], R[r].tolist())[0] for i in range(L)]
+        assert bk == res["buckets"][0, 0, r].tolist()
+        perms.append(brute.brute_sort(bk))
+    assert [p for p in perms] == [res["perm"][0, 0, r].tolist() for r in range(nr)]
+    bo, bl = brute.brute_multiset_union(X, v[0, 0].tolist(), perms, chunk, True, 1 / math.sqrt(D))
+    for i in range(L):
+        assert np.allclose(res["out"][0, 0, i], bo[i], atol=1e-12)
+        assert abs(res["lse"][0, 0, i] - bl[i]) < 1e-12

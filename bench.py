@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Throughput of the shared-QK LSH attention forward pass on B200.
+
+One step = the whole hot path over one batch of synthetic input already in
+HBM: lsh_hash -> lsh_sort_permute -> lsh_chunk_attend -> lsh_combine_rounds
+(four C-ABI calls).  Metric: tokens/s = B*H*L / step time, all rounds
+included, at the 64K workload (B 8, H 8, L 65536, D 128, bf16, 1024 buckets,
+chunk 64, 8 rounds).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one rank per GPU: every rank processes its own full
+workload (the (b, h) slices are independent, so there is no collective on the
+data path) -> weak scaling; the step time is the max over ranks.
+
+--impl reference times the float64 CPU oracle (the only other implementation
+of the method here) on rank 0, one bounded sample of the same workload per
+step.  Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LSH-attn fwd tokens/s (B·H·L) at L=64K, 8 rounds, 1×B200; % of roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES = ("hash", "sort", "attend", "combine")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
+
+
+def algorithmic(w):
+    """Algorithmic bytes / flops per stage (per launch = one step over the whole workload).
+
+    Per token-round: bucket write+read 8 B, perm write+read 8 B, gather of the
+    QK and V rows 2*D*s, per-round output write+read 2*(D*s + 4).  Per token:
+    the hash reads the row (D*s) and the merge writes the output (D*s).
+    """
+    s = 2 if w.dtype == "bf16" else 4
+    T = w.tokens
+    TR = T * w.n_rounds
+    row = w.D * s
+    return {
+        "hash": {"bytes": T * row + TR * 4, "flops": 2.0 * T * w.D * (w.n_buckets // 2) * w.n_rounds},
+        "sort": {"bytes": TR * (4 + 4), "flops": 0.0},
+        "attend": {"bytes": TR * (4 + 2 * row + row + 4), "flops": 8.0 * TR * w.chunk * w.D},
+        "combine": {"bytes": TR * (row + 4) + T * row, "flops": 0.0},
+        "total_bytes": TR * (2 * row + 2 * (row + 4) + 8 + 8) + T * 2 * row,
+        "attn_flops": 8.0 * TR * w.chunk * w.D,
+    }
+
+
+def kernel_bound(stage):
+    return "tensor" if stage == "hash" else "hbm"
+
+
+def source_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(stage):
+    """DRAM bytes per launch of `stage` from the committed ncu summary, or None.
+
+    The summary stores a digest of the kernel sources it was taken on; a
+    changed kernel invalidates it.
+    """
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(stage)
+    if not rec:
+        return None
+    try:
+        if source_digest(rec["sources"]) != rec["digest"]:
+            return None
+    except OSError:
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def oracle_sample(w, slices=1, seed=0):
+    """Runs the float64 oracle on `slices` (b, h) slices of the workload, all rounds.
+
+    Returns (seconds, tokens, threads).
+    """
+    import numpy as np
+    import threadpoolctl
+
+    from lsh_attention_hash_b200 import synth
+    from oracle import oracle_lsh_attention
+
+    R = synth.projections(w, seed)
+    tokens, secs = 0, 0.0
+    for n in range(slices):
+        b, h = divmod(n % (w.B * w.H), w.H)
+        qk_s, v_s = synth.slice_inputs(w, b, h, seed)
+        qk = qk_s[None, None]
+        v = v_s[None, None]
+        t0 = time.perf_counter()
+        oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk)
+        secs += time.perf_counter() - t0
+        tokens += w.L
+    info = threadpoolctl.threadpool_info()
+    threads = max([i.get("num_threads", 1) for i in info] + [1])
+    return secs, tokens, threads
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(w, 1)
+    secs, tokens, threads = 0.0, 0, 1
+    for _ in range(args.steps):
+        s, t, threads = oracle_sample(w, 1)
+        secs += s
+        tokens += t
+    value = tokens / secs
+    sample = f"one (b,h) slice of the workload per step ({w.L} tokens, all {w.n_rounds} rounds), float64 NumPy oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {
+        "workload": f"{w.name}: B={w.B} H={w.H} L={w.L} D={w.D} {w.dtype} n_buckets={w.n_buckets} "
+                    f"chunk={w.chunk} n_rounds={w.n_rounds}",
+        "global_batch": w.B, "seq_len": w.L, "heads": w.H, "head_dim": w.D,
+        "parallelism": "replicas (independent (b,h) slices per GPU)",
+        "l2": "inputs larger than L2 (QK+V = %.1f GiB per GPU), no flush" % (2 * w.tokens * w.D * (2 if w.dtype == 'bf16' else 4) / 2**30),
+    }
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import lsh_attention_hash_b200 as lsh
+    from lsh_attention_hash_b200 import binding, synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    qk_h, v_h, R_h = synth.make_inputs(w, seed=rank, pin=True)
+    qk = qk_h.to(dev)
+    v = v_h.to(dev)
+    R = R_h.to(dev)
+    bufs = binding.alloc_buffers(w.B, w.H, w.L, w.D, w.n_rounds, w.n_buckets, w.torch_dtype, dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+
+    def step(record):
+        if record:
+            ev[0].record(stream)
+        lsh.lsh_hash(qk, R, w.n_buckets, buckets=bufs["buckets"], with_near_tie=False, stream=stream)
+        if record:
+            ev[1].record(stream)
+        lsh.lsh_sort_permute(bufs["buckets"], w.n_buckets, perm=bufs["perm"], workspace=bufs["workspace"],
+                             stream=stream)
+        if record:
+            ev[2].record(stream)
+        lsh.lsh_chunk_attend(qk, v, bufs["perm"], w.chunk, out_rounds=bufs["out_rounds"],
+                             lse=bufs["lse_rounds"], stream=stream)
+        if record:
+            ev[3].record(stream)
+        lsh.lsh_combine_rounds(bufs["out_rounds"], bufs["lse_rounds"], out=bufs["out"], want_lse=False,
+                               stream=stream)
+        if record:
+            ev[4].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    assert lsh.lsh_get_device_status(stream) == 0
+
+    stage_ms = {s: 0.0 for s in STAGES}
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step(True)
+            ev[4].synchronize()
+            for i, s in enumerate(STAGES):
+                stage_ms[s] += ev[i].elapsed_time(ev[i + 1])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    assert lsh.lsh_get_device_status(stream) == 0
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # inputs from pinned memory, the four calls, D2H of the output
+    out_h = torch.empty((w.B, w.H, w.L, w.D), dtype=w.torch_dtype, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 3))
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        qk.copy_(qk_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        R.copy_(R_h, non_blocking=True)
+        lsh.lsh_attention(qk, v, R, w.n_buckets, w.chunk, stream=stream, bufs=bufs)
+        out_h.copy_(bufs["out"], non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end)
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = t.tolist()
+
+    if rank != 0:
+        return
+    ms_step = elapsed_ms / args.steps
+    value = world * w.tokens / (ms_step / 1e3)
+    e2e_value = world * w.tokens / (e2e_ms / e2e_steps / 1e3)
+    h2d = qk_h.numel() * qk_h.element_size() + v_h.numel() * v_h.element_size() + R_h.numel() * R_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    peaks, peak_src = load_peaks()
+    alg = algorithmic(w)
+    per_stage = {s: stage_ms[s] / args.steps for s in STAGES}
+    dominant = max(per_stage, key=per_stage.get)
+    bound = kernel_bound(dominant)
+    t_launch = per_stage[dominant] / 1e3
+    if bound == "hbm":
+        achieved = alg[dominant]["bytes"] / t_launch / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    else:
+        achieved = alg[dominant]["flops"] / t_launch / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        unit = "TFLOP/s"
+    t_roof = max(alg["total_bytes"] / (peaks["hbm_gbs"] * 1e9), alg["attn_flops"] / (peaks["bf16_tflops"] * 1e12))
+    launches_per_step = 6 + (1 if w.n_buckets > 16384 else 0)
+    sample_slices = 1
+    c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": workload_config(w),
+        "roofline": {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": recorded_traffic(dominant),
+                     "peak_source": peak_src + (", sustained tensor peak" if bound == "tensor" else "")},
+        "step_roofline": {"t_roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_step,
+                          "alg_bytes": alg["total_bytes"], "attn_flops": alg["attn_flops"],
+                          "note": "max(alg. bytes / HBM peak, chunk-attention FLOPs / bf16 peak) over measured step time"},
+        "stage_ms": per_stage,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": {"value": c_tokens / c_secs, "unit": UNIT, "cores": c_threads, "kind": "oracle",
+                         "sample": f"{sample_slices} (b,h) slice(s) of the workload ({c_tokens} tokens, all "
+                                   f"{w.n_rounds} rounds), float64 NumPy oracle, {c_secs:.1f} s"},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="64k")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from lsh_attention_hash_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

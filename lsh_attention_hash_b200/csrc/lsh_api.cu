@@ -1,0 +1,229 @@
+// C ABI entry points of the LSH attention library: argument validation and
+// kernel dispatch.  Every compute step runs in the kernels included below.
+#include <math.h>
+#include <stdint.h>
+
+#include "attend_simt.cuh"
+#include "combine.cuh"
+#include "common.cuh"
+#include "hash_simt.cuh"
+#include "lsh_attention_hash.h"
+#include "sort.cuh"
+
+namespace {
+
+using lsh::kSortSmemBuckets;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool valid_dtype(int d) { return d == LSH_F32 || d == LSH_BF16; }
+
+inline size_t elt_size(int d) { return d == LSH_F32 ? 4 : 2; }
+
+inline lsh_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
+}
+
+// Common shape rules for row tensors [B, H, L, D].
+inline lsh_status check_bhld(int B, int H, int L, int D) {
+  if (B < 0 || H < 0 || L < 0) return LSH_ERR_SHAPE;
+  if (D < 8 || D > 256 || (D % 8) != 0) return LSH_ERR_SHAPE;
+  if (L > (1 << 24)) return LSH_ERR_SHAPE;
+  return LSH_OK;
+}
+
+inline bool index_space_ok(int B, int H, int L, int n_rounds) {
+  return (long long)B * H * n_rounds * L < (1ll << 31);
+}
+
+}  // namespace
+
+extern "C" {
+
+int lsh_abi_version(void) { return 1; }
+
+const char* lsh_status_string(int s) {
+  switch (s) {
+    case LSH_OK: return "LSH_OK";
+    case LSH_ERR_INVALID_ARG: return "LSH_ERR_INVALID_ARG";
+    case LSH_ERR_SHAPE: return "LSH_ERR_SHAPE";
+    case LSH_ERR_DTYPE: return "LSH_ERR_DTYPE";
+    case LSH_ERR_ALIGN: return "LSH_ERR_ALIGN";
+    case LSH_ERR_WORKSPACE: return "LSH_ERR_WORKSPACE";
+    case LSH_ERR_CUDA: return "LSH_ERR_CUDA";
+    case LSH_ERR_TIMEOUT: return "LSH_ERR_TIMEOUT";
+    case LSH_ERR_UNSUPPORTED: return "LSH_ERR_UNSUPPORTED";
+    default: return "LSH_ERR_UNKNOWN";
+  }
+}
+
+lsh_status lsh_hash(const void* qk, int dtype, int B, int H, int L, int D, const void* R,
+                    int n_rounds, int n_buckets, int32_t* buckets, uint8_t* near_tie, void* stream) {
+  if (!valid_dtype(dtype)) return LSH_ERR_DTYPE;
+  lsh_status st = check_bhld(B, H, L, D);
+  if (st != LSH_OK) return st;
+  if (n_rounds < 1 || n_buckets < 2 || n_buckets > 65536 || (n_buckets & 1)) return LSH_ERR_SHAPE;
+  if (!index_space_ok(B, H, L, n_rounds)) return LSH_ERR_SHAPE;
+  if (!qk || !R || !buckets) return LSH_ERR_INVALID_ARG;
+  if (!aligned16(qk) || !aligned16(R) || !aligned16(buckets) || (near_tie && !aligned16(near_tie)))
+    return LSH_ERR_ALIGN;
+  const long long nrows = (long long)B * H * L;
+  if (nrows == 0) return LSH_OK;
+  const int half = n_buckets / 2;
+  dim3 grid((unsigned)((nrows + lsh::kHashRows - 1) / lsh::kHashRows), (unsigned)n_rounds);
+  const size_t smem = (size_t)lsh::kHashRows * D * sizeof(float);
+  cudaStream_t s = as_stream(stream);
+  if (dtype == LSH_F32)
+    lsh::hash_simt_kernel<float><<<grid, lsh::kHashThreads, smem, s>>>(
+        (const float*)qk, (const float*)R, nrows, L, D, n_rounds, half, buckets, near_tie);
+  else
+    lsh::hash_simt_kernel<__nv_bfloat16><<<grid, lsh::kHashThreads, smem, s>>>(
+        (const __nv_bfloat16*)qk, (const __nv_bfloat16*)R, nrows, L, D, n_rounds, half, buckets,
+        near_tie);
+  return launch_status();
+}
+
+size_t lsh_sort_workspace_bytes(int B, int H, int L, int n_rounds, int n_buckets) {
+  if (B <= 0 || H <= 0 || L <= 0 || n_rounds <= 0 || n_buckets < 2) return 0;
+  return lsh::sort_ws_elems((long long)B * H * n_rounds, L, n_buckets) * sizeof(uint32_t);
+}
+
+lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L, int n_rounds,
+                            int n_buckets, int32_t* perm, int32_t* inv, const void* qk,
+                            const void* v, int dtype, int D, void* qk_sorted, void* v_sorted,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 0 || H < 0 || L < 0 || L > (1 << 24)) return LSH_ERR_SHAPE;
+  if (n_rounds < 1 || n_buckets < 2 || n_buckets > 65536 || (n_buckets & 1)) return LSH_ERR_SHAPE;
+  if (!index_space_ok(B, H, L, n_rounds)) return LSH_ERR_SHAPE;
+  if (!buckets || !perm) return LSH_ERR_INVALID_ARG;
+  const bool gather = qk || v || qk_sorted || v_sorted;
+  if (gather) {
+    if (!qk || !v || !qk_sorted || !v_sorted) return LSH_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype)) return LSH_ERR_DTYPE;
+    lsh_status st = check_bhld(B, H, L, D);
+    if (st != LSH_OK) return st;
+    if (!aligned16(qk) || !aligned16(v) || !aligned16(qk_sorted) || !aligned16(v_sorted))
+      return LSH_ERR_ALIGN;
+  }
+  if (!aligned16(buckets) || !aligned16(perm) || (inv && !aligned16(inv))) return LSH_ERR_ALIGN;
+  const long long segs = (long long)B * H * n_rounds;
+  if (segs == 0 || L == 0) return LSH_OK;
+  const size_t need = lsh_sort_workspace_bytes(B, H, L, n_rounds, n_buckets);
+  if (!workspace || workspace_bytes < need) return LSH_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return LSH_ERR_ALIGN;
+  if (segs > 65535) return LSH_ERR_UNSUPPORTED;  // grid.y limit of this build
+
+  cudaStream_t s = as_stream(stream);
+  const int T = lsh::sort_tile(n_buckets);
+  const int nt = (L + T - 1) / T;
+  uint32_t* cnt = (uint32_t*)workspace;
+  const bool in_smem = n_buckets <= kSortSmemBuckets;
+  const size_t hist_smem = in_smem ? (size_t)n_buckets * sizeof(uint32_t) : 0;
+  if (!in_smem && cudaMemsetAsync(cnt, 0, need, s) != cudaSuccess) return LSH_ERR_CUDA;
+  if (hist_smem > 48 * 1024) {
+    cudaFuncSetAttribute(lsh::sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
+    cudaFuncSetAttribute(lsh::sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
+  }
+  dim3 grid(nt, (unsigned)segs);
+  lsh::sort_count_kernel<<<grid, 256, hist_smem, s>>>(buckets, L, n_buckets, T, cnt);
+  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+  lsh::sort_scan_kernel<<<(unsigned)segs, 1024, 0, s>>>(cnt, (long long)n_buckets * nt);
+  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+  lsh::sort_scatter_kernel<<<grid, 32, hist_smem, s>>>(buckets, L, n_buckets, T, cnt, perm, inv);
+  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+  if (gather) {
+    const int row_bytes = D * (int)elt_size(dtype);
+    const long long nrows = segs * L;
+    const long long work = nrows * (row_bytes / 16);
+    const unsigned blocks = (unsigned)min((work + 255) / 256, 148ll * 64);
+    lsh::gather_rows_kernel<<<blocks, 256, 0, s>>>((const uint8_t*)qk, perm, nrows, L, n_rounds,
+                                                   row_bytes, (uint8_t*)qk_sorted);
+    lsh::gather_rows_kernel<<<blocks, 256, 0, s>>>((const uint8_t*)v, perm, nrows, L, n_rounds,
+                                                   row_bytes, (uint8_t*)v_sorted);
+  }
+  return launch_status();
+}
+
+lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int H, int L, int D,
+                            int n_rounds, const int32_t* perm, const void* qk_sorted,
+                            const void* v_sorted, int chunk, int self_mask, float scale,
+                            void* out_rounds, int out_dtype, float* lse, void* stream) {
+  if (!valid_dtype(dtype) || !valid_dtype(out_dtype)) return LSH_ERR_DTYPE;
+  lsh_status st = check_bhld(B, H, L, D);
+  if (st != LSH_OK) return st;
+  if (n_rounds < 1 || !index_space_ok(B, H, L, n_rounds)) return LSH_ERR_SHAPE;
+  if (chunk < 1 || (L > 0 && (chunk > L || L % chunk != 0))) return LSH_ERR_SHAPE;
+  if (self_mask != 0 && self_mask != 1) return LSH_ERR_INVALID_ARG;
+  if (!qk || !v || !perm || !out_rounds || !lse) return LSH_ERR_INVALID_ARG;
+  if ((qk_sorted == nullptr) != (v_sorted == nullptr)) return LSH_ERR_INVALID_ARG;
+  if (!aligned16(qk) || !aligned16(v) || !aligned16(perm) || !aligned16(out_rounds) ||
+      !aligned16(lse) || (qk_sorted && (!aligned16(qk_sorted) || !aligned16(v_sorted))))
+    return LSH_ERR_ALIGN;
+  const long long segs = (long long)B * H * n_rounds;
+  if (segs == 0 || L == 0) return LSH_OK;
+  if (segs > 65535) return LSH_ERR_UNSUPPORTED;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)D);
+  cudaStream_t s = as_stream(stream);
+
+  const int qb_per_chunk = (chunk + lsh::kAttQ - 1) / lsh::kAttQ;
+  dim3 grid((unsigned)((L / chunk) * qb_per_chunk), (unsigned)segs);
+  const size_t smem = ((size_t)lsh::kAttQ * (D + 1) + lsh::kAttK * (D + 1) + lsh::kAttK * D + lsh::kAttK) * 4;
+  const int threads = lsh::kAttWarps * 32;
+#define LSH_ATT(T, TO)                                                                          \
+  do {                                                                                           \
+    auto kfn = lsh::attend_simt_kernel<T, TO>;                                                   \
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    kfn<<<grid, threads, smem, s>>>((const T*)qk, (const T*)v, perm, (const T*)qk_sorted,        \
+                                    (const T*)v_sorted, L, D, n_rounds, chunk, self_mask, scale, \
+                                    (TO*)out_rounds, lse);                                       \
+  } while (0)
+  if (dtype == LSH_F32) {
+    if (out_dtype == LSH_F32) LSH_ATT(float, float); else LSH_ATT(float, __nv_bfloat16);
+  } else {
+    if (out_dtype == LSH_F32) LSH_ATT(__nv_bfloat16, float); else LSH_ATT(__nv_bfloat16, __nv_bfloat16);
+  }
+#undef LSH_ATT
+  return launch_status();
+}
+
+lsh_status lsh_combine_rounds(const void* out_rounds, int in_dtype, const float* lse, int B, int H,
+                              int L, int D, int n_rounds, void* out, int out_dtype, float* lse_out,
+                              void* stream) {
+  if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return LSH_ERR_DTYPE;
+  lsh_status st = check_bhld(B, H, L, D);
+  if (st != LSH_OK) return st;
+  if (n_rounds < 1 || !index_space_ok(B, H, L, n_rounds)) return LSH_ERR_SHAPE;
+  if (!out_rounds || !lse || !out) return LSH_ERR_INVALID_ARG;
+  if (!aligned16(out_rounds) || !aligned16(lse) || !aligned16(out) || (lse_out && !aligned16(lse_out)))
+    return LSH_ERR_ALIGN;
+  const long long ntok = (long long)B * H * L;
+  if (ntok == 0) return LSH_OK;
+  const long long threads_total = ntok * (D / 8);
+  const unsigned blocks = (unsigned)((threads_total + 255) / 256);
+  cudaStream_t s = as_stream(stream);
+#define LSH_CMB(TI, TO)                                                                   \
+  lsh::combine_kernel<TI, TO><<<blocks, 256, 0, s>>>((const TI*)out_rounds, lse, ntok, L, D, \
+                                                     n_rounds, (TO*)out, lse_out)
+  if (in_dtype == LSH_F32) {
+    if (out_dtype == LSH_F32) LSH_CMB(float, float); else LSH_CMB(float, __nv_bfloat16);
+  } else {
+    if (out_dtype == LSH_F32) LSH_CMB(__nv_bfloat16, float); else LSH_CMB(__nv_bfloat16, __nv_bfloat16);
+  }
+#undef LSH_CMB
+  return launch_status();
+}
+
+lsh_status lsh_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return LSH_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, lsh::g_status, sizeof(int)) != cudaSuccess) return LSH_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(lsh::g_status, &zero, sizeof(int)) != cudaSuccess) return LSH_ERR_CUDA;
+  }
+  return (lsh_status)h;
+}
+
+}  // extern "C"

@@ -1,0 +1,174 @@
+// Stable bucket sort of each (b, h, round) segment, and the sorted-row gather.
+//
+// twgreatdaily ICLR 2020 Reformer article, section "1 LSH Attention": tokens
+// are ordered first by bucket and then by position inside the bucket.  Since
+// positions already ascend within a segment, this is one stable counting sort
+// on the bucket id:
+//   1. count:   per (segment, tile of T positions) histogram of bucket ids,
+//               stored bucket-major: cnt[seg][bucket][tile];
+//   2. scan:    exclusive prefix sum over each segment's cnt array, which makes
+//               cnt[seg][b][t] the first sorted slot of bucket b's elements in
+//               tile t;
+//   3. scatter: one warp walks its tile in position order and places every
+//               element at cnt + (number of equal ids before it), ranking equal
+//               ids inside a group of 32 with a warp match.
+// No step waits on another CTA, so there is no inter-CTA spin.
+#pragma once
+
+#include "common.cuh"
+
+namespace lsh {
+
+constexpr int kSortMinTile = 4096;
+constexpr int kSortSmemBuckets = 16384;  // counters kept in shared memory up to this many buckets
+
+__host__ __device__ inline int sort_tile(int n_buckets) {
+  return n_buckets > kSortMinTile ? n_buckets : kSortMinTile;
+}
+
+__host__ inline size_t sort_ws_elems(long long segs, int L, int n_buckets) {
+  const int T = sort_tile(n_buckets);
+  const long long nt = (L + T - 1) / T;
+  return (size_t)segs * n_buckets * nt;
+}
+
+// 1. histogram of one tile.
+__global__ void __launch_bounds__(256)
+sort_count_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, int T,
+                  uint32_t* __restrict__ cnt) {
+  extern __shared__ uint32_t hist[];
+  const int tile = blockIdx.x, nt = gridDim.x;
+  const long long seg = blockIdx.y;
+  const bool in_smem = n_buckets <= kSortSmemBuckets;
+  uint32_t* gcnt = cnt + (size_t)seg * n_buckets * nt;
+  if (in_smem) {
+    for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+  }
+  const int32_t* src = buckets + (size_t)seg * L;
+  const int lo = tile * T, hi = min(L, lo + T);
+  for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
+    int b = src[i];
+    if ((unsigned)b >= (unsigned)n_buckets) {
+      record_error(LSH_ERR_INVALID_ARG);
+      continue;
+    }
+    if (in_smem) atomicAdd(&hist[b], 1u);
+    else atomicAdd(&gcnt[(size_t)b * nt + tile], 1u);
+  }
+  if (in_smem) {
+    __syncthreads();
+    for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) gcnt[(size_t)b * nt + tile] = hist[b];
+  }
+}
+
+// 2. exclusive scan of one segment's n = n_buckets * nt counters (1024 threads,
+// 4 counters per thread per step, carried across steps).
+__global__ void __launch_bounds__(1024) sort_scan_kernel(uint32_t* __restrict__ cnt, long long n) {
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t carry_s;
+  uint32_t* a = cnt + (size_t)blockIdx.x * n;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry_s = 0;
+  __syncthreads();
+  for (long long base = 0; base < n; base += 4 * 1024) {
+    const long long i0 = base + 4ll * threadIdx.x;
+    uint32_t x[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) x[q] = (i0 + q < n) ? a[i0 + q] : 0u;
+    uint32_t local = x[0] + x[1] + x[2] + x[3];
+    uint32_t incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t w = warp_sums[lane];
+      uint32_t wi = w;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        uint32_t y = __shfl_up_sync(0xffffffffu, wi, off);
+        if (lane >= off) wi += y;
+      }
+      warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
+    }
+    __syncthreads();
+    const uint32_t carry = carry_s;
+    uint32_t run = carry + warp_sums[warp] + incl - local;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (i0 + q < n) a[i0 + q] = run;
+      run += x[q];
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) carry_s = run;
+    __syncthreads();
+  }
+}
+
+// 3. stable scatter of one tile by one warp.
+__global__ void __launch_bounds__(32)
+sort_scatter_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, int T,
+                    uint32_t* __restrict__ cnt, int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  extern __shared__ uint32_t run[];
+  const int tile = blockIdx.x, nt = gridDim.x;
+  const long long seg = blockIdx.y;
+  const int lane = threadIdx.x;
+  const bool in_smem = n_buckets <= kSortSmemBuckets;
+  uint32_t* gcnt = cnt + (size_t)seg * n_buckets * nt;
+  if (in_smem) {
+    for (int b = lane; b < n_buckets; b += 32) run[b] = gcnt[(size_t)b * nt + tile];
+    __syncwarp();
+  }
+  const int32_t* src = buckets + (size_t)seg * L;
+  int32_t* dst = perm + (size_t)seg * L;
+  int32_t* idst = inv ? inv + (size_t)seg * L : nullptr;
+  const int lo = tile * T, hi = min(L, lo + T);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    int b = i < hi ? src[i] : -1;
+    const bool valid = (unsigned)b < (unsigned)n_buckets;
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    unsigned peers = 0;
+    uint32_t slot = 0;
+    if (valid) {
+      peers = __match_any_sync(vmask, b);
+      uint32_t* c = in_smem ? &run[b] : &gcnt[(size_t)b * nt + tile];
+      slot = *c + __popc(peers & lt_mask);
+    }
+    __syncwarp();
+    if (valid && (peers & lt_mask) == 0) {
+      uint32_t* c = in_smem ? &run[b] : &gcnt[(size_t)b * nt + tile];
+      *c += __popc(peers);
+    }
+    __syncwarp();
+    if (valid) {
+      dst[slot] = i;
+      if (idst) idst[i] = (int32_t)slot;
+    }
+  }
+}
+
+// Gather of sorted rows: dst[seg][s][:] = src[bh][perm[seg][s]][:], 16 B per thread.
+__global__ void gather_rows_kernel(const uint8_t* __restrict__ src, const int32_t* __restrict__ perm,
+                                   long long n_rows, int L, int n_rounds, int row_bytes,
+                                   uint8_t* __restrict__ dst) {
+  const int per_row = row_bytes / 16;
+  const long long total = n_rows * per_row;
+  for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < total;
+       t += (long long)gridDim.x * blockDim.x) {
+    const long long row = t / per_row;          // row of the [B, H, n_rounds, L] index space
+    const int piece = (int)(t - row * per_row);
+    const long long seg = row / L;              // (bh, round)
+    const long long bh = seg / n_rounds;
+    const int p = perm[row];
+    const uint8_t* s = src + ((size_t)bh * L + p) * row_bytes + piece * 16;
+    st16(dst + (size_t)row * row_bytes + piece * 16, ld16(s));
+  }
+}
+
+}  // namespace lsh

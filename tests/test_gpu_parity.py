@@ -1,0 +1,191 @@
+"""Parity of the CUDA path (called through the C ABI) with the float64 oracle.
+
+Every test here needs a B200.  Inputs come from lsh_attention_hash_b200.synth;
+expected values come only from oracle/.  See tests/parity.py for the rules
+(bit-exact buckets except near ties, bit-exact perm, max-abs tolerance on
+outputs: 1e-4 for fp32 inputs, 2e-2 for bf16 inputs).
+"""
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import lsh_attention_hash_b200 as lsh
+from lsh_attention_hash_b200 import synth
+from oracle import oracle_combine, oracle_hash, oracle_sort
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run_gpu(w, qk, v, R, self_mask=True, scale=None, out_dtype=None):
+    qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
+    res = lsh.lsh_attention(qk_d, v_d, R_d, w.n_buckets, w.chunk, self_mask=self_mask, scale=scale,
+                            return_all=True)
+    torch.cuda.synchronize()
+    assert lsh.lsh_get_device_status() == 0
+    return res
+
+
+def full_parity(w, qk, v, R, self_mask=True, scale=None):
+    res = run_gpu(w, qk, v, R, self_mask, scale)
+    mism, flagged = parity.check_hash(qk, R, w.n_buckets, res["buckets"], res["near_tie"])
+    parity.check_sort(res["buckets"], res["perm"])
+    parity.check_attend(qk, v, res["perm"], w.chunk, self_mask, scale, res["o_rounds"], res["lse_rounds"],
+                        w.torch_dtype)
+    parity.check_combine(res["o_rounds"], res["lse_rounds"], res["out"], res["lse"], w.torch_dtype)
+    if mism == 0:  # all buckets agree: the whole pipeline must agree with the oracle's own run
+        from oracle import oracle_lsh_attention
+
+        ref = oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, self_mask, scale)
+        assert np.array_equal(ref["perm"], parity.np_(res["perm"]))
+        err = float(np.max(np.abs(ref["out"] - parity.f64(res["out"]))))
+        assert err <= parity.TOL[w.torch_dtype], err
+    return res, mism, flagged
+
+
+def test_tiny_workload_end_to_end():
+    w = synth.WORKLOADS["tiny"]
+    qk, v, R = synth.make_inputs(w)
+    _, mism, _ = full_parity(w, qk, v, R)
+    assert mism == 0
+
+
+def test_4k_workload_end_to_end():
+    w = synth.WORKLOADS["4k"]
+    qk, v, R = synth.make_inputs(w)
+    full_parity(w, qk, v, R)
+
+
+EDGE_CASES = [
+    # name, B, H, L, D, dtype, n_buckets, chunk, n_rounds, self_mask
+    ("ragged_rows_bf16", 1, 3, 200, 64, "bf16", 16, 8, 3, True),
+    ("chunk1_self_only", 1, 2, 64, 64, "bf16", 8, 1, 2, True),
+    ("chunk_eq_L", 2, 1, 256, 128, "bf16", 32, 256, 2, True),
+    ("two_chunks", 1, 2, 128, 128, "bf16", 8, 64, 2, True),
+    ("no_self_mask", 2, 2, 512, 128, "bf16", 16, 64, 2, False),
+    ("two_buckets", 1, 2, 384, 64, "bf16", 2, 64, 3, True),
+    ("fp32_odd_sizes", 1, 3, 120, 40, "f32", 10, 12, 2, True),
+    ("fp32_d256", 1, 1, 256, 256, "f32", 64, 32, 1, True),
+    ("many_buckets", 1, 1, 2048, 64, "bf16", 4096, 64, 2, True),
+    ("big_chunk", 1, 1, 4096, 64, "bf16", 8, 2048, 1, True),
+]
+
+
+@pytest.mark.parametrize("case", EDGE_CASES, ids=[c[0] for c in EDGE_CASES])
+def test_edge_cases(case):
+    name, B, H, L, D, dt, nb, c, nr, sm = case
+    w = synth.small_workload(name, B, H, L, D, dt, nb, c, nr)
+    qk, v, R = synth.make_inputs(w, seed=zlib.crc32(name.encode()) % 1000)
+    full_parity(w, qk, v, R, self_mask=sm)
+
+
+def test_zero_rows_and_custom_scale():
+    w = synth.small_workload("zero", 1, 1, 256, 64, "bf16", 16, 32, 2)
+    qk, v, R = synth.make_inputs(w, seed=3)
+    qk[0, 0, 5] = 0
+    qk[0, 0, 77] = 0
+    res = run_gpu(w, qk, v, R, scale=0.3)
+    nb = res["buckets"].cpu()
+    assert nb[0, 0, :, 5].tolist() == [0, 0] and nb[0, 0, :, 77].tolist() == [0, 0]
+    assert res["near_tie"].cpu()[0, 0, :, 5].tolist() == [1, 1]
+    full_parity(w, qk, v, R, scale=0.3)
+
+
+def test_fp32_output_from_bf16_input():
+    w = synth.small_workload("f32out", 2, 2, 512, 128, "bf16", 16, 64, 2)
+    qk, v, R = synth.make_inputs(w, seed=4)
+    qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
+    b, _ = lsh.lsh_hash(qk_d, R_d, w.n_buckets)
+    perm, _, _, _ = lsh.lsh_sort_permute(b, w.n_buckets)
+    o, lse = lsh.lsh_chunk_attend(qk_d, v_d, perm, w.chunk, out_dtype=torch.float32)
+    out, lse_out = lsh.lsh_combine_rounds(o, lse, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    parity.check_attend(qk, v, perm, w.chunk, True, None, o, lse, torch.bfloat16)
+    ref, _ = oracle_combine(parity.f64(o), parity.f64(lse))
+    assert np.max(np.abs(ref - parity.f64(out))) < 1e-5  # fp32 in, fp32 out
+
+
+def test_sorted_gather_and_inverse():
+    w = synth.small_workload("gather", 2, 2, 1024, 128, "bf16", 32, 64, 3)
+    qk, v, R = synth.make_inputs(w, seed=5)
+    qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
+    b, _ = lsh.lsh_hash(qk_d, R_d, w.n_buckets)
+    perm, inv, qs, vs = lsh.lsh_sort_permute(b, w.n_buckets, want_inv=True, qk=qk_d, v=v_d)
+    o1, l1 = lsh.lsh_chunk_attend(qk_d, v_d, perm, w.chunk)
+    o2, l2 = lsh.lsh_chunk_attend(qk_d, v_d, perm, w.chunk, qk_sorted=qs, v_sorted=vs)
+    torch.cuda.synchronize()
+    p = perm.long()
+    idx = torch.arange(w.L, device=DEV).expand_as(p)
+    assert torch.equal(torch.gather(inv.long(), -1, p), idx)
+    for r in range(w.n_rounds):
+        assert torch.equal(qs[:, :, r], torch.gather(qk_d, 2, p[:, :, r, :, None].expand(-1, -1, -1, w.D)))
+        assert torch.equal(vs[:, :, r], torch.gather(v_d, 2, p[:, :, r, :, None].expand(-1, -1, -1, w.D)))
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_deterministic_reruns():
+    w = synth.small_workload("det", 2, 2, 2048, 128, "bf16", 64, 64, 2)
+    qk, v, R = synth.make_inputs(w, seed=6)
+    a = run_gpu(w, qk, v, R)
+    b = run_gpu(w, qk, v, R)
+    for k in ("buckets", "near_tie", "perm", "o_rounds", "lse_rounds", "out", "lse"):
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_out_of_range_bucket_is_recorded_not_faulted():
+    """A host-made failure: bucket ids outside [0, n_buckets) are skipped and reported."""
+    buckets = torch.zeros((1, 1, 1, 1024), dtype=torch.int32, device=DEV)
+    buckets[0, 0, 0, 10] = 99
+    buckets[0, 0, 0, 11] = -3
+    perm = torch.full_like(buckets, -1)
+    lsh.lsh_sort_permute(buckets, 16, perm=perm)
+    assert lsh.lsh_get_device_status() == 1  # LSH_ERR_INVALID_ARG
+    assert lsh.lsh_get_device_status() == 0  # cleared by the read
+    p = perm.cpu()[0, 0, 0]
+    assert p[:1022].tolist() == [i for i in range(1024) if i not in (10, 11)]
+
+
+def _sampled_slices(w, slices, row_sample=None, slot_sample=None):
+    qk, v, R = synth.make_inputs(w)
+    res = run_gpu(w, qk, v, R)
+    for (b, h) in slices:
+        qk_bh, v_bh = qk[b, h], v[b, h]
+        rows = np.arange(w.L) if row_sample is None else np.sort(
+            np.random.default_rng(b * 100 + h).choice(w.L, row_sample, replace=False))
+        g_b = res["buckets"][b, h].cpu()
+        g_f = res["near_tie"][b, h].cpu()
+        parity.check_hash(qk_bh[rows][None, None], R, w.n_buckets, g_b[:, rows][None, None],
+                          g_f[:, rows][None, None])
+        parity.check_sort(g_b[None, None], res["perm"][b, h].cpu()[None, None])
+        slots = None if slot_sample is None else np.sort(
+            np.random.default_rng(b * 7 + h).choice(w.L, slot_sample, replace=False))
+        parity.check_slice_rounds(qk_bh, v_bh, res["perm"][b, h].cpu(), w.chunk, True, None,
+                                  res["o_rounds"][b, h].cpu(), res["lse_rounds"][b, h].cpu(), w.torch_dtype,
+                                  slots)
+        parity.check_combine(res["o_rounds"][b, h][None, None], res["lse_rounds"][b, h][None, None],
+                             res["out"][b, h][None, None], res["lse"][b, h][None, None], w.torch_dtype)
+    return res
+
+
+def test_skewed_workload_sampled_slices():
+    w = synth.WORKLOADS["skewed16k"]
+    res = _sampled_slices(w, [(0, 0), (5, 3)])
+    # the workload is meant to be uneven: the largest bucket is many times the mean
+    counts = torch.bincount(res["buckets"][0, 0, 0].long(), minlength=w.n_buckets)
+    assert counts.max().item() > 8 * w.L / w.n_buckets
+
+
+@pytest.mark.slow
+def test_64k_workload_sampled_slices():
+    w = synth.WORKLOADS["64k"]
+    _sampled_slices(w, [(0, 0), (7, 7)], slot_sample=4096)
+
+
+@pytest.mark.slow
+def test_1m_workload_sampled_slices():
+    w = synth.WORKLOADS["1m"]
+    _sampled_slices(w, [(0, 0), (0, 6)], row_sample=4096, slot_sample=2048)

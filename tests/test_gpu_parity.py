@@ -30,9 +30,9 @@ def run_gpu(w, qk, v, R, self_mask=True, scale=None, out_dtype=None):
     return res
 
 
-def full_parity(w, qk, v, R, self_mask=True, scale=None):
+def full_parity(w, qk, v, R, self_mask=True, scale=None, max_flag_frac=1e-3):
     res = run_gpu(w, qk, v, R, self_mask, scale)
-    mism, flagged = parity.check_hash(qk, R, w.n_buckets, res["buckets"], res["near_tie"])
+    mism, flagged = parity.check_hash(qk, R, w.n_buckets, res["buckets"], res["near_tie"], max_flag_frac)
     parity.check_sort(res["buckets"], res["perm"])
     parity.check_attend(qk, v, res["perm"], w.chunk, self_mask, scale, res["o_rounds"], res["lse_rounds"],
                         w.torch_dtype)
@@ -92,7 +92,8 @@ def test_zero_rows_and_custom_scale():
     nb = res["buckets"].cpu()
     assert nb[0, 0, :, 5].tolist() == [0, 0] and nb[0, 0, :, 77].tolist() == [0, 0]
     assert res["near_tie"].cpu()[0, 0, :, 5].tolist() == [1, 1]
-    full_parity(w, qk, v, R, scale=0.3)
+    # the two planted zero rows are near ties in both rounds: 4 of 512 hashes
+    full_parity(w, qk, v, R, scale=0.3, max_flag_frac=4 / 512 + 1e-3)
 
 
 def test_fp32_output_from_bf16_input():

@@ -1,9 +1,14 @@
 // C ABI entry points of the LSH attention library: argument validation and
 // kernel dispatch.  Every compute step runs in the kernels included below.
 #include <math.h>
+
+#include <algorithm>
 #include <stdint.h>
 
+#include <cudaTypedefs.h>
+
 #include "attend_simt.cuh"
+#include "attend_tc.cuh"
 #include "combine.cuh"
 #include "common.cuh"
 #include "hash_simt.cuh"
@@ -36,6 +41,94 @@ inline lsh_status check_bhld(int B, int H, int L, int D) {
 
 inline bool index_space_ok(int B, int H, int L, int n_rounds) {
   return (long long)B * H * n_rounds * L < (1ll << 31);
+}
+
+// Device properties of the current device, cached per device ordinal.
+struct DevInfo {
+  int major = 0, sms = 0;
+};
+inline DevInfo dev_info() {
+  static DevInfo cache[64];
+  static bool have[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DevInfo{};
+  if (!have[dev]) {
+    DevInfo d;
+    cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = d;
+    have[dev] = true;
+  }
+  return cache[dev];
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the
+// library does not link libcuda directly).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+inline EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    tried = true;
+  }
+  return fn;
+}
+
+// 2D bf16 view [rows, D] whose box is one row of 64 elements (128 B), 128-byte
+// swizzle: the source of tile::gather4 row gathers.
+inline bool make_row_gather_map(CUtensorMap* map, const void* base, long long rows, int D) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core chunk attention (bf16, chunk 64, D 64 or 128) on sm_100.
+template <int D, typename TO>
+lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted, const void* v_sorted,
+                            const int32_t* perm, int B, int H, int L, int n_rounds, int self_mask, float scale,
+                            void* out, float* lse, cudaStream_t s, int sms) {
+  using namespace lsh::att_tc;
+  const long long segs = (long long)B * H * n_rounds;
+  const bool sorted = qk_sorted != nullptr;
+  CUtensorMap mqk, mv;
+  const long long rows = sorted ? segs * L : (long long)B * H * L;
+  if (!make_row_gather_map(&mqk, sorted ? qk_sorted : qk, rows, D) ||
+      !make_row_gather_map(&mv, sorted ? v_sorted : v, rows, D))
+    return LSH_ERR_CUDA;
+  Params p;
+  p.perm = perm;
+  p.out = out;
+  p.lse = lse;
+  p.L = L;
+  p.n_rounds = n_rounds;
+  p.n_chunks = L / kC;
+  p.n_steps = (p.n_chunks + 1) / 2;
+  p.run = 32;
+  p.units_per_seg = (p.n_steps + p.run - 1) / p.run;
+  p.n_units = segs * p.units_per_seg;
+  p.self_mask = self_mask;
+  p.colscale = scale * 1.4426950408889634f;  // log2(e)
+  p.sorted_input = sorted ? 1 : 0;
+  const unsigned grid = (unsigned)std::min<long long>(p.n_units, sms);
+  auto kfn = attend_tc_kernel<D, TO>;
+  const int smem = (int)Layout<D>::kSmem;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return LSH_ERR_CUDA;
+  kfn<<<grid, kThreads, smem, s>>>(mqk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
 }
 
 }  // namespace
@@ -166,6 +259,19 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
   if (segs > 65535) return LSH_ERR_UNSUPPORTED;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)D);
   cudaStream_t s = as_stream(stream);
+
+  const DevInfo di = dev_info();
+  if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && di.major == 10) {
+#define LSH_ATT_TC(DD, TO)                                                                            \
+  return launch_attend_tc<DD, TO>(qk, v, qk_sorted, v_sorted, perm, B, H, L, n_rounds, self_mask, scale, \
+                                  out_rounds, lse, s, di.sms)
+    if (D == 128) {
+      if (out_dtype == LSH_BF16) LSH_ATT_TC(128, __nv_bfloat16); else LSH_ATT_TC(128, float);
+    } else {
+      if (out_dtype == LSH_BF16) LSH_ATT_TC(64, __nv_bfloat16); else LSH_ATT_TC(64, float);
+    }
+#undef LSH_ATT_TC
+  }
 
   const int qb_per_chunk = (chunk + lsh::kAttQ - 1) / lsh::kAttQ;
   dim3 grid((unsigned)((L / chunk) * qb_per_chunk), (unsigned)segs);

@@ -72,6 +72,11 @@ EDGE_CASES = [
     ("fp32_d256", 1, 1, 256, 256, "f32", 64, 32, 1, True),
     ("many_buckets", 1, 1, 2048, 64, "bf16", 4096, 64, 2, True),
     ("big_chunk", 1, 1, 4096, 64, "bf16", 8, 2048, 1, True),
+    # chunk 64 bf16 (tensor-core kernel): odd chunk count, one chunk, several work units per segment
+    ("tc_odd_chunks", 1, 2, 192, 128, "bf16", 8, 64, 2, True),
+    ("tc_single_chunk", 2, 1, 64, 64, "bf16", 4, 64, 3, True),
+    ("tc_units_d64", 1, 1, 8256, 64, "bf16", 128, 64, 2, True),
+    ("tc_units_d128_nomask", 1, 2, 8192, 128, "bf16", 128, 64, 1, False),
 ]
 
 

@@ -1,0 +1,255 @@
+// Angular LSH hash on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Ultralytics glossary "Reformer", section "Atencao LSH": bucket = position of
+// the largest value of [xR, -xR] for a random projection R per round.
+//
+// Served case: bf16 rows, D in {64, 128}, n_buckets/2 = `half` a multiple of
+// 64 with half <= 256 or half % 256 == 0, and R[round] small enough to stay in
+// shared memory (D * half * 2 <= 128 KB).  Each persistent CTA owns one round:
+// R[round] is loaded once by TMA (MN-major, 128-byte swizzle) and 128-row tiles
+// of QK stream through a two-stage TMA ring.  p = x R accumulates in fp32 in
+// TMEM (two buffers of NC <= 256 columns, so the next tile's UMMA overlaps the
+// current epilogue).
+//
+// Epilogue (one row per thread): the bucket is argmax over [p, -p], i.e. the
+// largest |p_k| and its sign.  Values are handled in groups of 16: the key of
+// p_k is |p_k| with its 4 lowest mantissa bits replaced by (15 - k % 16), so a
+// 3-input max tree over the keys yields the group's largest |p| (to 2^-19
+// relative, far below the 1e-5 near-tie threshold) together with its
+// position (ties prefer the lower column); a max tree over the raw values of
+// the winning group tells its sign.  The exact top-two |p| for the near-tie
+// flag are tracked only when that output is requested.
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace lsh {
+namespace hash_tc {
+
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 UMMA, warps 2-5 epilogue
+constexpr int kRows = 128;
+constexpr int kStages = 2;
+
+template <int D>
+struct Layout {
+  static constexpr uint32_t kHalfBytes = kRows * 128;           // 128 rows x 64 bf16
+  static constexpr uint32_t kStageBytes = (D / 64) * kHalfBytes;
+  static constexpr uint32_t kA = 0;
+  static constexpr uint32_t kR = kStages * kStageBytes;          // R[round]: (half/64) boxes of D x 128 B
+  __host__ __device__ static constexpr uint32_t bar_off(int half) { return kR + (uint32_t)D * half * 2; }
+  // a_full[2] a_empty[2] acc_full[2] acc_empty[2] r_full done
+  static constexpr int kNumBars = 10;
+  __host__ __device__ static constexpr uint32_t smem_bytes(int half) { return bar_off(half) + kNumBars * 8 + 16 + 1024; }
+};
+
+struct Params {
+  int32_t* buckets;    // [B*H][n_rounds][L]
+  uint8_t* near_tie;   // same, nullable
+  long long nrows;     // B*H*L
+  int L;
+  int n_rounds;
+  int half;
+  int nchunks;         // half / NC
+  int per_round;       // CTAs per round
+  long long n_tiles;
+};
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// max over 16 values with 3-input maxima
+__device__ __forceinline__ float max16(const float* v) {
+  const float a = max3(v[0], v[1], v[2]), b = max3(v[3], v[4], v[5]), c = max3(v[6], v[7], v[8]);
+  const float d = max3(v[9], v[10], v[11]), e = max3(v[12], v[13], v[14]);
+  return max3(max3(a, b, c), d, fmaxf(e, v[15]));
+}
+
+struct RowState {
+  float best_key;   // largest key so far
+  int best_g;       // its group (16 columns) within the round
+  float best_raw;   // largest raw value of that group
+  float v1, v2;     // exact top-two |p| (near-tie flag only)
+};
+
+template <bool FLAG>
+__device__ __forceinline__ void process16(RowState& st, const uint32_t* raw, int g) {
+  float key[16], val[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    val[j] = __uint_as_float(raw[j]);
+    key[j] = __uint_as_float((raw[j] & 0x7FFFFFF0u) | (uint32_t)(15 - j));
+  }
+  const float gk = max16(key);
+  const float gr = max16(val);
+  const bool gt = gk > st.best_key;
+  st.best_key = gt ? gk : st.best_key;
+  st.best_g = gt ? g : st.best_g;
+  st.best_raw = gt ? gr : st.best_raw;
+  if (FLAG) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float a = fabsf(val[j]);
+      st.v2 = fmaxf(st.v2, fminf(st.v1, a));
+      st.v1 = fmaxf(st.v1, a);
+    }
+  }
+}
+
+template <int D, int NC, bool FLAG>
+__global__ void __launch_bounds__(kThreads, 1)
+hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_r,
+               const Params p) {
+  using Lay = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off(p.half));
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = bars + 2;
+  uint64_t* acc_full = bars + 4;
+  uint64_t* acc_empty = bars + 6;
+  uint64_t* r_full = bars + 8;
+  uint64_t* done_bar = bars + 9;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + Lay::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + Lay::kNumBars) + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int round = blockIdx.x % p.n_rounds;
+  const int first_tile = blockIdx.x / p.n_rounds;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&a_full[i], 1);
+      tc::mbar_init(&a_empty[i], 1);
+      tc::mbar_init(&acc_full[i], 1);
+      tc::mbar_init(&acc_empty[i], 128);
+    }
+    tc::mbar_init(r_full, 1);
+    tc::mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_holder, 2 * NC < 32 ? 32 : 2 * NC);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tensormap(&map_x);
+      tc::prefetch_tensormap(&map_r);
+      tc::mbar_arrive_expect_tx(r_full, (uint32_t)D * p.half * 2);
+      for (int b = 0; b < p.half / 64; ++b)
+        tc::tma_load_2d(smem + Lay::kR + b * D * 128, &map_r, r_full, b * 64, round * D);
+      uint32_t it = 0;
+      bool ok = true;
+      for (long long tile = first_tile; tile < p.n_tiles; tile += p.per_round, ++it) {
+        const int s = it % kStages;
+        ok = tc::mbar_wait(&a_empty[s], ((it / kStages) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        tc::mbar_arrive_expect_tx(&a_full[s], kRows * D * 2);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tc::tma_load_2d(smem + Lay::kA + s * Lay::kStageBytes + h * Lay::kHalfBytes, &map_x, &a_full[s], h * 64,
+                          (int)(tile * kRows));
+      }
+      // never leave with copies in flight
+      for (uint32_t k = (it > kStages ? it - kStages : 0); k < it; ++k) {
+        const unsigned long long t0 = tc::globaltimer();
+        while (!tc::mbar_try_wait(&a_full[k % kStages], (k / kStages) & 1))
+          if (tc::globaltimer() - t0 > tc::kWaitNs / 16) break;
+      }
+      {
+        const unsigned long long t0 = tc::globaltimer();
+        while (!tc::mbar_try_wait(r_full, 0))
+          if (tc::globaltimer() - t0 > tc::kWaitNs / 16) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(128, NC, 0, 1);
+      const uint32_t a0 = tc::smem_u32(smem + Lay::kA);
+      const uint32_t r0 = tc::smem_u32(smem + Lay::kR);
+      bool ok = tc::mbar_wait(r_full, 0, abort_flag);
+      uint32_t it = 0, seq = 0;
+      for (long long tile = first_tile; ok && tile < p.n_tiles; tile += p.per_round, ++it) {
+        const int s = it % kStages;
+        ok = tc::mbar_wait(&a_full[s], (it / kStages) & 1, abort_flag);
+        if (!ok) break;
+        for (int c = 0; c < p.nchunks; ++c, ++seq) {
+          const int b = seq & 1;
+          ok = tc::mbar_wait(&acc_empty[b], ((seq >> 1) & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          tc::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = tc::sdesc_sw128(a0 + s * Lay::kStageBytes + (kk >> 2) * Lay::kHalfBytes + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = tc::sdesc_sw128(r0 + (c * (NC / 64)) * D * 128 + kk * 2048, D * 128, 1024);
+            tc::umma_ss(tmem + b * NC, ad, bd, idesc, kk > 0);
+          }
+          tc::umma_commit(&acc_full[b]);
+        }
+        if (!ok) break;
+        tc::umma_commit(&a_empty[s]);
+      }
+      tc::umma_commit(done_bar);
+      const unsigned long long t0 = tc::globaltimer();
+      while (!tc::mbar_try_wait(done_bar, 0))
+        if (tc::globaltimer() - t0 > tc::kWaitNs / 16) break;
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    uint32_t seq = 0;
+    bool ok = true;
+    for (long long tile = first_tile; ok && tile < p.n_tiles; tile += p.per_round) {
+      RowState st{-1.f, 0, 0.f, -INFINITY, -INFINITY};
+      for (int c = 0; c < p.nchunks; ++c, ++seq) {
+        const int b = seq & 1;
+        ok = att_tc::warp_wait(&acc_full[b], (seq >> 1) & 1, abort_flag);
+        if (!ok) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int piece = 0; piece < NC / 32; ++piece) {
+          uint32_t raw[32];
+          tc::tmem_ld32(lane_base + tmem + b * NC + piece * 32, raw);
+          tc::tmem_wait_ld();
+          const int g = c * (NC / 16) + piece * 2;
+          process16<FLAG>(st, raw, g);
+          process16<FLAG>(st, raw + 16, g + 1);
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(&acc_empty[b]);
+      }
+      if (!ok) break;
+      const long long row = tile * kRows + r;
+      if (row < p.nrows) {
+        const uint32_t kb = __float_as_uint(st.best_key);
+        const int k = st.best_g * 16 + (15 - (int)(kb & 15u));
+        const bool pos = st.best_raw >= 0.f && ((__float_as_uint(st.best_raw) & 0x7FFFFFF0u) == (kb & 0x7FFFFFF0u));
+        const long long bh = row / p.L, l = row - bh * p.L;
+        const size_t o = ((size_t)bh * p.n_rounds + round) * p.L + l;
+        p.buckets[o] = pos ? k : k + p.half;
+        if (FLAG) {
+          const float u1 = st.v1, u2 = fmaxf(st.v2, -st.v1);
+          p.near_tie[o] = (u1 - u2) < kTieRel * fmaxf(u1, 1e-30f) ? 1 : 0;
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 2 * NC < 32 ? 32 : 2 * NC);
+  }
+}
+
+}  // namespace hash_tc
+}  // namespace lsh

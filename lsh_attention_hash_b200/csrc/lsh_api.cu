@@ -12,6 +12,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "hash_simt.cuh"
+#include "hash_tc.cuh"
 #include "lsh_attention_hash.h"
 #include "sort.cuh"
 
@@ -95,6 +96,67 @@ inline bool make_row_gather_map(CUtensorMap* map, const void* base, long long ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D bf16 view [rows, cols] with a box of box_cols x box_rows, 128-byte swizzle.
+inline bool make_tile_map(CUtensorMap* map, const void* base, long long rows, long long cols, int box_cols,
+                          int box_rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Whether the tensor-core hash serves this shape (see hash_tc.cuh).
+inline bool hash_tc_eligible(int dtype, int D, int half, int n_rounds, const DevInfo& di) {
+  if (dtype != LSH_BF16 || di.major != 10 || (D != 64 && D != 128)) return false;
+  if (half % 64 != 0 || !(half <= 256 ? (half == 64 || half == 128 || half == 256) : half % 256 == 0)) return false;
+  if ((long long)D * half * 2 > 128 * 1024) return false;
+  return n_rounds <= di.sms;
+}
+
+template <int D, int NC, bool FLAG>
+lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, int n_rounds, int half,
+                          int32_t* buckets, uint8_t* near_tie, cudaStream_t s, int sms) {
+  using namespace lsh::hash_tc;
+  const long long rows = (long long)B * H * L;
+  CUtensorMap mx, mr;
+  if (!make_tile_map(&mx, qk, rows, D, 64, kRows) || !make_tile_map(&mr, R, (long long)n_rounds * D, half, 64, D))
+    return LSH_ERR_CUDA;
+  Params p;
+  p.buckets = buckets;
+  p.near_tie = near_tie;
+  p.nrows = rows;
+  p.L = L;
+  p.n_rounds = n_rounds;
+  p.half = half;
+  p.nchunks = half / NC;
+  p.n_tiles = (rows + kRows - 1) / kRows;
+  p.per_round = (int)std::max<long long>(1, std::min<long long>(sms / n_rounds, p.n_tiles));
+  const unsigned grid = (unsigned)(p.per_round * n_rounds);
+  auto kfn = hash_tc_kernel<D, NC, FLAG>;
+  const int smem = (int)Layout<D>::smem_bytes(half);
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return LSH_ERR_CUDA;
+  kfn<<<grid, kThreads, smem, s>>>(mx, mr, p);
+  return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
+}
+
+template <int D>
+lsh_status dispatch_hash_tc(const void* qk, const void* R, int B, int H, int L, int n_rounds, int half,
+                            int32_t* buckets, uint8_t* near_tie, cudaStream_t s, int sms) {
+#define LSH_HTC(NC)                                                                                           \
+  return near_tie ? launch_hash_tc<D, NC, true>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, sms)   \
+                  : launch_hash_tc<D, NC, false>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, sms)
+  if (half == 64) LSH_HTC(64);
+  if (half == 128) LSH_HTC(128);
+  LSH_HTC(256);
+#undef LSH_HTC
+}
+
 // Tensor-core chunk attention (bf16, chunk 64, D 64 or 128) on sm_100.
 template <int D, typename TO>
 lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted, const void* v_sorted,
@@ -165,6 +227,12 @@ lsh_status lsh_hash(const void* qk, int dtype, int B, int H, int L, int D, const
   const long long nrows = (long long)B * H * L;
   if (nrows == 0) return LSH_OK;
   const int half = n_buckets / 2;
+  const DevInfo di = dev_info();
+  if (hash_tc_eligible(dtype, D, half, n_rounds, di)) {
+    cudaStream_t s = as_stream(stream);
+    if (D == 128) return dispatch_hash_tc<128>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, di.sms);
+    return dispatch_hash_tc<64>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, di.sms);
+  }
   dim3 grid((unsigned)((nrows + lsh::kHashRows - 1) / lsh::kHashRows), (unsigned)n_rounds);
   const size_t smem = (size_t)lsh::kHashRows * D * sizeof(float);
   cudaStream_t s = as_stream(stream);

@@ -77,6 +77,11 @@ EDGE_CASES = [
     ("tc_single_chunk", 2, 1, 64, 64, "bf16", 4, 64, 3, True),
     ("tc_units_d64", 1, 1, 8256, 64, "bf16", 128, 64, 2, True),
     ("tc_units_d128_nomask", 1, 2, 8192, 128, "bf16", 128, 64, 1, False),
+    # shapes served by the tensor-core hash: ragged 128-row tiles, 1..4 column chunks per round
+    ("tc_hash_d64_nb2048", 1, 2, 1000, 64, "bf16", 2048, 8, 2, True),
+    ("tc_hash_d128_nb128_ragged", 2, 3, 200, 128, "bf16", 128, 8, 3, True),
+    ("tc_hash_d128_nb1024", 1, 1, 4096, 128, "bf16", 1024, 64, 2, True),
+    ("tc_hash_d64_nb512_many_rounds", 1, 1, 1024, 64, "bf16", 512, 64, 9, True),
 ]
 
 
@@ -99,6 +104,29 @@ def test_zero_rows_and_custom_scale():
     assert res["near_tie"].cpu()[0, 0, :, 5].tolist() == [1, 1]
     # the two planted zero rows are near ties in both rounds: 4 of 512 hashes
     full_parity(w, qk, v, R, scale=0.3, max_flag_frac=4 / 512 + 1e-3)
+
+
+@pytest.mark.parametrize("nb", [16, 256])
+def test_zero_rows_get_bucket_zero(nb):
+    """A zero row has p = 0 everywhere: bucket 0 (first maximum), flagged as a near tie."""
+    w = synth.small_workload("zero_nb", 1, 2, 256, 128, "bf16", nb, 64, 2)
+    qk, v, R = synth.make_inputs(w, seed=8)
+    qk[0, 1, 0] = 0
+    qk[0, 0, 131] = 0
+    b, f = lsh.lsh_hash(qk.to(DEV), R.to(DEV), nb)
+    b, f = b.cpu(), f.cpu()
+    assert b[0, 1, :, 0].tolist() == [0, 0] and b[0, 0, :, 131].tolist() == [0, 0]
+    assert f[0, 1, :, 0].tolist() == [1, 1] and f[0, 0, :, 131].tolist() == [1, 1]
+
+
+def test_hash_with_and_without_flags_agree():
+    """The near-tie output is optional; the buckets must not depend on asking for it."""
+    for nb in (32, 256, 1024):
+        w = synth.small_workload("flags", 2, 2, 1536, 128, "bf16", nb, 64, 3)
+        qk, v, R = synth.make_inputs(w, seed=nb)
+        b1, f1 = lsh.lsh_hash(qk.to(DEV), R.to(DEV), nb)
+        b2, f2 = lsh.lsh_hash(qk.to(DEV), R.to(DEV), nb, with_near_tie=False)
+        assert f2 is None and torch.equal(b1, b2)
 
 
 def test_fp32_output_from_bf16_input():

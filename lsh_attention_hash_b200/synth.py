@@ -55,6 +55,9 @@ WORKLOADS = {
     "skewed16k": Workload("skewed16k", 8, 8, 16384, 128, "bf16", 256, 64, 4, qk_kind="clusters"),
     # 8 x 8 x 65536 x 128 bf16, 1024 buckets, 8 rounds (64K char-LM shaped)
     "64k": Workload("64k", 8, 8, 65536, 128, "bf16", 1024, 64, 8),
+    # 8 x 8 x 16384 x 128 bf16, 256 buckets, 8 rounds: the 64K workload at a quarter of the
+    # length (profiling captures: inputs still larger than L2, a few GB on the device)
+    "16k": Workload("16k", 8, 8, 16384, 128, "bf16", 256, 64, 8),
     # 1 x 8 x 1048576 x 64 bf16, 16384 buckets, 4 rounds
     "1m": Workload("1m", 1, 8, 1048576, 64, "bf16", 16384, 64, 4),
 }

@@ -14,18 +14,26 @@
 //   S[128 x 192] = Q K^T        two UMMAs (N = 64 for chunk 2j-1, N = 128 for
 //                                the pair itself, whose rows are also Q)
 //   row r sees keys [64*(r>=64), 64*(r>=64) + 128); its own key is 64 + r%64
-//   P = exp2(S * s_j - max) in bf16, written back over S in TMEM
-//   O[128 x D] = P V            UMMA with A = P from TMEM, B = V (MN-major)
+//   P = exp2(S * s_j - max) in bf16, written back over the head of S in TMEM
+//   O[128 x D] = P V            UMMA with A = P from TMEM, B = V (MN-major),
+//                                accumulated behind P in the same TMEM buffer
 // and the rows go back to their original positions perm[s].
 //
-// Warp roles (192 threads, persistent CTAs, one per SM):
-//   warp 0     producer: reads perm, gathers the QK and V rows of each chunk
-//              with TMA tile::gather4 (128-byte swizzled, K-major) into a ring
-//              of three 128-row slots;
-//   warp 1     TMEM owner and single-thread UMMA issuer;
-//   warps 2-5  one query row per thread: key lengths, softmax, P, epilogue.
-// TMEM: two S/P buffers of 192 columns and one O buffer (512 columns).
-// Every wait is bounded (tc::mbar_wait); a timeout unwinds the CTA cleanly.
+// Warp roles (384 threads, persistent CTAs, one per SM):
+//   warps 0-1  producers: read perm and gather the QK and V rows of each chunk
+//              with 16-byte cp.async copies (32 lanes generate addresses in
+//              parallel; many small TMA row gathers were issue-bound) straight
+//              into 128-byte-swizzled K-major UMMA tiles, in a ring of three
+//              128-row slots;
+//   warp 2     TMEM owner and single-thread UMMA issuer; it never blocks on
+//              one step while another step's UMMA could go (S of step t+1 and
+//              PV of step t are issued in whichever order they become ready);
+//   warp 3     key multipliers scale * log2(e) / ||k|| of every gathered row;
+//   warps 4-7  softmax + epilogue of the even steps, warps 8-11 of the odd
+//              steps (one query row per thread), so that one step's softmax
+//              overlaps the other step's UMMAs, loads and stores.
+// TMEM: two step buffers of 256 columns (S: 192 fp32, P: first 96, O: 96..96+D).
+// Every wait is bounded; a timeout unwinds the CTA cleanly.
 #pragma once
 
 #include "tc_common.cuh"
@@ -36,10 +44,10 @@ namespace att_tc {
 constexpr int kC = 64;         // chunk length served
 constexpr int kRows = 128;     // query rows per step
 constexpr int kSlots = 3;      // 128-row slots in the shared-memory ring
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCols = 192;  // one S/P buffer
-constexpr uint32_t kOCol = 2 * kSCols;
+constexpr uint32_t kBufCols = 256;  // one step buffer
+constexpr uint32_t kOOff = 96;      // O columns inside a step buffer
 
 template <int D>
 struct Layout {
@@ -51,8 +59,8 @@ struct Layout {
   static constexpr uint32_t kPerm = 2 * kSlots * kSlotBytes;        // int32 [kSlots][128]
   static constexpr uint32_t kColMul = kPerm + kSlots * kRows * 4;   // float [kSlots][128]
   static constexpr uint32_t kBar = kColMul + kSlots * kRows * 4;
-  // full[3] empty[3] s_full[2] p_ready[2] o_full o_empty cm_ready done
-  static constexpr int kNumBars = 14;
+  // full[3] empty[3] cm_full[3] s_full[2] p_ready[2] o_full[2] buf_empty[2] done
+  static constexpr int kNumBars = 18;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;   // tmem base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;         // slack for 1024-byte alignment
@@ -71,7 +79,10 @@ struct Params {
   long long n_units;
   int self_mask;
   float colscale;        // logit scale * log2(e)
-  int sorted_input;      // rows of the tensor maps are [seg][slot] instead of [bh][pos]
+  int sorted_input;      // rows are [seg][slot] of the sorted copies instead of [bh][pos]
+  const uint8_t* qk;     // row sources (qk / v, or their sorted copies)
+  const uint8_t* v;
+  int out_v8;            // output rows 32-byte aligned: 32-byte stores
 };
 
 // Warp-uniform bounded wait: every lane acquires the phase itself, lane 0
@@ -110,57 +121,152 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-struct Unit {
+// Walks this CTA's steps in order.  A work unit is a run of consecutive steps
+// of one (b, h, round) segment; each unit starts with one fill holding the
+// chunk before its first pair, then one fill per step.  f is the fill index of
+// the step's own pair; the previous chunk is always in fill f - 1.
+struct StepIter {
+  long long u;
   long long seg;
-  int j0, j1;
+  int j, j1;
+  uint32_t f;   // fill of the step's pair
+  uint32_t t;   // step counter of this CTA
+  bool valid;
+
+  __device__ __forceinline__ void load_unit(const Params& p) {
+    valid = u < p.n_units;
+    if (!valid) return;
+    seg = u / p.units_per_seg;
+    j = (int)(u - seg * p.units_per_seg) * p.run;
+    j1 = min(j + p.run, p.n_steps);
+  }
+  __device__ __forceinline__ void init(const Params& p) {
+    u = blockIdx.x;
+    f = 1;
+    t = 0;
+    load_unit(p);
+  }
+  __device__ __forceinline__ bool last_of_unit() const { return j + 1 >= j1; }
+  __device__ __forceinline__ void advance(const Params& p) {
+    ++t;
+    if (j + 1 < j1) {
+      ++j;
+      ++f;
+    } else {
+      u += gridDim.x;
+      f += 2;  // the next unit's leading fill, then its first pair
+      load_unit(p);
+    }
+  }
 };
 
-__device__ __forceinline__ Unit decode_unit(const Params& p, long long u) {
-  Unit w;
-  w.seg = u / p.units_per_seg;
-  const int run_i = (int)(u - w.seg * p.units_per_seg);
-  w.j0 = run_i * p.run;
-  w.j1 = min(w.j0 + p.run, p.n_steps);
-  return w;
+// One fill of the slot ring: `nrows` rows (64 or 128) starting at local row
+// `row0`; local rows [row0, row0+64) hold chunk cA, [row0+64, row0+128) chunk cB.
+struct Fill {
+  long long seg;
+  int row0, nrows, cA, cB;
+};
+
+// Walks the fills of this CTA in order: per unit one leading fill (the chunk
+// before the unit's first pair; chunk 0 again at a segment start, masked
+// later) and then one fill per step (odd tail: the last chunk repeated, rows
+// unused).
+struct FillIter {
+  long long u;
+  int j, j0, j1;
+  bool valid;
+  __device__ __forceinline__ void load_unit(const Params& p) {
+    valid = u < p.n_units;
+    if (!valid) return;
+    const long long seg = u / p.units_per_seg;
+    j0 = (int)(u - seg * p.units_per_seg) * p.run;
+    j1 = min(j0 + p.run, p.n_steps);
+    j = j0 - 1;
+  }
+  __device__ __forceinline__ void init(const Params& p) {
+    u = blockIdx.x;
+    load_unit(p);
+  }
+  __device__ __forceinline__ Fill get(const Params& p) const {
+    Fill f;
+    f.seg = u / p.units_per_seg;
+    if (j < j0) {
+      f.row0 = 64;
+      f.nrows = 64;
+      f.cA = f.cB = j0 > 0 ? 2 * j0 - 1 : 0;
+    } else {
+      f.row0 = 0;
+      f.nrows = 128;
+      f.cA = 2 * j;
+      f.cB = (2 * j + 1 < p.n_chunks) ? 2 * j + 1 : 2 * j;
+    }
+    return f;
+  }
+  __device__ __forceinline__ void advance(const Params& p) {
+    if (j + 1 < j1) {
+      ++j;
+    } else {
+      u += gridDim.x;
+      load_unit(p);
+    }
+  }
+};
+
+// Original positions of this lane's two rows of the producer warp's half of a
+// fill (global loads; issued one fill ahead so that their latency hides behind
+// the slot wait).  Producer warp pw owns local rows [64 pw, 64 pw + 64).
+__device__ __forceinline__ void fill_positions(const Params& p, const Fill& f, int pw, int (&pos)[2]) {
+  const int lane = threadIdx.x & 31;
+  const int32_t* pseg = p.perm + f.seg * p.L;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = 64 * pw + 32 * k + lane;  // local row of the slot
+    if (i >= f.row0 && i < f.row0 + f.nrows) {
+      const int chunk = (i - f.row0) < 64 ? f.cA : f.cB;
+      pos[k] = pseg[chunk * kC + (i & 63)];
+    }
+  }
 }
 
-// Loads `nrows` rows (64 or 128) of chunks (cA for local rows [row0, row0+64),
-// cB for [row0+64, row0+128)) into slot `slot`, rows starting at `row0`.
+// Gathers the producer warp's rows of a fill into slot `slot` with 16-byte
+// cp.async copies: row r of a 128 x 64-element half tile sits at r * 128 bytes
+// and its 16-byte piece c at ((c ^ (r % 8)) * 16), the 128-byte swizzle the
+// UMMA descriptors expect.  Every producer lane then arrives on `full_bar`
+// when its copies have landed.
 template <int D>
-__device__ __forceinline__ void producer_fill(const Params& p, const CUtensorMap* mqk, const CUtensorMap* mv,
-                                              uint8_t* smem, uint64_t* full_bar, int slot, long long seg,
-                                              int row0, int nrows, int cA, int cB) {
+__device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, uint64_t* full_bar, int slot,
+                                              const Fill& f, int pw, const int (&pos)[2]) {
   using Lay = Layout<D>;
+  constexpr int kPieces = D / 8;            // 16-byte pieces per row
+  constexpr int kRowsPerInst = 32 / kPieces;
   const int lane = threadIdx.x & 31;
   int32_t* perm_s = reinterpret_cast<int32_t*>(smem + Lay::kPerm) + slot * kRows;
-  const long long bh = seg / p.n_rounds;
-  const int32_t* pseg = p.perm + seg * p.L;
-  int grow[4];
-  const bool active = lane * 4 < nrows;
-  if (active) {
+  const long long bh = f.seg / p.n_rounds;
+  const int base = 64 * pw;
+  const bool mine = base + 64 > f.row0 && base < f.row0 + f.nrows;  // the fill covers this warp's rows
+  if (mine) {
+    long long grow[2];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int rr = row0 + lane * 4 + k;                 // local row in the slot
-      const int chunk = (rr - row0) < 64 ? cA : cB;
-      const int s = chunk * kC + (rr & 63);
-      const int pos = pseg[s];
-      perm_s[rr] = pos;
-      grow[k] = p.sorted_input ? (int)(seg * p.L + s) : (int)(bh * p.L + pos);
+    for (int k = 0; k < 2; ++k) {
+      const int i = base + 32 * k + lane;
+      const int chunk = (i - f.row0) < 64 ? f.cA : f.cB;
+      perm_s[i] = pos[k];
+      grow[k] = p.sorted_input ? f.seg * p.L + chunk * kC + (i & 63) : bh * p.L + pos[k];
+    }
+    const uint32_t qk_dst = tc::smem_u32(smem + Lay::kQK + slot * Lay::kSlotBytes);
+    const uint32_t v_dst = tc::smem_u32(smem + Lay::kV + slot * Lay::kSlotBytes);
+    const int c = lane % kPieces;
+#pragma unroll 4
+    for (int it = 0; it < 64 / kRowsPerInst; ++it) {
+      const int rl = it * kRowsPerInst + lane / kPieces;  // row within the warp's 64
+      const long long g = __shfl_sync(0xffffffffu, rl < 32 ? grow[0] : grow[1], rl & 31);
+      const int r = base + rl;
+      const uint32_t off = (c >> 3) * Lay::kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+      tc::cp_async16(qk_dst + off, p.qk + (g * D + c * 8) * 2);
+      tc::cp_async16(v_dst + off, p.v + (g * D + c * 8) * 2);
     }
   }
-  __syncwarp();
-  if (lane == 0) tc::mbar_arrive_expect_tx(full_bar, (uint32_t)(nrows * D * 2 * 2));
-  __syncwarp();
-  if (active) {
-    const int rr = row0 + lane * 4;
-#pragma unroll
-    for (int h = 0; h < Lay::kHalves; ++h) {
-      uint8_t* dq = smem + Lay::kQK + slot * Lay::kSlotBytes + h * Lay::kHalfBytes + rr * 128;
-      uint8_t* dv = smem + Lay::kV + slot * Lay::kSlotBytes + h * Lay::kHalfBytes + rr * 128;
-      tc::tma_gather4(dq, mqk, full_bar, h * 64, grow[0], grow[1], grow[2], grow[3]);
-      tc::tma_gather4(dv, mv, full_bar, h * 64, grow[0], grow[1], grow[2], grow[3]);
-    }
-  }
+  tc::cp_async_arrive(full_bar);
 }
 
 // scale * log2(e) / ||row||, read from the swizzled row of a QK slot (the
@@ -185,20 +291,19 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
 
 template <int D, typename TO>
 __global__ void __launch_bounds__(kThreads, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap map_qk, const __grid_constant__ CUtensorMap map_v,
-                 const Params p) {
+attend_tc_kernel(const Params p) {
   using Lay = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
-  uint64_t* full = bars;          // [3] slot filled (TMA bytes landed)
-  uint64_t* empty = bars + 3;     // [3] slot released by the MMAs
-  uint64_t* s_full = bars + 6;    // [2] S buffer computed
-  uint64_t* p_ready = bars + 8;   // [2] P buffer written (128 arrivals)
-  uint64_t* o_full = bars + 10;   // O computed
-  uint64_t* o_empty = bars + 11;  // O read (128 arrivals)
-  uint64_t* cm_ready = bars + 12; // key multipliers of the step written (128 arrivals)
-  uint64_t* done_bar = bars + 13; // all MMAs retired
+  uint64_t* full = bars;            // [3] slot filled (64 producer lanes' copies landed)
+  uint64_t* empty = bars + 3;       // [3] slot released by the UMMAs
+  uint64_t* cm_full = bars + 6;     // [3] key multipliers of the slot's fill written (32 arrivals)
+  uint64_t* s_full = bars + 9;      // [2] S of the step buffer computed
+  uint64_t* p_ready = bars + 11;    // [2] P written (128 arrivals)
+  uint64_t* o_full = bars + 13;     // [2] O computed
+  uint64_t* buf_empty = bars + 15;  // [2] O read (128 arrivals)
+  uint64_t* done_bar = bars + 17;   // all UMMAs retired
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
   float* colmul = reinterpret_cast<float*>(smem + Lay::kColMul);
@@ -207,59 +312,51 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_qk, const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
-      tc::mbar_init(&full[i], 1);
+      tc::mbar_init(&full[i], 64);
       tc::mbar_init(&empty[i], 1);
+      tc::mbar_init(&cm_full[i], 32);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&s_full[i], 1);
       tc::mbar_init(&p_ready[i], 128);
+      tc::mbar_init(&o_full[i], 1);
+      tc::mbar_init(&buf_empty[i], 128);
     }
-    tc::mbar_init(o_full, 1);
-    tc::mbar_init(o_empty, 128);
-    tc::mbar_init(cm_ready, 128);
     tc::mbar_init(done_bar, 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tc::prefetch_tensormap(&map_qk);
-    tc::prefetch_tensormap(&map_v);
-  }
-  if (warp == 1) tc::tmem_alloc(tmem_holder, kTmemCols);
+  if (warp == 2) tc::tmem_alloc(tmem_holder, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp < 2) {
+    // ------------------------------------------------------------ producers
+    const int pw = warp;
     uint32_t f = 0;
-    bool ok = true;
-    for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit w = decode_unit(p, u);
-      {  // the chunk before the unit's first pair (chunk 0 again at the segment start: masked)
-        const int slot = f % kSlots;
-        ok = warp_wait(&empty[slot], ((f / kSlots) & 1) ^ 1, abort_flag);
-        if (!ok) break;
-        const int cp = w.j0 > 0 ? 2 * w.j0 - 1 : 0;
-        producer_fill<D>(p, &map_qk, &map_v, smem, &full[slot], slot, w.seg, 64, 64, cp, cp);
-        ++f;
-      }
-      for (int j = w.j0; j < w.j1; ++j) {
-        const int slot = f % kSlots;
-        ok = warp_wait(&empty[slot], ((f / kSlots) & 1) ^ 1, abort_flag);
-        if (!ok) break;
-        const int c0 = 2 * j;
-        const int c1 = (2 * j + 1 < p.n_chunks) ? 2 * j + 1 : 2 * j;  // odd tail: repeat (rows unused)
-        producer_fill<D>(p, &map_qk, &map_v, smem, &full[slot], slot, w.seg, 0, 128, c0, c1);
-        ++f;
-      }
+    FillIter fi;
+    fi.init(p);
+    int pos[2] = {0, 0};
+    if (fi.valid) fill_positions(p, fi.get(p), pw, pos);
+    while (fi.valid) {
+      const Fill cur = fi.get(p);
+      FillIter nx = fi;
+      nx.advance(p);
+      int npos[2] = {0, 0};
+      if (nx.valid) fill_positions(p, nx.get(p), pw, npos);  // next fill's positions, in flight during the wait
+      const int slot = f % kSlots;
+      if (!warp_wait(&empty[slot], ((f / kSlots) & 1) ^ 1, abort_flag)) break;
+      producer_fill<D>(p, smem, &full[slot], slot, cur, pw, pos);
+      ++f;
+      fi = nx;
+      pos[0] = npos[0];
+      pos[1] = npos[1];
     }
     // never leave with copies in flight
-    if (lane == 0) {
-      for (uint32_t k = (f > kSlots ? f - kSlots : 0); k < f; ++k) drain_wait(&full[k % kSlots], (k / kSlots) & 1);
-    }
-  } else if (warp == 1) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 2) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       const uint32_t id_prev = tc::idesc_bf16_f32(128, 64, 0, 0);
@@ -267,177 +364,214 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_qk, const __grid_consta
       const uint32_t id_pv = tc::idesc_bf16_f32(128, D, 0, 1);
       const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK);
       const uint32_t v0 = tc::smem_u32(smem + Lay::kV);
-      uint32_t f = 0, t = 0;
-      bool ok = true;
-      for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(p, u);
-        ++f;  // the unit's leading chunk fill
-        for (int j = w.j0; j < w.j1; ++j) {
-          const uint32_t fp = f - 1, fc = f;
-          ++f;
-          const int sp = fp % kSlots, sc = fc % kSlots;
-          ok = tc::mbar_wait(&full[sp], (fp / kSlots) & 1, abort_flag) &&
-               tc::mbar_wait(&full[sc], (fc / kSlots) & 1, abort_flag);
-          if (!ok) break;
-          tc::tc_fence_after();
-          const uint32_t sbuf = tmem + (t & 1) * kSCols;
-          const uint32_t qk_c = qk0 + sc * Lay::kSlotBytes;
-          const uint32_t qk_p = qk0 + sp * Lay::kSlotBytes + 64 * 128;  // rows 64..127 of the previous slot
+      StepIter si, pi;  // next step to receive S, next step to receive PV
+      si.init(p);
+      pi.init(p);
+      unsigned long long t_idle = 0;
+      while (pi.valid) {
+        bool progress = false;
+        if (si.valid && si.t < pi.t + 2) {
+          const uint32_t fp = si.f - 1, fc = si.f;
+          if (tc::mbar_try_wait(&full[fp % kSlots], (fp / kSlots) & 1) &&
+              tc::mbar_try_wait(&full[fc % kSlots], (fc / kSlots) & 1) &&
+              tc::mbar_try_wait(&buf_empty[si.t & 1], ((si.t >> 1) & 1) ^ 1)) {
+            tc::tc_fence_after();
+            const uint32_t sbuf = tmem + (si.t & 1) * kBufCols;
+            const uint32_t qk_c = qk0 + (fc % kSlots) * Lay::kSlotBytes;
+            const uint32_t qk_p = qk0 + (fp % kSlots) * Lay::kSlotBytes + 64 * 128;  // rows 64..127
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * Lay::kHalfBytes + (kk & 3) * 32;
-            const uint64_t a = tc::sdesc_sw128(qk_c + koff, 16, 1024);
-            const uint64_t bp = tc::sdesc_sw128(qk_p + koff, 16, 1024);
-            tc::umma_ss(sbuf, a, bp, id_prev, kk > 0);
-            tc::umma_ss(sbuf + 64, a, a, id_pair, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t koff = (kk >> 2) * Lay::kHalfBytes + (kk & 3) * 32;
+              const uint64_t a = tc::sdesc_sw128(qk_c + koff, 16, 1024);
+              const uint64_t bp = tc::sdesc_sw128(qk_p + koff, 16, 1024);
+              tc::umma_ss(sbuf, a, bp, id_prev, kk > 0);
+              tc::umma_ss(sbuf + 64, a, a, id_pair, kk > 0);
+            }
+            tc::umma_commit(&s_full[si.t & 1]);
+            si.advance(p);
+            progress = true;
           }
-          tc::umma_commit(&s_full[t & 1]);
-          ok = tc::mbar_wait(&p_ready[t & 1], (t >> 1) & 1, abort_flag) &&
-               tc::mbar_wait(o_empty, (t & 1) ^ 1, abort_flag);
-          if (!ok) break;
+        }
+        if (pi.t < si.t && tc::mbar_try_wait(&p_ready[pi.t & 1], (pi.t >> 1) & 1)) {
           tc::tc_fence_after();
+          const uint32_t sbuf = tmem + (pi.t & 1) * kBufCols;
+          const uint32_t sp = (pi.f - 1) % kSlots, sc = pi.f % kSlots;
 #pragma unroll
           for (int kk = 0; kk < 12; ++kk) {
             const uint32_t vrow = kk < 4 ? v0 + sp * Lay::kSlotBytes + (64 + 16 * kk) * 128
                                          : v0 + sc * Lay::kSlotBytes + (16 * (kk - 4)) * 128;
             const uint64_t b = tc::sdesc_sw128(vrow, Lay::kHalfBytes, 1024);
-            tc::umma_ts(tmem + kOCol, sbuf + kk * 8, b, id_pv, kk > 0);
+            tc::umma_ts(sbuf + kOOff, sbuf + kk * 8, b, id_pv, kk > 0);
           }
-          tc::umma_commit(o_full);
+          tc::umma_commit(&o_full[pi.t & 1]);
           tc::umma_commit(&empty[sp]);
-          ++t;
+          if (pi.last_of_unit()) tc::umma_commit(&empty[sc]);
+          pi.advance(p);
+          progress = true;
         }
-        if (!ok) break;
-        tc::umma_commit(&empty[(f - 1) % kSlots]);
+        if (progress) {
+          t_idle = 0;
+        } else {
+          const unsigned long long now = tc::globaltimer();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > tc::kWaitNs || *abort_flag) {
+            if (!*abort_flag) record_error(LSH_ERR_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+        }
       }
       tc::umma_commit(done_bar);
       drain_wait(done_bar, 0);
     }
     __syncwarp();
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ key multipliers
+    uint32_t f = 0;
+    FillIter fi;
+    fi.init(p);
+    while (fi.valid) {
+      const Fill cur = fi.get(p);
+      const int slot = f % kSlots;
+      if (!warp_wait(&full[slot], (f / kSlots) & 1, abort_flag)) break;
+      const uint8_t* qs = smem + Lay::kQK + slot * Lay::kSlotBytes;
+      for (int i = cur.row0 + lane; i < cur.row0 + cur.nrows; i += 32)
+        colmul[slot * kRows + i] = row_colmul<D>(qs, i, p.colscale);
+      tc::mbar_arrive(&cm_full[slot]);
+      ++f;
+      fi.advance(p);
+    }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    const int wg = (warp - 4) >> 2;      // 0: even steps, 1: odd steps
     const int q = warp & 3;              // TMEM lane quarter of this warp
     const int r = q * 32 + lane;         // query row of the step
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const bool low = q < 2;              // rows 0..63: keys [0, 128); rows 64..127: keys [64, 192)
     const int self_i = 64 + (r & 63);    // own key, as an index into the row's 128 keys
-    uint32_t f = 0, t = 0;
+    StepIter it;
+    it.init(p);
+    if (wg == 1) it.advance(p);
     bool ok = true;
-    for (long long u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit w = decode_unit(p, u);
-      ++f;
-      bool first = true;
-      for (int j = w.j0; j < w.j1; ++j) {
-        const uint32_t fp = f - 1, fc = f;
-        ++f;
-        const int sp = fp % kSlots, sc = fc % kSlots;
-        ok = warp_wait(&full[sp], (fp / kSlots) & 1, abort_flag) &&
-             warp_wait(&full[sc], (fc / kSlots) & 1, abort_flag);
-        if (!ok) break;
-        // key multipliers of the pair (and, at a unit start, of the leading chunk)
-        colmul[sc * kRows + r] = row_colmul<D>(smem + Lay::kQK + sc * Lay::kSlotBytes, r, p.colscale);
-        if (first && !low)
-          colmul[sp * kRows + r] = row_colmul<D>(smem + Lay::kQK + sp * Lay::kSlotBytes, r, p.colscale);
-        tc::mbar_arrive(cm_ready);
-        const int chunk = 2 * j + (low ? 0 : 1);
-        const bool valid = chunk < p.n_chunks;
-        const int pos = perm_s[sc * kRows + r];
-        ok = warp_wait(cm_ready, t & 1, abort_flag) && warp_wait(&s_full[t & 1], (t >> 1) & 1, abort_flag);
-        if (!ok) break;
-        tc::tc_fence_after();
-        const uint32_t sbuf = tmem + (t & 1) * kSCols;
-        float x[128];
-        {
-          uint32_t raw[32];
+    while (it.valid) {
+      const uint32_t t = it.t, b = t & 1;
+      const uint32_t fp = it.f - 1, fc = it.f;
+      const int sp = fp % kSlots, sc = fc % kSlots;
+      ok = warp_wait(&cm_full[sp], (fp / kSlots) & 1, abort_flag) &&
+           warp_wait(&cm_full[sc], (fc / kSlots) & 1, abort_flag) &&
+           warp_wait(&s_full[b], (t >> 1) & 1, abort_flag);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const int chunk = 2 * it.j + (low ? 0 : 1);
+      const bool valid = chunk < p.n_chunks;
+      const int pos = perm_s[sc * kRows + r];
+      const uint32_t sbuf = lane_base + tmem + b * kBufCols;
+      const uint32_t scol = low ? 0 : 64;  // S column of the row's first key
+      const float* cm_lo = low ? colmul + sp * kRows + 64 : colmul + sc * kRows;  // keys 0..63 of the row
+      const float* cm_hi = low ? colmul + sc * kRows : colmul + sc * kRows + 64;  // keys 64..127
+      const int g_first = (low && it.j == 0) ? 2 : 0;  // chunk 0 has no previous chunk
+      // pass 1: row maximum of the scaled logits (log2 domain)
+      float m = -INFINITY;
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            tc::tmem_ld32(lane_base + sbuf + (low ? 0 : 64) + 32 * g, raw);
-            tc::tmem_wait_ld();
+      for (int g = 0; g < 4; ++g) {
+        uint32_t raw[32];
+        tc::tmem_ld32(sbuf + scol + 32 * g, raw);
+        tc::tmem_wait_ld();
+        if (g < g_first) continue;
+        const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[32 * g + e] = __uint_as_float(raw[e]);
-          }
-        }
-        // multipliers: local key i -> low rows: i < 64 prev slot rows 64+i, else pair rows i-64;
-        //                              high rows: pair rows i
-        const float* cm_lo = low ? colmul + sp * kRows + 64 : colmul + sc * kRows;
-        const float* cm_hi = low ? colmul + sc * kRows : colmul + sc * kRows + 64;
-        const bool mask_prev = low && j == 0;  // chunk 0 has no previous chunk
-        float m = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          float v = x[i] * (i < 64 ? cm_lo[i] : cm_hi[i - 64]);
-          if ((p.self_mask && i == self_i) || (mask_prev && i < 64)) v = -INFINITY;
-          x[i] = v;
+        for (int e = 0; e < 32; ++e) {
+          float v = __uint_as_float(raw[e]) * cm[e];
+          if (p.self_mask && 32 * g + e == self_i) v = -INFINITY;
           m = fmaxf(m, v);
         }
-        float l = 0.f;
-        uint32_t pk[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float a = tc::ex2_approx(x[2 * i] - m);
-          const float b = tc::ex2_approx(x[2 * i + 1] - m);
-          l += a + b;
-          pk[i] = tc::pack_bf16x2(a, b);
-        }
-        {
-          uint32_t g0[32], g1[32], z[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            g0[e] = pk[e];
-            g1[e] = pk[32 + e];
-            z[e] = 0u;
-          }
-          if (low) {
-            tc::tmem_st32(lane_base + sbuf + 0, g0);
-            tc::tmem_st32(lane_base + sbuf + 32, g1);
-            tc::tmem_st32(lane_base + sbuf + 64, z);
-          } else {
-            tc::tmem_st32(lane_base + sbuf + 0, z);
-            tc::tmem_st32(lane_base + sbuf + 32, g0);
-            tc::tmem_st32(lane_base + sbuf + 64, g1);
-          }
-          tc::tmem_wait_st();
-        }
-        tc::tc_fence_before();
-        tc::mbar_arrive(&p_ready[t & 1]);
-        // epilogue: O row -> original position
-        ok = warp_wait(o_full, t & 1, abort_flag);
-        if (!ok) break;
-        tc::tc_fence_after();
-        float o[D];
-        {
-          uint32_t raw[32];
-#pragma unroll
-          for (int g = 0; g < D / 32; ++g) {
-            tc::tmem_ld32(lane_base + tmem + kOCol + 32 * g, raw);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[32 * g + e] = __uint_as_float(raw[e]);
-          }
-        }
-        tc::tc_fence_before();
-        tc::mbar_arrive(o_empty);
-        if (valid) {
-          const float inv_l = 1.f / l;
-          TO* dst = reinterpret_cast<TO*>(p.out) + (w.seg * p.L + pos) * (long long)D;
-#pragma unroll
-          for (int e = 0; e < D; e += 8) {
-            float y[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) y[k] = o[e + k] * inv_l;
-            store8(dst + e, y);
-          }
-          p.lse[w.seg * p.L + pos] = (m + __log2f(l)) * 0.6931471805599453f;
-        }
-        ++t;
-        first = false;
       }
+      // pass 2: P = exp2(x - m) in bf16 over the head of the buffer, row sum
+      float l = 0.f;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint32_t raw[32];
+        tc::tmem_ld32(sbuf + scol + 32 * g, raw);
+        tc::tmem_wait_ld();
+        const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
+        const bool dead = g < g_first;
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float v0 = __uint_as_float(raw[e]) * cm[e];
+          float v1 = __uint_as_float(raw[e + 1]) * cm[e + 1];
+          if (p.self_mask && 32 * g + e == self_i) v0 = -INFINITY;
+          if (p.self_mask && 32 * g + e + 1 == self_i) v1 = -INFINITY;
+          const float a = dead ? 0.f : tc::ex2_approx(v0 - m);
+          const float c = dead ? 0.f : tc::ex2_approx(v1 - m);
+          l += a + c;
+          pk[e >> 1] = tc::pack_bf16x2(a, c);
+        }
+        tc::tmem_st16(sbuf + (low ? 16 * g : 32 + 16 * g), pk);
+      }
+      {
+        uint32_t z[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) z[e] = 0u;
+        tc::tmem_st32(sbuf + (low ? 64 : 0), z);
+      }
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(&p_ready[b]);
+      // epilogue: O row -> original position
+      ok = warp_wait(&o_full[b], (t >> 1) & 1, abort_flag);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const float inv_l = 1.f / l;
+      TO* dst = reinterpret_cast<TO*>(p.out) + (it.seg * p.L + pos) * (long long)D;
+#pragma unroll
+      for (int g = 0; g < D / 32; ++g) {
+        uint32_t raw[32];
+        tc::tmem_ld32(sbuf + kOOff + 32 * g, raw);
+        tc::tmem_wait_ld();
+        if (g == D / 32 - 1) {
+          tc::tc_fence_before();
+          tc::mbar_arrive(&buf_empty[b]);
+        }
+        if (valid) {
+          if (sizeof(TO) == 2 && p.out_v8) {  // 32 bf16 = two 32-byte stores
+#pragma unroll
+            for (int e = 0; e < 32; e += 16) {
+              uint32_t w[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                w[k] = tc::pack_bf16x2(__uint_as_float(raw[e + 2 * k]) * inv_l, __uint_as_float(raw[e + 2 * k + 1]) * inv_l);
+              tc::st_global_v8(dst + 32 * g + e, w);
+            }
+          } else if (sizeof(TO) == 4 && p.out_v8) {  // 32 floats = four 32-byte stores
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t w[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) w[k] = __float_as_uint(__uint_as_float(raw[e + k]) * inv_l);
+              tc::st_global_v8(dst + 32 * g + e, w);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              float y[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) y[k] = __uint_as_float(raw[e + k]) * inv_l;
+              store8(dst + 32 * g + e, y);
+            }
+          }
+        }
+      }
+      if (valid) p.lse[it.seg * p.L + pos] = (m + __log2f(l)) * 0.6931471805599453f;
+      it.advance(p);
+      if (it.valid) it.advance(p);
     }
   }
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 2) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }

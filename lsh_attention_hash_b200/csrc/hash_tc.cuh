@@ -19,6 +19,11 @@
 // position (ties prefer the lower column); a max tree over the raw values of
 // the winning group tells its sign.  The exact top-two |p| for the near-tie
 // flag are tracked only when that output is requested.
+//
+// Warps: 0 TMA producer, 1 UMMA issuer, 2-9 epilogue.  Two epilogue warps
+// share each TMEM lane quarter (32 rows) and take one half of the columns of
+// every accumulator chunk each; at the end of a tile the second half's row
+// states go through shared memory to the first half, which merges and stores.
 #pragma once
 
 #include "tc_common.cuh"
@@ -26,7 +31,7 @@
 namespace lsh {
 namespace hash_tc {
 
-constexpr int kThreads = 192;  // warp 0 TMA, warp 1 UMMA, warps 2-5 epilogue
+constexpr int kThreads = 320;  // warp 0 TMA, warp 1 UMMA, warps 2-9 epilogue
 constexpr int kRows = 128;
 constexpr int kStages = 2;
 
@@ -37,9 +42,11 @@ struct Layout {
   static constexpr uint32_t kA = 0;
   static constexpr uint32_t kR = kStages * kStageBytes;          // R[round]: (half/64) boxes of D x 128 B
   __host__ __device__ static constexpr uint32_t bar_off(int half) { return kR + (uint32_t)D * half * 2; }
-  // a_full[2] a_empty[2] acc_full[2] acc_empty[2] r_full done
-  static constexpr int kNumBars = 10;
-  __host__ __device__ static constexpr uint32_t smem_bytes(int half) { return bar_off(half) + kNumBars * 8 + 16 + 1024; }
+  // a_full[2] a_empty[2] acc_full[2] acc_empty[2] r_full done half_done[2] merged[2]
+  static constexpr int kNumBars = 14;
+  // second-half row states: [2 tile parities][5 fields][128 rows] x 4 B
+  __host__ __device__ static constexpr uint32_t xchg_off(int half) { return bar_off(half) + kNumBars * 8 + 16; }
+  __host__ __device__ static constexpr uint32_t smem_bytes(int half) { return xchg_off(half) + 2 * 5 * kRows * 4 + 1024; }
 };
 
 struct Params {
@@ -112,6 +119,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   uint64_t* acc_empty = bars + 6;
   uint64_t* r_full = bars + 8;
   uint64_t* done_bar = bars + 9;
+  uint64_t* half_done = bars + 10;  // [2] second-half states written (128 arrivals)
+  uint64_t* merged = bars + 12;     // [2] second-half states consumed (128 arrivals)
+  float* xchg = reinterpret_cast<float*>(smem + Lay::xchg_off(p.half));
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + Lay::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + Lay::kNumBars) + 1;
 
@@ -123,7 +133,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       tc::mbar_init(&a_full[i], 1);
       tc::mbar_init(&a_empty[i], 1);
       tc::mbar_init(&acc_full[i], 1);
-      tc::mbar_init(&acc_empty[i], 128);
+      tc::mbar_init(&acc_empty[i], 256);
+      tc::mbar_init(&half_done[i], 128);
+      tc::mbar_init(&merged[i], 128);
     }
     tc::mbar_init(r_full, 1);
     tc::mbar_init(done_bar, 1);
@@ -203,11 +215,12 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     __syncwarp();
   } else {
     const int q = warp & 3;
+    const int ch = (warp - 2) >> 2;      // column half of every chunk
     const int r = q * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    uint32_t seq = 0;
+    uint32_t seq = 0, it = 0;
     bool ok = true;
-    for (long long tile = first_tile; ok && tile < p.n_tiles; tile += p.per_round) {
+    for (long long tile = first_tile; ok && tile < p.n_tiles; tile += p.per_round, ++it) {
       RowState st{-1.f, 0, 0.f, -INFINITY, -INFINITY};
       for (int c = 0; c < p.nchunks; ++c, ++seq) {
         const int b = seq & 1;
@@ -215,11 +228,12 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int piece = 0; piece < NC / 32; ++piece) {
+        for (int piece = 0; piece < NC / 64; ++piece) {
           uint32_t raw[32];
-          tc::tmem_ld32(lane_base + tmem + b * NC + piece * 32, raw);
+          const int col = ch * (NC / 2) + piece * 32;
+          tc::tmem_ld32(lane_base + tmem + b * NC + col, raw);
           tc::tmem_wait_ld();
-          const int g = c * (NC / 16) + piece * 2;
+          const int g = (c * NC + col) >> 4;
           process16<FLAG>(st, raw, g);
           process16<FLAG>(st, raw + 16, g + 1);
         }
@@ -227,6 +241,36 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         tc::mbar_arrive(&acc_empty[b]);
       }
       if (!ok) break;
+      const int tp = it & 1;
+      float* xs = xchg + tp * 5 * kRows;
+      if (ch == 1) {
+        ok = att_tc::warp_wait(&merged[tp], ((it >> 1) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        xs[r] = st.best_key;
+        xs[kRows + r] = __int_as_float(st.best_g);
+        xs[2 * kRows + r] = st.best_raw;
+        xs[3 * kRows + r] = st.v1;
+        xs[4 * kRows + r] = st.v2;
+        tc::mbar_arrive(&half_done[tp]);
+        continue;
+      }
+      ok = att_tc::warp_wait(&half_done[tp], (it >> 1) & 1, abort_flag);
+      if (!ok) break;
+      const float ok_key = xs[r];
+      const int o_g = __float_as_int(xs[kRows + r]);
+      const float o_raw = xs[2 * kRows + r];
+      const float o_v1 = xs[3 * kRows + r], o_v2 = xs[4 * kRows + r];
+      tc::mbar_arrive(&merged[tp]);
+      // the two halves cover disjoint groups; on equal keys the lower group wins
+      if (ok_key > st.best_key || (ok_key == st.best_key && o_g < st.best_g)) {
+        st.best_key = ok_key;
+        st.best_g = o_g;
+        st.best_raw = o_raw;
+      }
+      if (FLAG) {
+        st.v2 = fmaxf(fmaxf(st.v2, o_v2), fminf(st.v1, o_v1));
+        st.v1 = fmaxf(st.v1, o_v1);
+      }
       const long long row = tile * kRows + r;
       if (row < p.nrows) {
         const uint32_t kb = __float_as_uint(st.best_key);

@@ -82,20 +82,6 @@ inline EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// 2D bf16 view [rows, D] whose box is one row of 64 elements (128 B), 128-byte
-// swizzle: the source of tile::gather4 row gathers.
-inline bool make_row_gather_map(CUtensorMap* map, const void* base, long long rows, int D) {
-  EncodeTiledFn enc = encode_tiled();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // 2D bf16 view [rows, cols] with a box of box_cols x box_rows, 128-byte swizzle.
 inline bool make_tile_map(CUtensorMap* map, const void* base, long long rows, long long cols, int box_cols,
                           int box_rows) {
@@ -165,11 +151,6 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
   using namespace lsh::att_tc;
   const long long segs = (long long)B * H * n_rounds;
   const bool sorted = qk_sorted != nullptr;
-  CUtensorMap mqk, mv;
-  const long long rows = sorted ? segs * L : (long long)B * H * L;
-  if (!make_row_gather_map(&mqk, sorted ? qk_sorted : qk, rows, D) ||
-      !make_row_gather_map(&mv, sorted ? v_sorted : v, rows, D))
-    return LSH_ERR_CUDA;
   Params p;
   p.perm = perm;
   p.out = out;
@@ -184,12 +165,15 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
   p.self_mask = self_mask;
   p.colscale = scale * 1.4426950408889634f;  // log2(e)
   p.sorted_input = sorted ? 1 : 0;
+  p.qk = (const uint8_t*)(sorted ? qk_sorted : qk);
+  p.v = (const uint8_t*)(sorted ? v_sorted : v);
+  p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   const unsigned grid = (unsigned)std::min<long long>(p.n_units, sms);
   auto kfn = attend_tc_kernel<D, TO>;
   const int smem = (int)Layout<D>::kSmem;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LSH_ERR_CUDA;
-  kfn<<<grid, kThreads, smem, s>>>(mqk, mv, p);
+  kfn<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
 }
 

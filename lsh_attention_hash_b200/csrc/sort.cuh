@@ -153,6 +153,123 @@ sort_scatter_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
   }
 }
 
+// Whole-segment sort in one CTA (L <= 65536, n_buckets <= 1024): the bucket
+// ids of the segment are cached in shared memory as uint16, each of the 16
+// warps counts a contiguous range into its own histogram, the CTA turns the
+// (bucket, warp) counts into exclusive offsets (bucket-major, so warp ranges
+// stay in position order inside a bucket), and each warp then places its range
+// in order with the same warp-match ranking as sort_scatter_kernel.
+constexpr int kSegWarps = 16;
+constexpr int kSegMaxL = 65536;
+constexpr int kSegMaxBuckets = 1024;
+
+__host__ __device__ inline size_t sort_segment_smem(int L, int n_buckets) {
+  return (size_t)kSegWarps * n_buckets * 4      // per-warp histograms / offsets
+         + (size_t)kSegMaxBuckets * 4           // bucket totals / bases
+         + 32 * 4                               // warp sums of the scan
+         + (((size_t)L * 2 + 15) & ~(size_t)15);  // cached bucket ids
+}
+
+__global__ void __launch_bounds__(kSegWarps * 32)
+sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, int32_t* __restrict__ perm,
+                    int32_t* __restrict__ inv) {
+  extern __shared__ uint32_t sm_u32[];
+  uint32_t* hist = sm_u32;                          // [kSegWarps][n_buckets]
+  uint32_t* tot = hist + kSegWarps * n_buckets;     // [n_buckets]
+  uint32_t* ws = tot + kSegMaxBuckets;              // [32]
+  uint16_t* ids = reinterpret_cast<uint16_t*>(ws + 32);  // [L]
+  const long long seg = blockIdx.x;
+  const int32_t* src = buckets + seg * L;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per_warp = (L + kSegWarps - 1) / kSegWarps;
+  const int lo = min(L, warp * per_warp), hi = min(L, lo + per_warp);
+
+  for (int i = threadIdx.x; i < kSegWarps * n_buckets; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  // 1. per-warp counts of a contiguous range; ids cached (out-of-range ids: 0xFFFF, skipped)
+  uint32_t* my = hist + warp * n_buckets;
+  for (int i = lo + lane; i < hi; i += 32) {
+    int b = src[i];
+    if ((unsigned)b >= (unsigned)n_buckets) {
+      record_error(LSH_ERR_INVALID_ARG);
+      b = 0xFFFF;
+    } else {
+      atomicAdd(&my[b], 1u);
+    }
+    ids[i] = (uint16_t)b;
+  }
+  __syncthreads();
+  // 2a. within each bucket, exclusive offsets over the warps (in warp = position order)
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
+    uint32_t run = 0;
+    for (int w = 0; w < kSegWarps; ++w) {
+      const uint32_t c = hist[w * n_buckets + b];
+      hist[w * n_buckets + b] = run;
+      run += c;
+    }
+    tot[b] = run;
+  }
+  __syncthreads();
+  // 2b. exclusive scan of the bucket totals (two buckets per thread)
+  {
+    const int b0 = 2 * threadIdx.x;
+    const uint32_t t0 = b0 < n_buckets ? tot[b0] : 0u, t1 = b0 + 1 < n_buckets ? tot[b0 + 1] : 0u;
+    const uint32_t local = t0 + t1;
+    uint32_t incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) ws[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t w = lane < kSegWarps ? ws[lane] : 0u;
+      uint32_t wi = w;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, wi, off);
+        if (lane >= off) wi += y;
+      }
+      if (lane < kSegWarps) ws[lane] = wi - w;
+    }
+    __syncthreads();
+    const uint32_t excl = ws[warp] + incl - local;
+    if (b0 < n_buckets) tot[b0] = excl;
+    if (b0 + 1 < n_buckets) tot[b0 + 1] = excl + t0;
+  }
+  __syncthreads();
+  // 2c. first sorted slot of (bucket, warp)
+  for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
+    const uint32_t base = tot[b];
+    for (int w = 0; w < kSegWarps; ++w) hist[w * n_buckets + b] += base;
+  }
+  __syncthreads();
+  // 3. stable placement of the warp's range
+  int32_t* dst = perm + seg * L;
+  int32_t* idst = inv ? inv + seg * L : nullptr;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = lo; base < hi; base += 32) {
+    const int i = base + lane;
+    const int b = i < hi ? (int)ids[i] : 0xFFFF;
+    const bool valid = b < n_buckets;
+    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+    unsigned peers = 0;
+    uint32_t slot = 0;
+    if (valid) {
+      peers = __match_any_sync(vmask, b);
+      slot = my[b] + __popc(peers & lt_mask);
+    }
+    __syncwarp();
+    if (valid && (peers & lt_mask) == 0) my[b] += __popc(peers);
+    __syncwarp();
+    if (valid) {
+      dst[slot] = i;
+      if (idst) idst[i] = (int32_t)slot;
+    }
+  }
+}
+
 // Gather of sorted rows: dst[seg][s][:] = src[bh][perm[seg][s]][:], 16 B per thread.
 __global__ void gather_rows_kernel(const uint8_t* __restrict__ src, const int32_t* __restrict__ perm,
                                    long long n_rows, int L, int n_rounds, int row_bytes,

@@ -129,6 +129,40 @@ LSH_API lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L,
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * lsh_sort_permute_noalloc -- lsh_sort_permute (without the optional row
+ * gather) for callers that cannot hand the library any scratch memory.
+ * The pages have no counterpart of this call; it exists for this library's
+ * users only.
+ *
+ * Some callers cannot allocate device memory while they run: a plugin that a
+ * host application gives only its input and output buffers, a process whose
+ * device memory another framework's pool has already reserved, or a code path
+ * that must not pay cudaMalloc's implicit synchronisation.  This entry point
+ * takes no workspace and allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library call): its scratch is a 16 MiB array of static device
+ * memory inside the library, which every GPU that loads the library holds
+ * until the process exits.
+ *
+ *   buckets, perm, inv: as for lsh_sort_permute (inv nullable).
+ *
+ * Returns LSH_ERR_WORKSPACE, before any launch, when the sizes need more
+ * scratch than the 16 MiB array holds, i.e. when
+ * lsh_sort_workspace_bytes(B, H, L, n_rounds, n_buckets) > 16 MiB for the
+ * count-scan-scatter kernels this call always uses.  All other argument
+ * rules and errors are those of lsh_sort_permute.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current), so make that first call before any stream capture.  Every
+ * call on a device shares the one array and leaves its contents behind; the
+ * call clears what must start at zero itself.  Calls whose work overlaps on the
+ * GPU (different streams, or graphs running at the same time) race on the
+ * array: order them, for example on one stream.
+ */
+LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H, int L,
+                                            int n_rounds, int n_buckets, int32_t* perm,
+                                            int32_t* inv, void* stream);
+
+/*
  * lsh_chunk_attend -- attention of every sorted slot to its own chunk and the
  * previous chunk, per round, scattered back to original token order.
  * (twgreatdaily ICLR 2020 Reformer article, "1 LSH Attention": sum over the

@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     LSHError,
     lsh_hash,
     lsh_sort_permute,
+    lsh_sort_permute_noalloc,
     lsh_sort_workspace_bytes,
     lsh_chunk_attend,
     lsh_combine_rounds,

@@ -43,6 +43,7 @@ _SIGS = {
     "lsh_sort_workspace_bytes": (_c_size, [_c_int] * 5),
     "lsh_sort_permute": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                   _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp]),
+    "lsh_sort_permute_noalloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "lsh_chunk_attend": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp,
                                   _vp, _c_int, _c_int, _c_float, _vp, _c_int, _vp, _vp]),
     "lsh_combine_rounds": (_c_int, [_vp, _c_int, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp,
@@ -164,6 +165,29 @@ def lsh_sort_permute(buckets, n_buckets, *, perm=None, inv=None, want_inv=False,
                                 _ptr(qk), _ptr(v), dtype_code, D, _ptr(qk_sorted), _ptr(v_sorted),
                                 _ptr(workspace), workspace.numel(), _stream(stream)), "lsh_sort_permute")
     return perm, inv, qk_sorted, v_sorted
+
+
+def lsh_sort_permute_noalloc(buckets, n_buckets, *, perm=None, inv=None, want_inv=False, stream=None):
+    """perm (and optionally inv) using the library's own static scratch instead of a workspace.
+
+    For callers that cannot provide device scratch memory; raises LSHError
+    (LSH_ERR_WORKSPACE) when the sizes need more than the library's 16 MiB.
+    Returns (perm, inv).
+    """
+    lib = load_library()
+    _need(buckets, "buckets", torch.int32)
+    B, H, n_rounds, L = buckets.shape
+    shape = tuple(buckets.shape)
+    if perm is None:
+        perm = torch.empty(shape, dtype=torch.int32, device=buckets.device)
+    _need(perm, "perm", torch.int32, shape)
+    if inv is None and want_inv:
+        inv = torch.empty(shape, dtype=torch.int32, device=buckets.device)
+    if inv is not None:
+        _need(inv, "inv", torch.int32, shape)
+    _check(lib.lsh_sort_permute_noalloc(_ptr(buckets), B, H, L, n_rounds, n_buckets, _ptr(perm), _ptr(inv),
+                                        _stream(stream)), "lsh_sort_permute_noalloc")
+    return perm, inv
 
 
 def lsh_chunk_attend(qk, v, perm, chunk, *, self_mask=True, scale=None, qk_sorted=None, v_sorted=None,

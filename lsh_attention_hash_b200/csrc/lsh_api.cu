@@ -3,6 +3,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
 #include <stdint.h>
 
 #include <cudaTypedefs.h>
@@ -288,6 +289,70 @@ lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L, int n_r
     lsh::gather_rows_kernel<<<blocks, 256, 0, s>>>((const uint8_t*)v, perm, nrows, L, n_rounds,
                                                    row_bytes, (uint8_t*)v_sorted);
   }
+  return launch_status();
+}
+
+}  // extern "C"
+
+namespace {
+
+// Scratch of lsh_sort_permute_noalloc: static device memory of this library,
+// 16 MiB of uint32 counters on every device that loads it.
+constexpr size_t kNoallocScratchWords = (size_t)4 << 20;
+__device__ __align__(256) uint32_t g_noalloc_scratch[kNoallocScratchWords];
+
+// Device address of g_noalloc_scratch, looked up once per device with that
+// device current (in host code the array's name is only a host-side stand-in).
+uint32_t* noalloc_scratch_ptr() {
+  static std::mutex mu;
+  static uint32_t* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<uint32_t*>(p);
+  }
+  return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H, int L, int n_rounds,
+                                    int n_buckets, int32_t* perm, int32_t* inv, void* stream) {
+  if (B < 0 || H < 0 || L < 0 || L > (1 << 24)) return LSH_ERR_SHAPE;
+  if (n_rounds < 1 || n_buckets < 2 || n_buckets > 65536 || (n_buckets & 1)) return LSH_ERR_SHAPE;
+  if (!index_space_ok(B, H, L, n_rounds)) return LSH_ERR_SHAPE;
+  if (!buckets || !perm) return LSH_ERR_INVALID_ARG;
+  if (!aligned16(buckets) || !aligned16(perm) || (inv && !aligned16(inv))) return LSH_ERR_ALIGN;
+  const long long segs = (long long)B * H * n_rounds;
+  if (segs == 0 || L == 0) return LSH_OK;
+  const size_t words = lsh::sort_ws_elems(segs, L, n_buckets);
+  if (words > kNoallocScratchWords) return LSH_ERR_WORKSPACE;
+  if (segs > 65535) return LSH_ERR_UNSUPPORTED;
+  uint32_t* cnt = noalloc_scratch_ptr();
+  if (!cnt) return LSH_ERR_CUDA;
+
+  cudaStream_t s = as_stream(stream);
+  const int T = lsh::sort_tile(n_buckets);
+  const int nt = (L + T - 1) / T;
+  const bool in_smem = n_buckets <= kSortSmemBuckets;
+  const size_t hist_smem = in_smem ? (size_t)n_buckets * sizeof(uint32_t) : 0;
+  // with global-memory counters the previous call's counts must not leak in
+  if (!in_smem && cudaMemsetAsync(cnt, 0, words * sizeof(uint32_t), s) != cudaSuccess) return LSH_ERR_CUDA;
+  if (hist_smem > 48 * 1024) {
+    cudaFuncSetAttribute(lsh::sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
+    cudaFuncSetAttribute(lsh::sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
+  }
+  dim3 grid(nt, (unsigned)segs);
+  lsh::sort_count_kernel<<<grid, 256, hist_smem, s>>>(buckets, L, n_buckets, T, cnt);
+  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+  lsh::sort_scan_kernel<<<(unsigned)segs, 1024, 0, s>>>(cnt, (long long)n_buckets * nt);
+  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+  lsh::sort_scatter_kernel<<<grid, 32, hist_smem, s>>>(buckets, L, n_buckets, T, cnt, perm, inv);
   return launch_status();
 }
 

@@ -20,10 +20,11 @@
 // the winning group tells its sign.  The exact top-two |p| for the near-tie
 // flag are tracked only when that output is requested.
 //
-// Warps: 0 TMA producer, 1 UMMA issuer, 2-9 epilogue.  Two epilogue warps
-// share each TMEM lane quarter (32 rows) and take one half of the columns of
-// every accumulator chunk each; at the end of a tile the second half's row
-// states go through shared memory to the first half, which merges and stores.
+// Warps: 0 TMA producer, 1 UMMA issuer, then 4 * SPLIT epilogue warps.  SPLIT
+// epilogue warps share each TMEM lane quarter (32 rows) and take 1/SPLIT of
+// the columns of every accumulator chunk each; at the end of a tile the other
+// parts' row states go through shared memory to part 0, which merges and
+// stores.
 #pragma once
 
 #include "tc_common.cuh"
@@ -31,8 +32,8 @@
 namespace lsh {
 namespace hash_tc {
 
-constexpr int kThreads = 320;  // warp 0 TMA, warp 1 UMMA, warps 2-9 epilogue
 constexpr int kRows = 128;
+__host__ __device__ constexpr int threads_for(int split) { return 64 + 128 * split; }
 constexpr int kStages = 2;
 
 template <int D>
@@ -42,11 +43,11 @@ struct Layout {
   static constexpr uint32_t kA = 0;
   static constexpr uint32_t kR = kStages * kStageBytes;          // R[round]: (half/64) boxes of D x 128 B
   __host__ __device__ static constexpr uint32_t bar_off(int half) { return kR + (uint32_t)D * half * 2; }
-  // a_full[2] a_empty[2] acc_full[2] acc_empty[2] r_full done half_done[2] merged[2]
+  // a_full[2] a_empty[2] acc_full[2] acc_empty[2] r_full done part_done[2] merged[2]
   static constexpr int kNumBars = 14;
-  // second-half row states: [2 tile parities][5 fields][128 rows] x 4 B
+  // row states of parts 1..3: [2 tile parities][3 parts][5 fields][128 rows] x 4 B
   __host__ __device__ static constexpr uint32_t xchg_off(int half) { return bar_off(half) + kNumBars * 8 + 16; }
-  __host__ __device__ static constexpr uint32_t smem_bytes(int half) { return xchg_off(half) + 2 * 5 * kRows * 4 + 1024; }
+  __host__ __device__ static constexpr uint32_t smem_bytes(int half) { return xchg_off(half) + 2 * 3 * 5 * kRows * 4 + 1024; }
 };
 
 struct Params {
@@ -105,8 +106,8 @@ __device__ __forceinline__ void process16(RowState& st, const uint32_t* raw, int
   }
 }
 
-template <int D, int NC, bool FLAG>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int NC, bool FLAG, int SPLIT>
+__global__ void __launch_bounds__(threads_for(SPLIT), 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_r,
                const Params p) {
   using Lay = Layout<D>;
@@ -119,8 +120,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   uint64_t* acc_empty = bars + 6;
   uint64_t* r_full = bars + 8;
   uint64_t* done_bar = bars + 9;
-  uint64_t* half_done = bars + 10;  // [2] second-half states written (128 arrivals)
-  uint64_t* merged = bars + 12;     // [2] second-half states consumed (128 arrivals)
+  uint64_t* part_done = bars + 10;  // [2] parts 1.. states written ((SPLIT-1) * 128 arrivals)
+  uint64_t* merged = bars + 12;     // [2] those states consumed (128 arrivals)
   float* xchg = reinterpret_cast<float*>(smem + Lay::xchg_off(p.half));
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + Lay::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + Lay::kNumBars) + 1;
@@ -133,8 +134,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       tc::mbar_init(&a_full[i], 1);
       tc::mbar_init(&a_empty[i], 1);
       tc::mbar_init(&acc_full[i], 1);
-      tc::mbar_init(&acc_empty[i], 256);
-      tc::mbar_init(&half_done[i], 128);
+      tc::mbar_init(&acc_empty[i], 128 * SPLIT);
+      tc::mbar_init(&part_done[i], 128 * (SPLIT - 1));
       tc::mbar_init(&merged[i], 128);
     }
     tc::mbar_init(r_full, 1);
@@ -214,8 +215,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     }
     __syncwarp();
   } else {
+    constexpr int kCols = NC / SPLIT;    // columns of every chunk handled by one part
     const int q = warp & 3;
-    const int ch = (warp - 2) >> 2;      // column half of every chunk
+    const int ch = (warp - 2) >> 2;      // part of every chunk
     const int r = q * 32 + lane;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t seq = 0, it = 0;
@@ -228,9 +230,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int piece = 0; piece < NC / 64; ++piece) {
+        for (int piece = 0; piece < kCols / 32; ++piece) {
           uint32_t raw[32];
-          const int col = ch * (NC / 2) + piece * 32;
+          const int col = ch * kCols + piece * 32;
           tc::tmem_ld32(lane_base + tmem + b * NC + col, raw);
           tc::tmem_wait_ld();
           const int g = (c * NC + col) >> 4;
@@ -242,8 +244,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       }
       if (!ok) break;
       const int tp = it & 1;
-      float* xs = xchg + tp * 5 * kRows;
-      if (ch == 1) {
+      if (ch > 0) {
+        float* xs = xchg + (tp * 3 + (ch - 1)) * 5 * kRows;
         ok = att_tc::warp_wait(&merged[tp], ((it >> 1) & 1) ^ 1, abort_flag);
         if (!ok) break;
         xs[r] = st.best_key;
@@ -251,26 +253,29 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         xs[2 * kRows + r] = st.best_raw;
         xs[3 * kRows + r] = st.v1;
         xs[4 * kRows + r] = st.v2;
-        tc::mbar_arrive(&half_done[tp]);
+        tc::mbar_arrive(&part_done[tp]);
         continue;
       }
-      ok = att_tc::warp_wait(&half_done[tp], (it >> 1) & 1, abort_flag);
+      ok = att_tc::warp_wait(&part_done[tp], (it >> 1) & 1, abort_flag);
       if (!ok) break;
-      const float ok_key = xs[r];
-      const int o_g = __float_as_int(xs[kRows + r]);
-      const float o_raw = xs[2 * kRows + r];
-      const float o_v1 = xs[3 * kRows + r], o_v2 = xs[4 * kRows + r];
+#pragma unroll
+      for (int o = 0; o < SPLIT - 1; ++o) {
+        const float* xs = xchg + (tp * 3 + o) * 5 * kRows;
+        const float o_key = xs[r];
+        const int o_g = __float_as_int(xs[kRows + r]);
+        // the parts cover disjoint groups; on equal keys the lower group wins
+        if (o_key > st.best_key || (o_key == st.best_key && o_g < st.best_g)) {
+          st.best_key = o_key;
+          st.best_g = o_g;
+          st.best_raw = xs[2 * kRows + r];
+        }
+        if (FLAG) {
+          const float o_v1 = xs[3 * kRows + r], o_v2 = xs[4 * kRows + r];
+          st.v2 = fmaxf(fmaxf(st.v2, o_v2), fminf(st.v1, o_v1));
+          st.v1 = fmaxf(st.v1, o_v1);
+        }
+      }
       tc::mbar_arrive(&merged[tp]);
-      // the two halves cover disjoint groups; on equal keys the lower group wins
-      if (ok_key > st.best_key || (ok_key == st.best_key && o_g < st.best_g)) {
-        st.best_key = ok_key;
-        st.best_g = o_g;
-        st.best_raw = o_raw;
-      }
-      if (FLAG) {
-        st.v2 = fmaxf(fmaxf(st.v2, o_v2), fminf(st.v1, o_v1));
-        st.v1 = fmaxf(st.v1, o_v1);
-      }
       const long long row = tile * kRows + r;
       if (row < p.nrows) {
         const uint32_t kb = __float_as_uint(st.best_key);

@@ -105,7 +105,7 @@ inline bool hash_tc_eligible(int dtype, int D, int half, int n_rounds, const Dev
   return n_rounds <= di.sms;
 }
 
-template <int D, int NC, bool FLAG>
+template <int D, int NC, bool FLAG, int SPLIT>
 lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, int n_rounds, int half,
                           int32_t* buckets, uint8_t* near_tie, cudaStream_t s, int sms) {
   using namespace lsh::hash_tc;
@@ -124,20 +124,23 @@ lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, in
   p.n_tiles = (rows + kRows - 1) / kRows;
   p.per_round = (int)std::max<long long>(1, std::min<long long>(sms / n_rounds, p.n_tiles));
   const unsigned grid = (unsigned)(p.per_round * n_rounds);
-  auto kfn = hash_tc_kernel<D, NC, FLAG>;
+  auto kfn = hash_tc_kernel<D, NC, FLAG, SPLIT>;
   const int smem = (int)Layout<D>::smem_bytes(half);
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LSH_ERR_CUDA;
-  kfn<<<grid, kThreads, smem, s>>>(mx, mr, p);
+  kfn<<<grid, threads_for(SPLIT), smem, s>>>(mx, mr, p);
   return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
 }
 
 template <int D>
 lsh_status dispatch_hash_tc(const void* qk, const void* R, int B, int H, int L, int n_rounds, int half,
                             int32_t* buckets, uint8_t* near_tie, cudaStream_t s, int sms) {
-#define LSH_HTC(NC)                                                                                           \
-  return near_tie ? launch_hash_tc<D, NC, true>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, sms)   \
-                  : launch_hash_tc<D, NC, false>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, sms)
+#define LSH_HTC(NC)                                                                                    \
+  return near_tie                                                                                      \
+             ? launch_hash_tc<D, NC, true, (NC >= 128 ? 4 : 2)>(qk, R, B, H, L, n_rounds, half, buckets, \
+                                                                 near_tie, s, sms)                     \
+             : launch_hash_tc<D, NC, false, (NC >= 128 ? 4 : 2)>(qk, R, B, H, L, n_rounds, half, buckets, \
+                                                                  near_tie, s, sms)
   if (half == 64) LSH_HTC(64);
   if (half == 128) LSH_HTC(128);
   LSH_HTC(256);

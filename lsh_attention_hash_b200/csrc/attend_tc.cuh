@@ -19,19 +19,27 @@
 //                                accumulated behind P in the same TMEM buffer
 // and the rows go back to their original positions perm[s].
 //
-// Warp roles (384 threads, persistent CTAs, one per SM):
+// Warp roles (384 threads, persistent CTAs, one per SM; 12 warps leave 168
+// registers per thread):
 //   warps 0-1  producers: read perm and gather the QK and V rows of each chunk
 //              with 16-byte cp.async copies (32 lanes generate addresses in
 //              parallel; many small TMA row gathers were issue-bound) straight
 //              into 128-byte-swizzled K-major UMMA tiles, in a ring of three
-//              128-row slots;
+//              128-row slots (warp w copies rows 64w..64w+63 of a slot);
 //   warp 2     TMEM owner and single-thread UMMA issuer; it never blocks on
 //              one step while another step's UMMA could go (S of step t+1 and
 //              PV of step t are issued in whichever order they become ready);
-//   warp 3     key multipliers scale * log2(e) / ||k|| of every gathered row;
+//   warp 3     idle;
 //   warps 4-7  softmax + epilogue of the even steps, warps 8-11 of the odd
 //              steps (one query row per thread), so that one step's softmax
 //              overlaps the other step's UMMAs, loads and stores.
+// Key lengths come from the S tile itself: the pair's rows are also its keys,
+// so row r finds ||k||^2 of its own row on the diagonal (key 64 + r % 64) and
+// publishes the key multiplier scale * log2(e) / ||k||; the rows of a unit's
+// leading chunk (which no earlier step of this CTA saw) are measured directly
+// from shared memory.  The softmax uses the Cauchy-Schwarz bound
+// q.k / ||k|| <= ||q|| as its shift (one pass over S); a row whose sum would
+// underflow under that shift is redone with its exact maximum.
 // TMEM: two step buffers of 256 columns (S: 192 fp32, P: first 96, O: 96..96+D).
 // Every wait is bounded; a timeout unwinds the CTA cleanly.
 #pragma once
@@ -213,17 +221,17 @@ struct FillIter {
 };
 
 // Original positions of this lane's two rows of the producer warp's half of a
-// fill (global loads; issued one fill ahead so that their latency hides behind
+// fill (global loads, issued one fill ahead so that their latency hides behind
 // the slot wait).  Producer warp pw owns local rows [64 pw, 64 pw + 64).
 __device__ __forceinline__ void fill_positions(const Params& p, const Fill& f, int pw, int (&pos)[2]) {
   const int lane = threadIdx.x & 31;
-  const int32_t* pseg = p.perm + f.seg * p.L;
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int i = 64 * pw + 32 * k + lane;  // local row of the slot
+    pos[k] = 0;
     if (i >= f.row0 && i < f.row0 + f.nrows) {
       const int chunk = (i - f.row0) < 64 ? f.cA : f.cB;
-      pos[k] = pseg[chunk * kC + (i & 63)];
+      pos[k] = p.perm[f.seg * p.L + chunk * kC + (i & 63)];
     }
   }
 }
@@ -241,9 +249,8 @@ __device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, ui
   constexpr int kRowsPerInst = 32 / kPieces;
   const int lane = threadIdx.x & 31;
   int32_t* perm_s = reinterpret_cast<int32_t*>(smem + Lay::kPerm) + slot * kRows;
-  const long long bh = f.seg / p.n_rounds;
   const int base = 64 * pw;
-  const bool mine = base + 64 > f.row0 && base < f.row0 + f.nrows;  // the fill covers this warp's rows
+  const bool mine = base >= f.row0 && base < f.row0 + f.nrows;  // the fill covers this warp's rows
   if (mine) {
     long long grow[2];
 #pragma unroll
@@ -251,7 +258,7 @@ __device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, ui
       const int i = base + 32 * k + lane;
       const int chunk = (i - f.row0) < 64 ? f.cA : f.cB;
       perm_s[i] = pos[k];
-      grow[k] = p.sorted_input ? f.seg * p.L + chunk * kC + (i & 63) : bh * p.L + pos[k];
+      grow[k] = p.sorted_input ? f.seg * p.L + chunk * kC + (i & 63) : (f.seg / p.n_rounds) * p.L + pos[k];
     }
     const uint32_t qk_dst = tc::smem_u32(smem + Lay::kQK + slot * Lay::kSlotBytes);
     const uint32_t v_dst = tc::smem_u32(smem + Lay::kV + slot * Lay::kSlotBytes);
@@ -290,15 +297,14 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
 }
 
 template <int D, typename TO>
-__global__ void __launch_bounds__(kThreads, 1)
-attend_tc_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) {
   using Lay = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* full = bars;            // [3] slot filled (64 producer lanes' copies landed)
   uint64_t* empty = bars + 3;       // [3] slot released by the UMMAs
-  uint64_t* cm_full = bars + 6;     // [3] key multipliers of the slot's fill written (32 arrivals)
+  uint64_t* cm_full = bars + 6;     // [3] key multipliers of the slot's fill written (128 arrivals)
   uint64_t* s_full = bars + 9;      // [2] S of the step buffer computed
   uint64_t* p_ready = bars + 11;    // [2] P written (128 arrivals)
   uint64_t* o_full = bars + 13;     // [2] O computed
@@ -314,7 +320,7 @@ attend_tc_kernel(const Params p) {
     for (int i = 0; i < kSlots; ++i) {
       tc::mbar_init(&full[i], 64);
       tc::mbar_init(&empty[i], 1);
-      tc::mbar_init(&cm_full[i], 32);
+      tc::mbar_init(&cm_full[i], 128);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&s_full[i], 1);
@@ -345,7 +351,7 @@ attend_tc_kernel(const Params p) {
       FillIter nx = fi;
       nx.advance(p);
       int npos[2] = {0, 0};
-      if (nx.valid) fill_positions(p, nx.get(p), pw, npos);  // next fill's positions, in flight during the wait
+      if (nx.valid) fill_positions(p, nx.get(p), pw, npos);  // in flight during the wait
       const int slot = f % kSlots;
       if (!warp_wait(&empty[slot], ((f / kSlots) & 1) ^ 1, abort_flag)) break;
       producer_fill<D>(p, smem, &full[slot], slot, cur, pw, pos);
@@ -426,30 +432,14 @@ attend_tc_kernel(const Params p) {
       drain_wait(done_bar, 0);
     }
     __syncwarp();
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ key multipliers
-    uint32_t f = 0;
-    FillIter fi;
-    fi.init(p);
-    while (fi.valid) {
-      const Fill cur = fi.get(p);
-      const int slot = f % kSlots;
-      if (!warp_wait(&full[slot], (f / kSlots) & 1, abort_flag)) break;
-      const uint8_t* qs = smem + Lay::kQK + slot * Lay::kSlotBytes;
-      for (int i = cur.row0 + lane; i < cur.row0 + cur.nrows; i += 32)
-        colmul[slot * kRows + i] = row_colmul<D>(qs, i, p.colscale);
-      tc::mbar_arrive(&cm_full[slot]);
-      ++f;
-      fi.advance(p);
-    }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
     const int wg = (warp - 4) >> 2;      // 0: even steps, 1: odd steps
     const int q = warp & 3;              // TMEM lane quarter of this warp
     const int r = q * 32 + lane;         // query row of the step
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const bool low = q < 2;              // rows 0..63: keys [0, 128); rows 64..127: keys [64, 192)
-    const int self_i = 64 + (r & 63);    // own key, as an index into the row's 128 keys
+    const int g_self = 2 + (q & 1);      // 32-key group of the row's own key; in it, element `lane`
     StepIter it;
     it.init(p);
     if (wg == 1) it.advance(p);
@@ -458,57 +448,95 @@ attend_tc_kernel(const Params p) {
       const uint32_t t = it.t, b = t & 1;
       const uint32_t fp = it.f - 1, fc = it.f;
       const int sp = fp % kSlots, sc = fc % kSlots;
-      ok = warp_wait(&cm_full[sp], (fp / kSlots) & 1, abort_flag) &&
-           warp_wait(&cm_full[sc], (fc / kSlots) & 1, abort_flag) &&
+      // the first step of a unit is the one whose previous chunk is the unit's leading fill
+      const bool first = (it.j == (int)((it.u - it.seg * p.units_per_seg) * p.run));
+      ok = warp_wait(&full[sc], (fc / kSlots) & 1, abort_flag) && warp_wait(&full[sp], (fp / kSlots) & 1, abort_flag) &&
            warp_wait(&s_full[b], (t >> 1) & 1, abort_flag);
       if (!ok) break;
       tc::tc_fence_after();
+      const uint32_t sbuf = lane_base + tmem + b * kBufCols;
+      const uint32_t scol = low ? 0 : 64;  // S column of the row's first key
+      if (first) {  // the leading chunk's key multipliers, measured directly
+        if (!low) colmul[sp * kRows + r] = row_colmul<D>(smem + Lay::kQK + sp * Lay::kSlotBytes, r, p.colscale);
+        tc::mbar_arrive(&cm_full[sp]);
+      }
+      // own key multiplier from the diagonal of S (||k_r||^2 at key 64 + r % 64)
+      float diag;
+      {
+        uint32_t raw[32];
+        tc::tmem_ld32(sbuf + scol + 32 * g_self, raw);
+        tc::tmem_wait_ld();
+        diag = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) diag = (e == lane) ? __uint_as_float(raw[e]) : diag;
+      }
+      const float cm_own = p.colscale / fmaxf(sqrtf(fmaxf(diag, 0.f)), 1e-12f);
+      colmul[sc * kRows + r] = cm_own;
+      tc::mbar_arrive(&cm_full[sc]);
       const int chunk = 2 * it.j + (low ? 0 : 1);
       const bool valid = chunk < p.n_chunks;
       const int pos = perm_s[sc * kRows + r];
-      const uint32_t sbuf = lane_base + tmem + b * kBufCols;
-      const uint32_t scol = low ? 0 : 64;  // S column of the row's first key
+      ok = warp_wait(&cm_full[sp], (fp / kSlots) & 1, abort_flag) && warp_wait(&cm_full[sc], (fc / kSlots) & 1, abort_flag);
+      if (!ok) break;
       const float* cm_lo = low ? colmul + sp * kRows + 64 : colmul + sc * kRows;  // keys 0..63 of the row
       const float* cm_hi = low ? colmul + sc * kRows : colmul + sc * kRows + 64;  // keys 64..127
       const int g_first = (low && it.j == 0) ? 2 : 0;  // chunk 0 has no previous chunk
-      // pass 1: row maximum of the scaled logits (log2 domain)
-      float m = -INFINITY;
+      // shift: ||q|| * scale * log2(e) bounds every logit of the row (log2 domain)
+      float m = diag * cm_own;
+      float l = 0.f;   // sum of the weights (log-sum-exp)
+      float lr = 0.f;  // sum of the bf16-rounded weights that P holds (normalises O)
+      uint32_t pk[64];  // the row's P, packed bf16 pairs, stored once the row sum is known to be safe
+      for (int attempt = 0; attempt < 2; ++attempt) {
+        l = 0.f;
+        lr = 0.f;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t raw[32];
-        tc::tmem_ld32(sbuf + scol + 32 * g, raw);
-        tc::tmem_wait_ld();
-        if (g < g_first) continue;
-        const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
+        for (int g = 0; g < 4; ++g) {
+          uint32_t raw[32];
+          tc::tmem_ld32(sbuf + scol + 32 * g, raw);
+          tc::tmem_wait_ld();
+          const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
+          const bool dead = g < g_first;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float v = __uint_as_float(raw[e]) * cm[e];
-          if (p.self_mask && 32 * g + e == self_i) v = -INFINITY;
-          m = fmaxf(m, v);
+          for (int e = 0; e < 32; e += 2) {
+            float v0 = __uint_as_float(raw[e]) * cm[e];
+            float v1 = __uint_as_float(raw[e + 1]) * cm[e + 1];
+            if (g == g_self && p.self_mask) {
+              if (e == lane) v0 = -INFINITY;
+              if (e + 1 == lane) v1 = -INFINITY;
+            }
+            const float a = dead ? 0.f : tc::ex2_approx(v0 - m);
+            const float c = dead ? 0.f : tc::ex2_approx(v1 - m);
+            l += a + c;
+            const uint32_t w = tc::pack_bf16x2(a, c);
+            lr += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+            pk[16 * g + (e >> 1)] = w;
+          }
+        }
+        if (l > 1e-30f) break;
+        // the bound was too loose (long query rows): redo with the exact maximum; S is intact
+        // because P has not been written yet
+        m = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t raw[32];
+          tc::tmem_ld32(sbuf + scol + 32 * g, raw);
+          tc::tmem_wait_ld();
+          if (g < g_first) continue;
+          const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float v = __uint_as_float(raw[e]) * cm[e];
+            if (g == g_self && p.self_mask && e == lane) v = -INFINITY;
+            m = fmaxf(m, v);
+          }
         }
       }
-      // pass 2: P = exp2(x - m) in bf16 over the head of the buffer, row sum
-      float l = 0.f;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        uint32_t raw[32];
-        tc::tmem_ld32(sbuf + scol + 32 * g, raw);
-        tc::tmem_wait_ld();
-        const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
-        const bool dead = g < g_first;
-        uint32_t pk[16];
+        uint32_t w16[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float v0 = __uint_as_float(raw[e]) * cm[e];
-          float v1 = __uint_as_float(raw[e + 1]) * cm[e + 1];
-          if (p.self_mask && 32 * g + e == self_i) v0 = -INFINITY;
-          if (p.self_mask && 32 * g + e + 1 == self_i) v1 = -INFINITY;
-          const float a = dead ? 0.f : tc::ex2_approx(v0 - m);
-          const float c = dead ? 0.f : tc::ex2_approx(v1 - m);
-          l += a + c;
-          pk[e >> 1] = tc::pack_bf16x2(a, c);
-        }
-        tc::tmem_st16(sbuf + (low ? 16 * g : 32 + 16 * g), pk);
+        for (int e = 0; e < 16; ++e) w16[e] = pk[16 * g + e];
+        tc::tmem_st16(sbuf + (low ? 16 * g : 32 + 16 * g), w16);
       }
       {
         uint32_t z[32];
@@ -523,7 +551,7 @@ attend_tc_kernel(const Params p) {
       ok = warp_wait(&o_full[b], (t >> 1) & 1, abort_flag);
       if (!ok) break;
       tc::tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / lr;  // O = sum p~ v / sum p~: a convex combination of the values
       TO* dst = reinterpret_cast<TO*>(p.out) + (it.seg * p.L + pos) * (long long)D;
 #pragma unroll
       for (int g = 0; g < D / 32; ++g) {

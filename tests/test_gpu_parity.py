@@ -129,6 +129,15 @@ def test_hash_with_and_without_flags_agree():
         assert f2 is None and torch.equal(b1, b2)
 
 
+@pytest.mark.parametrize("scale", [0.02, 6.0, 40.0])
+def test_chunk64_attention_scales(scale):
+    """Small and large logit scales on the tensor-core attention (40: the row sums underflow
+    under the Cauchy-Schwarz shift, so the kernel falls back to the exact maximum)."""
+    w = synth.small_workload("scales", 1, 2, 1024, 128, "bf16", 16, 64, 2)
+    qk, v, R = synth.make_inputs(w, seed=9)
+    full_parity(w, qk, v, R, scale=scale)
+
+
 def test_fp32_output_from_bf16_input():
     w = synth.small_workload("f32out", 2, 2, 512, 128, "bf16", 16, 64, 2)
     qk, v, R = synth.make_inputs(w, seed=4)

@@ -331,7 +331,11 @@ def run_ours(args, w, rank, world, local_rank):
         peak = peaks["bf16_tflops_sustained"]
         unit = "TFLOP/s"
     t_roof = max(alg["total_bytes"] / (peaks["hbm_gbs"] * 1e9), alg["attn_flops"] / (peaks["bf16_tflops"] * 1e12))
-    launches_per_step = 6 + (1 if w.n_buckets > 16384 else 0)
+    if w.L <= 65536 and w.n_buckets <= 1024:
+        sort_launches = 1                                  # one CTA per segment
+    else:
+        sort_launches = 3 + (1 if w.n_buckets > 16384 else 0)  # count, scan, scatter (+ counter clear)
+    launches_per_step = 3 + sort_launches                  # hash, sort, attend, combine
     sample_slices = 1
     c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices)
     line = {

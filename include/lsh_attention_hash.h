@@ -145,11 +145,11 @@ LSH_API lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L,
  *
  *   buckets, perm, inv: as for lsh_sort_permute (inv nullable).
  *
- * Returns LSH_ERR_WORKSPACE, before any launch, when the sizes need more
- * scratch than the 16 MiB array holds, i.e. when
- * lsh_sort_workspace_bytes(B, H, L, n_rounds, n_buckets) > 16 MiB for the
- * count-scan-scatter kernels this call always uses.  All other argument
- * rules and errors are those of lsh_sort_permute.
+ * This call always runs the count-scan-scatter sort, whose counters take
+ * B*H*n_rounds * n_buckets * ceil(L / max(4096, n_buckets)) uint32 words; it
+ * returns LSH_ERR_WORKSPACE, before any launch, when that exceeds the array's
+ * 4 Mi words (16 MiB).  All other argument rules and errors are those of
+ * lsh_sort_permute.
  *
  * The first call on a device looks up the array's device address (with that
  * device current), so make that first call before any stream capture.  Every

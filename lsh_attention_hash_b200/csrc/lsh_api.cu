@@ -234,8 +234,14 @@ lsh_status lsh_hash(const void* qk, int dtype, int B, int H, int L, int D, const
   return launch_status();
 }
 
+// Shapes sorted by one CTA per segment (no workspace).
+static inline bool sort_by_segment(int L, int n_buckets) {
+  return L <= lsh::kSegMaxL && n_buckets <= lsh::kSegMaxBuckets;
+}
+
 size_t lsh_sort_workspace_bytes(int B, int H, int L, int n_rounds, int n_buckets) {
   if (B <= 0 || H <= 0 || L <= 0 || n_rounds <= 0 || n_buckets < 2) return 0;
+  if (sort_by_segment(L, n_buckets)) return 0;
   return lsh::sort_ws_elems((long long)B * H * n_rounds, L, n_buckets) * sizeof(uint32_t);
 }
 
@@ -260,28 +266,38 @@ lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L, int n_r
   const long long segs = (long long)B * H * n_rounds;
   if (segs == 0 || L == 0) return LSH_OK;
   const size_t need = lsh_sort_workspace_bytes(B, H, L, n_rounds, n_buckets);
-  if (!workspace || workspace_bytes < need) return LSH_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return LSH_ERR_ALIGN;
-  if (segs > 65535) return LSH_ERR_UNSUPPORTED;  // grid.y limit of this build
+  if (need > 0 && (!workspace || workspace_bytes < need)) return LSH_ERR_WORKSPACE;
+  if (need > 0 && !aligned16(workspace)) return LSH_ERR_ALIGN;
 
   cudaStream_t s = as_stream(stream);
-  const int T = lsh::sort_tile(n_buckets);
-  const int nt = (L + T - 1) / T;
-  uint32_t* cnt = (uint32_t*)workspace;
-  const bool in_smem = n_buckets <= kSortSmemBuckets;
-  const size_t hist_smem = in_smem ? (size_t)n_buckets * sizeof(uint32_t) : 0;
-  if (!in_smem && cudaMemsetAsync(cnt, 0, need, s) != cudaSuccess) return LSH_ERR_CUDA;
-  if (hist_smem > 48 * 1024) {
-    cudaFuncSetAttribute(lsh::sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
-    cudaFuncSetAttribute(lsh::sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
+  if (sort_by_segment(L, n_buckets)) {
+    const size_t smem = lsh::sort_segment_smem(L, n_buckets);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(lsh::sort_segment_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+      return LSH_ERR_CUDA;
+    lsh::sort_segment_kernel<<<(unsigned)segs, lsh::kSegWarps * 32, smem, s>>>(buckets, L, n_buckets, perm, inv);
+    if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+  } else {
+    if (segs > 65535) return LSH_ERR_UNSUPPORTED;  // grid.y limit of the multi-launch sort
+    const int T = lsh::sort_tile(n_buckets);
+    const int nt = (L + T - 1) / T;
+    uint32_t* cnt = (uint32_t*)workspace;
+    const bool in_smem = n_buckets <= kSortSmemBuckets;
+    const size_t hist_smem = in_smem ? (size_t)n_buckets * sizeof(uint32_t) : 0;
+    if (!in_smem && cudaMemsetAsync(cnt, 0, need, s) != cudaSuccess) return LSH_ERR_CUDA;
+    if (hist_smem > 48 * 1024) {
+      cudaFuncSetAttribute(lsh::sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
+      cudaFuncSetAttribute(lsh::sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
   }
-  dim3 grid(nt, (unsigned)segs);
-  lsh::sort_count_kernel<<<grid, 256, hist_smem, s>>>(buckets, L, n_buckets, T, cnt);
-  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
-  lsh::sort_scan_kernel<<<(unsigned)segs, 1024, 0, s>>>(cnt, (long long)n_buckets * nt);
-  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
-  lsh::sort_scatter_kernel<<<grid, 32, hist_smem, s>>>(buckets, L, n_buckets, T, cnt, perm, inv);
-  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+    dim3 grid(nt, (unsigned)segs);
+    lsh::sort_count_kernel<<<grid, 256, hist_smem, s>>>(buckets, L, n_buckets, T, cnt);
+    if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+    lsh::sort_scan_kernel<<<(unsigned)segs, 1024, 0, s>>>(cnt, (long long)n_buckets * nt);
+    if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+    lsh::sort_scatter_kernel<<<grid, 32, hist_smem, s>>>(buckets, L, n_buckets, T, cnt, perm, inv);
+    if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+  }
   if (gather) {
     const int row_bytes = D * (int)elt_size(dtype);
     const long long nrows = segs * L;
@@ -429,14 +445,29 @@ lsh_status lsh_combine_rounds(const void* out_rounds, int in_dtype, const float*
   const long long threads_total = ntok * (D / 8);
   const unsigned blocks = (unsigned)((threads_total + 255) / 256);
   cudaStream_t s = as_stream(stream);
-#define LSH_CMB(TI, TO)                                                                   \
-  lsh::combine_kernel<TI, TO><<<blocks, 256, 0, s>>>((const TI*)out_rounds, lse, ntok, L, D, \
-                                                     n_rounds, (TO*)out, lse_out)
+  const int G = D / 8;
+  const bool g_pow2 = (G & (G - 1)) == 0;
+  const int NR = (g_pow2 && n_rounds <= G && (n_rounds == 1 || n_rounds == 2 || n_rounds == 4 || n_rounds == 8))
+                     ? n_rounds : 0;
+#define LSH_CMB_NR(TI, TO, NRV)                                                                       \
+  lsh::combine_kernel<TI, TO, NRV><<<blocks, 256, 0, s>>>((const TI*)out_rounds, lse, ntok, L, D, n_rounds, \
+                                                          (TO*)out, lse_out)
+#define LSH_CMB(TI, TO)                   \
+  do {                                    \
+    switch (NR) {                         \
+      case 1: LSH_CMB_NR(TI, TO, 1); break; \
+      case 2: LSH_CMB_NR(TI, TO, 2); break; \
+      case 4: LSH_CMB_NR(TI, TO, 4); break; \
+      case 8: LSH_CMB_NR(TI, TO, 8); break; \
+      default: LSH_CMB_NR(TI, TO, 0); break; \
+    }                                     \
+  } while (0)
   if (in_dtype == LSH_F32) {
     if (out_dtype == LSH_F32) LSH_CMB(float, float); else LSH_CMB(float, __nv_bfloat16);
   } else {
     if (out_dtype == LSH_F32) LSH_CMB(__nv_bfloat16, float); else LSH_CMB(__nv_bfloat16, __nv_bfloat16);
   }
+#undef LSH_CMB_NR
 #undef LSH_CMB
   return launch_status();
 }

@@ -66,15 +66,20 @@ def test_hash_rejects_bad_arguments_before_launch(lib):
 
 def test_sort_rejects_bad_arguments_before_launch(lib):
     s = lib.lsh_sort_permute
-    ws = lib.lsh_sort_workspace_bytes(1, 1, 1024, 1, 16)
+    # one CTA per segment (L <= 65536, <= 1024 buckets) needs no workspace
+    assert lib.lsh_sort_workspace_bytes(1, 1, 1024, 1, 16) == 0
+    # more buckets: the count / scan / scatter sort and its workspace
+    nb = 2048
+    ws = lib.lsh_sort_workspace_bytes(1, 1, 1024, 1, nb)
     assert ws > 0
     assert s(A, 1, 1, 1024, 1, 15, A, None, None, None, BF16, 64, None, None, A, ws, None) == SHAPE
-    assert s(None, 1, 1, 1024, 1, 16, A, None, None, None, BF16, 64, None, None, A, ws, None) == INVALID
-    assert s(A, 1, 1, 1024, 1, 16, A, None, None, None, BF16, 64, None, None, None, 0, None) == WORKSPACE
-    assert s(A, 1, 1, 1024, 1, 16, A, None, None, None, BF16, 64, None, None, A, ws - 4, None) == WORKSPACE
-    assert s(A, 1, 1, 1024, 1, 16, A, None, A, None, BF16, 64, None, None, A, ws, None) == INVALID  # half a gather
-    assert s(A, 1, 1, 1024, 1, 16, A, A + 8, None, None, BF16, 64, None, None, A, ws, None) == ALIGN
-    assert s(A, 0, 1, 1024, 1, 16, A, None, None, None, BF16, 64, None, None, None, 0, None) == OK
+    assert s(None, 1, 1, 1024, 1, nb, A, None, None, None, BF16, 64, None, None, A, ws, None) == INVALID
+    assert s(A, 1, 1, 1024, 1, nb, A, None, None, None, BF16, 64, None, None, None, 0, None) == WORKSPACE
+    assert s(A, 1, 1, 1024, 1, nb, A, None, None, None, BF16, 64, None, None, A, ws - 4, None) == WORKSPACE
+    assert s(A, 1, 1, 1024, 1, nb, A, None, None, None, BF16, 64, None, None, A + 8, ws, None) == ALIGN
+    assert s(A, 1, 1, 1024, 1, nb, A, None, A, None, BF16, 64, None, None, A, ws, None) == INVALID  # half a gather
+    assert s(A, 1, 1, 1024, 1, nb, A, A + 8, None, None, BF16, 64, None, None, A, ws, None) == ALIGN
+    assert s(A, 0, 1, 1024, 1, nb, A, None, None, None, BF16, 64, None, None, None, 0, None) == OK
 
 
 def test_attend_rejects_bad_arguments_before_launch(lib):
@@ -116,8 +121,11 @@ def test_binding_refuses_host_tensors():
 
 
 def test_sort_workspace_formula_bounds(lib):
+    # whole segments in one CTA need none
+    for (B, H, L, nr, nb) in [(8, 8, 65536, 8, 1024), (1, 1, 1024, 1, 16), (8, 8, 16384, 4, 256)]:
+        assert lib.lsh_sort_workspace_bytes(B, H, L, nr, nb) == 0
     # bucket-major per-tile counters: at most 4 bytes per element plus 4 per bucket per segment
-    for (B, H, L, nr, nb) in [(8, 8, 65536, 8, 1024), (1, 8, 1 << 20, 4, 16384), (1, 1, 1024, 1, 16)]:
+    for (B, H, L, nr, nb) in [(1, 8, 1 << 20, 4, 16384), (1, 1, 1024, 1, 2048), (2, 2, 70000, 2, 64)]:
         ws = lib.lsh_sort_workspace_bytes(B, H, L, nr, nb)
         segs = B * H * nr
         assert 0 < ws <= 4 * segs * (L + nb) + 4 * segs * nb

@@ -153,12 +153,14 @@ sort_scatter_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
   }
 }
 
-// Whole-segment sort in one CTA (L <= 65536, n_buckets <= 1024): the bucket
-// ids of the segment are cached in shared memory as uint16, each of the 16
-// warps counts a contiguous range into its own histogram, the CTA turns the
-// (bucket, warp) counts into exclusive offsets (bucket-major, so warp ranges
-// stay in position order inside a bucket), and each warp then places its range
-// in order with the same warp-match ranking as sort_scatter_kernel.
+// Whole-segment sort in one CTA (L <= 65536, n_buckets <= 1024): each of the
+// 16 warps counts a contiguous range of the segment into its own histogram, the
+// CTA turns the (bucket, warp) counts into exclusive offsets (bucket-major, so
+// warp ranges stay in position order inside a bucket), and each warp then
+// places its range in order with the warp-match ranking of
+// sort_scatter_kernel.  The permutation is built in shared memory as uint16
+// (positions < 65536) and written out with coalesced stores; the inverse is
+// written directly (its writes are already in position order).
 constexpr int kSegWarps = 16;
 constexpr int kSegMaxL = 65536;
 constexpr int kSegMaxBuckets = 1024;
@@ -167,7 +169,7 @@ __host__ __device__ inline size_t sort_segment_smem(int L, int n_buckets) {
   return (size_t)kSegWarps * n_buckets * 4      // per-warp histograms / offsets
          + (size_t)kSegMaxBuckets * 4           // bucket totals / bases
          + 32 * 4                               // warp sums of the scan
-         + (((size_t)L * 2 + 15) & ~(size_t)15);  // cached bucket ids
+         + (((size_t)L * 2 + 15) & ~(size_t)15);  // the permutation, uint16
 }
 
 __global__ void __launch_bounds__(kSegWarps * 32)
@@ -177,26 +179,21 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
   uint32_t* hist = sm_u32;                          // [kSegWarps][n_buckets]
   uint32_t* tot = hist + kSegWarps * n_buckets;     // [n_buckets]
   uint32_t* ws = tot + kSegMaxBuckets;              // [32]
-  uint16_t* ids = reinterpret_cast<uint16_t*>(ws + 32);  // [L]
+  uint16_t* pm = reinterpret_cast<uint16_t*>(ws + 32);  // [L] sorted slot -> position
   const long long seg = blockIdx.x;
   const int32_t* src = buckets + seg * L;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int per_warp = (L + kSegWarps - 1) / kSegWarps;
+  const int per_warp = (((L + kSegWarps - 1) / kSegWarps) + 31) & ~31;
   const int lo = min(L, warp * per_warp), hi = min(L, lo + per_warp);
 
   for (int i = threadIdx.x; i < kSegWarps * n_buckets; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  // 1. per-warp counts of a contiguous range; ids cached (out-of-range ids: 0xFFFF, skipped)
+  // 1. per-warp counts of a contiguous range (out-of-range ids are skipped)
   uint32_t* my = hist + warp * n_buckets;
   for (int i = lo + lane; i < hi; i += 32) {
-    int b = src[i];
-    if ((unsigned)b >= (unsigned)n_buckets) {
-      record_error(LSH_ERR_INVALID_ARG);
-      b = 0xFFFF;
-    } else {
-      atomicAdd(&my[b], 1u);
-    }
-    ids[i] = (uint16_t)b;
+    const int b = src[i];
+    if ((unsigned)b >= (unsigned)n_buckets) record_error(LSH_ERR_INVALID_ARG);
+    else atomicAdd(&my[b], 1u);
   }
   __syncthreads();
   // 2a. within each bucket, exclusive offsets over the warps (in warp = position order)
@@ -245,14 +242,13 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
     for (int w = 0; w < kSegWarps; ++w) hist[w * n_buckets + b] += base;
   }
   __syncthreads();
-  // 3. stable placement of the warp's range
-  int32_t* dst = perm + seg * L;
+  // 3. stable placement of the warp's range (ids re-read, now from L2)
   int32_t* idst = inv ? inv + seg * L : nullptr;
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int base = lo; base < hi; base += 32) {
     const int i = base + lane;
-    const int b = i < hi ? (int)ids[i] : 0xFFFF;
-    const bool valid = b < n_buckets;
+    const int b = i < hi ? src[i] : -1;
+    const bool valid = (unsigned)b < (unsigned)n_buckets;
     const unsigned vmask = __ballot_sync(0xffffffffu, valid);
     unsigned peers = 0;
     uint32_t slot = 0;
@@ -264,10 +260,18 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
     if (valid && (peers & lt_mask) == 0) my[b] += __popc(peers);
     __syncwarp();
     if (valid) {
-      dst[slot] = i;
+      pm[slot] = (uint16_t)i;
       if (idst) idst[i] = (int32_t)slot;
     }
   }
+  __syncthreads();
+  // 4. coalesced write of the permutation.  After placement the last warp's
+  //    offset of the last bucket is the end of that bucket, i.e. the number of
+  //    valid ids; slots past it (left by out-of-range ids) stay as they were.
+  const uint32_t n_valid = hist[(kSegWarps - 1) * n_buckets + n_buckets - 1];
+  int32_t* dst = perm + seg * L;
+  for (int s = threadIdx.x; s < L; s += blockDim.x)
+    if ((uint32_t)s < n_valid) dst[s] = pm[s];
 }
 
 // Gather of sorted rows: dst[seg][s][:] = src[bh][perm[seg][s]][:], 16 B per thread.

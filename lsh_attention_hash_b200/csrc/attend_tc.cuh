@@ -25,7 +25,8 @@
 //              with 16-byte cp.async copies (32 lanes generate addresses in
 //              parallel; many small TMA row gathers were issue-bound) straight
 //              into 128-byte-swizzled K-major UMMA tiles, in a ring of three
-//              128-row slots (warp w copies rows 64w..64w+63 of a slot);
+//              128-row slots (warp w copies rows 64w..64w+63 of a slot); they
+//              also prefetch the rows of the fill two steps ahead into L2;
 //   warp 2     TMEM owner and single-thread UMMA issuer; it never blocks on
 //              one step while another step's UMMA could go (S of step t+1 and
 //              PV of step t are issued in whichever order they become ready);
@@ -340,25 +341,59 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
 
   if (warp < 2) {
     // ------------------------------------------------------------ producers
+    // Fills F (gathered now), F+1 (positions loaded), F+2 (rows warmed in L2 with
+    // per-line prefetches now; positions loaded one iteration earlier), F+3
+    // (positions loading).  The gathers are latency-bound and shared memory holds
+    // one fill in flight, so rows that reach L2 early shorten the next gathers.
     const int pw = warp;
     uint32_t f = 0;
-    FillIter fi;
-    fi.init(p);
-    int pos[2] = {0, 0};
-    if (fi.valid) fill_positions(p, fi.get(p), pw, pos);
-    while (fi.valid) {
-      const Fill cur = fi.get(p);
-      FillIter nx = fi;
-      nx.advance(p);
-      int npos[2] = {0, 0};
-      if (nx.valid) fill_positions(p, nx.get(p), pw, npos);  // in flight during the wait
+    FillIter it0, it1, it2, it3;
+    it0.init(p);
+    it1 = it0;
+    if (it1.valid) it1.advance(p);
+    it2 = it1;
+    if (it2.valid) it2.advance(p);
+    it3 = it2;
+    if (it3.valid) it3.advance(p);
+    int pos0[2] = {0, 0}, pos1[2] = {0, 0}, pos2[2] = {0, 0};
+    if (it0.valid) fill_positions(p, it0.get(p), pw, pos0);
+    if (it1.valid) fill_positions(p, it1.get(p), pw, pos1);
+    if (it2.valid) fill_positions(p, it2.get(p), pw, pos2);
+    while (it0.valid) {
+      int pos3[2] = {0, 0};
+      if (it3.valid) fill_positions(p, it3.get(p), pw, pos3);
+      if (it2.valid) {
+        const Fill pf = it2.get(p);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int i = 64 * pw + 32 * k + lane;
+          if (i >= pf.row0 && i < pf.row0 + pf.nrows) {
+            const int chunk = (i - pf.row0) < 64 ? pf.cA : pf.cB;
+            const long long g = p.sorted_input ? pf.seg * p.L + chunk * kC + (i & 63)
+                                               : (pf.seg / p.n_rounds) * p.L + pos2[k];
+#pragma unroll
+            for (int ln = 0; ln < D * 2; ln += 128) {
+              tc::prefetch_l2_line(p.qk + g * D * 2 + ln);
+              tc::prefetch_l2_line(p.v + g * D * 2 + ln);
+            }
+          }
+        }
+      }
+      const Fill cur = it0.get(p);
       const int slot = f % kSlots;
       if (!warp_wait(&empty[slot], ((f / kSlots) & 1) ^ 1, abort_flag)) break;
-      producer_fill<D>(p, smem, &full[slot], slot, cur, pw, pos);
+      producer_fill<D>(p, smem, &full[slot], slot, cur, pw, pos0);
       ++f;
-      fi = nx;
-      pos[0] = npos[0];
-      pos[1] = npos[1];
+      it0 = it1;
+      it1 = it2;
+      it2 = it3;
+      if (it3.valid) it3.advance(p);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        pos0[k] = pos1[k];
+        pos1[k] = pos2[k];
+        pos2[k] = pos3[k];
+      }
     }
     // never leave with copies in flight
     asm volatile("cp.async.wait_all;" ::: "memory");

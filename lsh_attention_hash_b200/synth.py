@@ -55,6 +55,9 @@ WORKLOADS = {
     "skewed16k": Workload("skewed16k", 8, 8, 16384, 128, "bf16", 256, 64, 4, qk_kind="clusters"),
     # 8 x 8 x 65536 x 128 bf16, 1024 buckets, 8 rounds (64K char-LM shaped)
     "64k": Workload("64k", 8, 8, 65536, 128, "bf16", 1024, 64, 8),
+    # 1 x 8 x 65536 x 128 bf16, 1024 buckets, 8 rounds: the 64K workload at batch 1
+    # (profiling captures at the real per-slice shape; QK 128 MB, still larger than L2)
+    "64k_b1": Workload("64k_b1", 1, 8, 65536, 128, "bf16", 1024, 64, 8),
     # 8 x 8 x 16384 x 128 bf16, 256 buckets, 8 rounds: the 64K workload at a quarter of the
     # length (profiling captures: inputs still larger than L2, a few GB on the device)
     "16k": Workload("16k", 8, 8, 16384, 128, "bf16", 256, 64, 8),

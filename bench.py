@@ -81,8 +81,9 @@ def source_digest(files):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(stage):
-    """DRAM bytes per launch of `stage` from the committed ncu summary, or None.
+def recorded_traffic(stage, workload):
+    """DRAM bytes per launch of `stage` on `workload` from the committed ncu
+    summary (profiles/traffic.json), or None.
 
     The summary stores a digest of the kernel sources it was taken on; a
     changed kernel invalidates it.
@@ -92,14 +93,14 @@ def recorded_traffic(stage):
         return None
     with open(path) as f:
         rec = json.load(f).get(stage)
-    if not rec:
+    if not rec or workload not in rec.get("per_launch_bytes", {}):
         return None
     try:
         if source_digest(rec["sources"]) != rec["digest"]:
             return None
     except OSError:
         return None
-    return rec["dram_bytes_per_launch"]
+    return rec["per_launch_bytes"][workload]
 
 
 class ClockSampler:
@@ -344,7 +345,7 @@ def run_ours(args, w, rank, world, local_rank):
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": workload_config(w),
         "roofline": {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": recorded_traffic(dominant),
+                     "frac": achieved / peak, "traffic": recorded_traffic(dominant, args.workload),
                      "peak_source": peak_src + (", sustained tensor peak" if bound == "tensor" else "")},
         "step_roofline": {"t_roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_step,
                           "alg_bytes": alg["total_bytes"], "attn_flops": alg["attn_flops"],

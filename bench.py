@@ -332,6 +332,9 @@ def run_ours(args, w, rank, world, local_rank):
         peak = peaks["bf16_tflops_sustained"]
         unit = "TFLOP/s"
     t_roof = max(alg["total_bytes"] / (peaks["hbm_gbs"] * 1e9), alg["attn_flops"] / (peaks["bf16_tflops"] * 1e12))
+    # method-inclusive bound: the hash GEMM's FLOPs added to the attention FLOPs
+    t_roof_hash = max(alg["total_bytes"] / (peaks["hbm_gbs"] * 1e9),
+                      (alg["attn_flops"] + alg["hash"]["flops"]) / (peaks["bf16_tflops"] * 1e12))
     if w.L <= 65536 and w.n_buckets <= 1024:
         sort_launches = 1                                  # one CTA per segment
     else:
@@ -348,7 +351,10 @@ def run_ours(args, w, rank, world, local_rank):
                      "frac": achieved / peak, "traffic": recorded_traffic(dominant, args.workload),
                      "peak_source": peak_src + (", sustained tensor peak" if bound == "tensor" else "")},
         "step_roofline": {"t_roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_step,
+                          "t_roofline_hash_inclusive_ms": t_roof_hash * 1e3,
+                          "frac_hash_inclusive": t_roof_hash * 1e3 / ms_step,
                           "alg_bytes": alg["total_bytes"], "attn_flops": alg["attn_flops"],
+                          "hash_flops": alg["hash"]["flops"],
                           "note": "max(alg. bytes / HBM peak, chunk-attention FLOPs / bf16 peak) over measured step time"},
         "stage_ms": per_stage,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -60,6 +60,7 @@ struct Params {
   int nchunks;         // half / NC
   int per_round;       // CTAs per round
   long long n_tiles;
+  uint32_t key_mask;   // 0x7FFFFFF0: |p| without its 4 lowest mantissa bits
 };
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -82,13 +83,16 @@ struct RowState {
   float v1, v2;     // exact top-two |p| (near-tie flag only)
 };
 
+// `mask` is 0x7FFFFFF0, passed in at run time: with the mask in a register
+// (or constant operand) and 15 - j as the immediate, each key is a single
+// three-input logic operation instead of two.
 template <bool FLAG>
-__device__ __forceinline__ void process16(RowState& st, const uint32_t* raw, int g) {
+__device__ __forceinline__ void process16(RowState& st, const uint32_t* raw, int g, uint32_t mask) {
   float key[16], val[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     val[j] = __uint_as_float(raw[j]);
-    key[j] = __uint_as_float((raw[j] & 0x7FFFFFF0u) | (uint32_t)(15 - j));
+    key[j] = __uint_as_float((raw[j] & mask) | (uint32_t)(15 - j));
   }
   const float gk = max16(key);
   const float gr = max16(val);
@@ -236,8 +240,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
           tc::tmem_ld32(lane_base + tmem + b * NC + col, raw);
           tc::tmem_wait_ld();
           const int g = (c * NC + col) >> 4;
-          process16<FLAG>(st, raw, g);
-          process16<FLAG>(st, raw + 16, g + 1);
+          process16<FLAG>(st, raw, g, p.key_mask);
+          process16<FLAG>(st, raw + 16, g + 1, p.key_mask);
         }
         tc::tc_fence_before();
         tc::mbar_arrive(&acc_empty[b]);

@@ -123,6 +123,7 @@ lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, in
   p.nchunks = half / NC;
   p.n_tiles = (rows + kRows - 1) / kRows;
   p.per_round = (int)std::max<long long>(1, std::min<long long>(sms / n_rounds, p.n_tiles));
+  p.key_mask = 0x7FFFFFF0u;
   const unsigned grid = (unsigned)(p.per_round * n_rounds);
   auto kfn = hash_tc_kernel<D, NC, FLAG, SPLIT>;
   const int smem = (int)Layout<D>::smem_bytes(half);

@@ -190,10 +190,20 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
   __syncthreads();
   // 1. per-warp counts of a contiguous range (out-of-range ids are skipped)
   uint32_t* my = hist + warp * n_buckets;
-  for (int i = lo + lane; i < hi; i += 32) {
-    const int b = src[i];
-    if ((unsigned)b >= (unsigned)n_buckets) record_error(LSH_ERR_INVALID_ARG);
-    else atomicAdd(&my[b], 1u);
+  for (int base = lo; base < hi; base += 128) {
+    int bq[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = base + 32 * k + lane;
+      bq[k] = i < hi ? src[i] : 0x7fffffff;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (base + 32 * k + lane >= hi) continue;
+      const int b = bq[k];
+      if ((unsigned)b >= (unsigned)n_buckets) record_error(LSH_ERR_INVALID_ARG);
+      else atomicAdd(&my[b], 1u);
+    }
   }
   __syncthreads();
   // 2a. within each bucket, exclusive offsets over the warps (in warp = position order)
@@ -242,26 +252,36 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
     for (int w = 0; w < kSegWarps; ++w) hist[w * n_buckets + b] += base;
   }
   __syncthreads();
-  // 3. stable placement of the warp's range (ids re-read, now from L2)
+  // 3. stable placement of the warp's range (ids re-read, now from L2, four groups
+  //    of 32 at a time so that the loads overlap)
   int32_t* idst = inv ? inv + seg * L : nullptr;
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = lo; base < hi; base += 32) {
-    const int i = base + lane;
-    const int b = i < hi ? src[i] : -1;
-    const bool valid = (unsigned)b < (unsigned)n_buckets;
-    const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-    unsigned peers = 0;
-    uint32_t slot = 0;
-    if (valid) {
-      peers = __match_any_sync(vmask, b);
-      slot = my[b] + __popc(peers & lt_mask);
+  for (int base = lo; base < hi; base += 128) {
+    int bq[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = base + 32 * k + lane;
+      bq[k] = i < hi ? src[i] : -1;
     }
-    __syncwarp();
-    if (valid && (peers & lt_mask) == 0) my[b] += __popc(peers);
-    __syncwarp();
-    if (valid) {
-      pm[slot] = (uint16_t)i;
-      if (idst) idst[i] = (int32_t)slot;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = base + 32 * k + lane;
+      const int b = bq[k];
+      const bool valid = (unsigned)b < (unsigned)n_buckets;
+      const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+      unsigned peers = 0;
+      uint32_t slot = 0;
+      if (valid) {
+        peers = __match_any_sync(vmask, b);
+        slot = my[b] + __popc(peers & lt_mask);
+      }
+      __syncwarp();
+      if (valid && (peers & lt_mask) == 0) my[b] += __popc(peers);
+      __syncwarp();
+      if (valid) {
+        pm[slot] = (uint16_t)i;
+        if (idst) idst[i] = (int32_t)slot;
+      }
     }
   }
   __syncthreads();

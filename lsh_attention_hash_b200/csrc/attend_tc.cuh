@@ -57,6 +57,8 @@ constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBufCols = 256;  // one step buffer
 constexpr uint32_t kOOff = 96;      // O columns inside a step buffer
+template <int D>
+__host__ __device__ constexpr uint32_t lr_col() { return kOOff + D; }
 
 template <int D>
 struct Layout {
@@ -65,7 +67,8 @@ struct Layout {
   static constexpr uint32_t kSlotBytes = kHalves * kHalfBytes; // one tensor, one slot
   static constexpr uint32_t kQK = 0;
   static constexpr uint32_t kV = kSlots * kSlotBytes;
-  static constexpr uint32_t kPerm = 2 * kSlots * kSlotBytes;        // int32 [kSlots][128]
+  static constexpr uint32_t kOnes = 2 * kSlots * kSlotBytes;        // 16 x 128 B of bf16 1.0 (row sums)
+  static constexpr uint32_t kPerm = kOnes + 16 * 128;               // int32 [kSlots][128]
   static constexpr uint32_t kColMul = kPerm + kSlots * kRows * 4;   // float [kSlots][128]
   static constexpr uint32_t kBar = kColMul + kSlots * kRows * 4;
   // full[3] empty[3] cm_full[3] s_full[2] p_ready[2] o_full[2] buf_empty[2] done
@@ -101,7 +104,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   if (__all_sync(0xffffffffu, done)) return true;
   const unsigned long long t0 = tc::globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (!done) done = tc::mbar_try_wait(bar, parity);
+    if (!done) done = tc::mbar_try_wait_sleep(bar, parity, 20000u);
     if (__all_sync(0xffffffffu, done)) return true;
     if ((i & 31u) == 0) {
       int bail = 0;
@@ -115,6 +118,24 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
         }
       }
       if (__shfl_sync(0xffffffffu, bail, 0)) return false;
+    }
+  }
+}
+
+// Single-thread bounded wait for an UMMA issuer: sleeps in the barrier wait,
+// gives up on abort or after kWaitNs.
+__device__ __forceinline__ bool issuer_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (tc::mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = tc::globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (tc::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((i & 7u) == 0) {
+      if (*abort_flag) return false;
+      if (tc::globaltimer() - t0 > tc::kWaitNs) {
+        *abort_flag = 1;
+        record_error(LSH_ERR_TIMEOUT);
+        return false;
+      }
     }
   }
 }
@@ -297,6 +318,103 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
   return colscale / fmaxf(sqrtf(ss), 1e-12f);
 }
 
+// One pass of the softmax over a row's 128 keys (four groups of 32 S columns,
+// the next group's TMEM load in flight while the current one is processed):
+// w = 2^(S * colmul - m) in fp32 (self masked, a missing previous chunk dead),
+// l += w, and the weights go to P as bf16 pairs right away: P's group g lands
+// on S columns whose values this row has already consumed.
+template <int D>
+__device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint32_t pcol, const float* cm_lo,
+                                             const float* cm_hi, int g_first, int g_self, int lane, int self_mask,
+                                             float m, float& l) {
+  uint32_t ra[32], rb[32];
+  tc::tmem_ld32(sbuf + scol, ra);
+  tc::tmem_wait_ld_regs(ra);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint32_t(&cur)[32] = (g & 1) ? rb : ra;
+    uint32_t(&nxt)[32] = (g & 1) ? ra : rb;
+    if (g < 3) tc::tmem_ld32(sbuf + scol + 32 * (g + 1), nxt);
+    const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
+    const bool dead = g < g_first;
+    uint32_t w16[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float v0 = __uint_as_float(cur[e]) * cm[e];
+      float v1 = __uint_as_float(cur[e + 1]) * cm[e + 1];
+      if (g == g_self && self_mask) {
+        if (e == lane) v0 = -INFINITY;
+        if (e + 1 == lane) v1 = -INFINITY;
+      }
+      const float a = dead ? 0.f : tc::ex2_approx(v0 - m);
+      const float c = dead ? 0.f : tc::ex2_approx(v1 - m);
+      l += a + c;
+      w16[e >> 1] = tc::pack_bf16x2(a, c);
+    }
+    tc::tmem_st16(sbuf + pcol + 16 * g, w16);
+    if (g < 3) tc::tmem_wait_ld_regs(nxt);
+  }
+}
+
+// Exact maximum of a row's scaled logits (self excluded while it has other keys).
+__device__ __forceinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const float* cm_lo, const float* cm_hi,
+                                               int g_first, int g_self, int lane, int self_mask) {
+  float m = -INFINITY;
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    uint32_t raw[32];
+    tc::tmem_ld32(sbuf + scol + 32 * g, raw);
+    tc::tmem_wait_ld_regs(raw);
+    if (g < g_first) continue;
+    const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      float v = __uint_as_float(raw[e]) * cm[e];
+      if (g == g_self && self_mask && e == lane) v = -INFINITY;
+      m = fmaxf(m, v);
+    }
+  }
+  return m;
+}
+
+// Rebuilds the row's 128 S values (q . k, fp32) in TMEM from the QK tiles in
+// shared memory: row r of the pair slot against keys [prev chunk rows 64..127,
+// pair rows 0..63] (rows 0..63) or [pair rows 0..127] (rows 64..127).  Only
+// the rare underflow path runs this.
+template <int D>
+__device__ __noinline__ void restore_s(const uint8_t* smem, uint32_t sbuf, uint32_t scol, int sp, int sc, int r,
+                                       bool low) {
+  using Lay = Layout<D>;
+  const uint8_t* qs = smem + Lay::kQK + sc * Lay::kSlotBytes;
+  const uint8_t* ps = smem + Lay::kQK + sp * Lay::kSlotBytes;
+  tc::tmem_wait_st();  // P stores of the first pass land before S is rewritten
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    uint32_t out[32];
+#pragma unroll 1
+    for (int e = 0; e < 32; ++e) {
+      const int k = 32 * g + e;  // key of the row's window
+      const uint8_t* kt = low ? (k < 64 ? ps : qs) : qs;
+      const int kr = low ? (k < 64 ? 64 + k : k - 64) : k;
+      float acc = 0.f;
+#pragma unroll 1
+      for (int h = 0; h < Lay::kHalves; ++h) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float x[8], y[8];
+          load8(reinterpret_cast<const __nv_bfloat16*>(qs + h * Lay::kHalfBytes + r * 128 + ((c ^ (r & 7)) << 4)), x);
+          load8(reinterpret_cast<const __nv_bfloat16*>(kt + h * Lay::kHalfBytes + kr * 128 + ((c ^ (kr & 7)) << 4)), y);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc = fmaf(x[i], y[i], acc);
+        }
+      }
+      out[e] = __float_as_uint(acc);
+    }
+    tc::tmem_st32(sbuf + scol + 32 * g, out);
+  }
+  tc::tmem_wait_st();
+}
+
 template <int D, typename TO>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) {
   using Lay = Layout<D>;
@@ -329,9 +447,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       tc::mbar_init(&o_full[i], 1);
       tc::mbar_init(&buf_empty[i], 128);
     }
-    tc::mbar_init(done_bar, 1);
+    tc::mbar_init(done_bar, 2);
     *abort_flag = 0;
     tc::fence_mbar_init();
+  }
+  {
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + Lay::kOnes);
+    for (int i = threadIdx.x; i < 16 * 128 / 4; i += kThreads) ones[i] = 0x3F803F80u;  // two bf16 1.0
+    tc::fence_proxy_async_smem();
   }
   if (warp == 2) tc::tmem_alloc(tmem_holder, kTmemCols);
   tc::tc_fence_before();
@@ -397,46 +520,49 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
     }
     // never leave with copies in flight
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ UMMA issuer
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ UMMA issuers
+    // warp 2 lane 0 issues the S UMMAs, warp 3 lane 0 the PV UMMAs; each blocks
+    // on one barrier at a time (the thread sleeps in the barrier wait instead
+    // of polling).  tcgen05.commit tracks the issuing thread's own UMMAs.
     if (lane == 0) {
-      const uint32_t id_prev = tc::idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t id_pair = tc::idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t id_pv = tc::idesc_bf16_f32(128, D, 0, 1);
       const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK);
       const uint32_t v0 = tc::smem_u32(smem + Lay::kV);
-      StepIter si, pi;  // next step to receive S, next step to receive PV
-      si.init(p);
-      pi.init(p);
-      unsigned long long t_idle = 0;
-      while (pi.valid) {
-        bool progress = false;
-        if (si.valid && si.t < pi.t + 2) {
-          const uint32_t fp = si.f - 1, fc = si.f;
-          if (tc::mbar_try_wait(&full[fp % kSlots], (fp / kSlots) & 1) &&
-              tc::mbar_try_wait(&full[fc % kSlots], (fc / kSlots) & 1) &&
-              tc::mbar_try_wait(&buf_empty[si.t & 1], ((si.t >> 1) & 1) ^ 1)) {
-            tc::tc_fence_after();
-            const uint32_t sbuf = tmem + (si.t & 1) * kBufCols;
-            const uint32_t qk_c = qk0 + (fc % kSlots) * Lay::kSlotBytes;
-            const uint32_t qk_p = qk0 + (fp % kSlots) * Lay::kSlotBytes + 64 * 128;  // rows 64..127
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t koff = (kk >> 2) * Lay::kHalfBytes + (kk & 3) * 32;
-              const uint64_t a = tc::sdesc_sw128(qk_c + koff, 16, 1024);
-              const uint64_t bp = tc::sdesc_sw128(qk_p + koff, 16, 1024);
-              tc::umma_ss(sbuf, a, bp, id_prev, kk > 0);
-              tc::umma_ss(sbuf + 64, a, a, id_pair, kk > 0);
-            }
-            tc::umma_commit(&s_full[si.t & 1]);
-            si.advance(p);
-            progress = true;
-          }
-        }
-        if (pi.t < si.t && tc::mbar_try_wait(&p_ready[pi.t & 1], (pi.t >> 1) & 1)) {
+      StepIter it;
+      it.init(p);
+      if (warp == 2) {
+        const uint32_t id_prev = tc::idesc_bf16_f32(128, 64, 0, 0);
+        const uint32_t id_pair = tc::idesc_bf16_f32(128, 128, 0, 0);
+        while (it.valid) {
+          const uint32_t fp = it.f - 1, fc = it.f;
+          if (!issuer_wait(&full[fp % kSlots], (fp / kSlots) & 1, abort_flag) ||
+              !issuer_wait(&full[fc % kSlots], (fc / kSlots) & 1, abort_flag) ||
+              !issuer_wait(&buf_empty[it.t & 1], ((it.t >> 1) & 1) ^ 1, abort_flag))
+            break;
           tc::tc_fence_after();
-          const uint32_t sbuf = tmem + (pi.t & 1) * kBufCols;
-          const uint32_t sp = (pi.f - 1) % kSlots, sc = pi.f % kSlots;
+          const uint32_t sbuf = tmem + (it.t & 1) * kBufCols;
+          const uint32_t qk_c = qk0 + (fc % kSlots) * Lay::kSlotBytes;
+          const uint32_t qk_p = qk0 + (fp % kSlots) * Lay::kSlotBytes + 64 * 128;  // rows 64..127
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * Lay::kHalfBytes + (kk & 3) * 32;
+            const uint64_t a = tc::sdesc_sw128(qk_c + koff, 16, 1024);
+            const uint64_t bp = tc::sdesc_sw128(qk_p + koff, 16, 1024);
+            tc::umma_ss(sbuf, a, bp, id_prev, kk > 0);
+            tc::umma_ss(sbuf + 64, a, a, id_pair, kk > 0);
+          }
+          tc::umma_commit(&s_full[it.t & 1]);
+          it.advance(p);
+        }
+      } else {
+        const uint32_t id_pv = tc::idesc_bf16_f32(128, D, 0, 1);
+        const uint32_t id_lr = tc::idesc_bf16_f32(128, 16, 0, 1);
+        const uint64_t ones_desc = tc::sdesc_sw128(tc::smem_u32(smem + Lay::kOnes), Lay::kHalfBytes, 1024);
+        while (it.valid) {
+          if (!issuer_wait(&p_ready[it.t & 1], (it.t >> 1) & 1, abort_flag)) break;
+          tc::tc_fence_after();
+          const uint32_t sbuf = tmem + (it.t & 1) * kBufCols;
+          const uint32_t sp = (it.f - 1) % kSlots, sc = it.f % kSlots;
 #pragma unroll
           for (int kk = 0; kk < 12; ++kk) {
             const uint32_t vrow = kk < 4 ? v0 + sp * Lay::kSlotBytes + (64 + 16 * kk) * 128
@@ -444,23 +570,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
             const uint64_t b = tc::sdesc_sw128(vrow, Lay::kHalfBytes, 1024);
             tc::umma_ts(sbuf + kOOff, sbuf + kk * 8, b, id_pv, kk > 0);
           }
-          tc::umma_commit(&o_full[pi.t & 1]);
+#pragma unroll
+          for (int kk = 0; kk < 12; ++kk)  // every 16-key step reads the same 16 rows of ones
+            tc::umma_ts(sbuf + lr_col<D>(), sbuf + kk * 8, ones_desc, id_lr, kk > 0);
+          tc::umma_commit(&o_full[it.t & 1]);
           tc::umma_commit(&empty[sp]);
-          if (pi.last_of_unit()) tc::umma_commit(&empty[sc]);
-          pi.advance(p);
-          progress = true;
-        }
-        if (progress) {
-          t_idle = 0;
-        } else {
-          const unsigned long long now = tc::globaltimer();
-          if (t_idle == 0) {
-            t_idle = now;
-          } else if (now - t_idle > tc::kWaitNs || *abort_flag) {
-            if (!*abort_flag) record_error(LSH_ERR_TIMEOUT);
-            *abort_flag = 1;
-            break;
-          }
+          if (it.last_of_unit()) tc::umma_commit(&empty[sc]);
+          it.advance(p);
         }
       }
       tc::umma_commit(done_bar);
@@ -518,60 +634,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       const int g_first = (low && it.j == 0) ? 2 : 0;  // chunk 0 has no previous chunk
       // shift: ||q|| * scale * log2(e) bounds every logit of the row (log2 domain)
       float m = diag * cm_own;
-      float l = 0.f;   // sum of the weights (log-sum-exp)
-      float lr = 0.f;  // sum of the bf16-rounded weights that P holds (normalises O)
-      uint32_t pk[64];  // the row's P, packed bf16 pairs, stored once the row sum is known to be safe
-      for (int attempt = 0; attempt < 2; ++attempt) {
+      float l = 0.f;  // sum of the weights (log-sum-exp); O is normalised by the rounded weights' sum
+      const uint32_t pcol = low ? 0 : 32;  // P column of the row's first key
+      softmax_pass<D>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l);
+      if (__any_sync(0xffffffffu, !(l > 1e-30f))) {
+        // the bound was too loose for some row of the warp (long query rows): S is
+        // rebuilt in TMEM from the rows in shared memory (P has overwritten part of
+        // it) and the warp's rows are redone with their exact maxima
+        restore_s<D>(smem, sbuf, scol, sp, sc, r, low);
+        m = exact_row_max(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask);
         l = 0.f;
-        lr = 0.f;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t raw[32];
-          tc::tmem_ld32(sbuf + scol + 32 * g, raw);
-          tc::tmem_wait_ld();
-          const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
-          const bool dead = g < g_first;
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float v0 = __uint_as_float(raw[e]) * cm[e];
-            float v1 = __uint_as_float(raw[e + 1]) * cm[e + 1];
-            if (g == g_self && p.self_mask) {
-              if (e == lane) v0 = -INFINITY;
-              if (e + 1 == lane) v1 = -INFINITY;
-            }
-            const float a = dead ? 0.f : tc::ex2_approx(v0 - m);
-            const float c = dead ? 0.f : tc::ex2_approx(v1 - m);
-            l += a + c;
-            const uint32_t w = tc::pack_bf16x2(a, c);
-            lr += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
-            pk[16 * g + (e >> 1)] = w;
-          }
-        }
-        if (l > 1e-30f) break;
-        // the bound was too loose (long query rows): redo with the exact maximum; S is intact
-        // because P has not been written yet
-        m = -INFINITY;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t raw[32];
-          tc::tmem_ld32(sbuf + scol + 32 * g, raw);
-          tc::tmem_wait_ld();
-          if (g < g_first) continue;
-          const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float v = __uint_as_float(raw[e]) * cm[e];
-            if (g == g_self && p.self_mask && e == lane) v = -INFINITY;
-            m = fmaxf(m, v);
-          }
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t w16[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) w16[e] = pk[16 * g + e];
-        tc::tmem_st16(sbuf + (low ? 16 * g : 32 + 16 * g), w16);
+        softmax_pass<D>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l);
       }
       {
         uint32_t z[32];
@@ -586,7 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       ok = warp_wait(&o_full[b], (t >> 1) & 1, abort_flag);
       if (!ok) break;
       tc::tc_fence_after();
-      const float inv_l = 1.f / lr;  // O = sum p~ v / sum p~: a convex combination of the values
+      // O = sum p~ v / sum p~ (p~ the bf16 weights in P): a convex combination of the values
+      const float inv_l = 1.f / __uint_as_float(tc::tmem_ld1(sbuf + lr_col<D>()));
       TO* dst = reinterpret_cast<TO*>(p.out) + (it.seg * p.L + pos) * (long long)D;
 #pragma unroll
       for (int g = 0; g < D / 32; ++g) {

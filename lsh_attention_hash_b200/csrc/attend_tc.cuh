@@ -27,10 +27,8 @@
 //              into 128-byte-swizzled K-major UMMA tiles, in a ring of three
 //              128-row slots (warp w copies rows 64w..64w+63 of a slot); they
 //              also prefetch the rows of the fill two steps ahead into L2;
-//   warp 2     TMEM owner and single-thread UMMA issuer; it never blocks on
-//              one step while another step's UMMA could go (S of step t+1 and
-//              PV of step t are issued in whichever order they become ready);
-//   warp 3     idle;
+//   warp 2     TMEM owner; its lane 0 issues the S UMMAs, lane 0 of warp 3
+//              the PV UMMAs, each sleeping on one barrier at a time;
 //   warps 4-7  softmax + epilogue of the even steps, warps 8-11 of the odd
 //              steps (one query row per thread), so that one step's softmax
 //              overlaps the other step's UMMAs, loads and stores.
@@ -39,9 +37,13 @@
 // publishes the key multiplier scale * log2(e) / ||k||; the rows of a unit's
 // leading chunk (which no earlier step of this CTA saw) are measured directly
 // from shared memory.  The softmax uses the Cauchy-Schwarz bound
-// q.k / ||k|| <= ||q|| as its shift (one pass over S); a row whose sum would
-// underflow under that shift is redone with its exact maximum.
-// TMEM: two step buffers of 256 columns (S: 192 fp32, P: first 96, O: 96..96+D).
+// q.k / ||k|| <= ||q|| as its shift (one pass over S, P written back as it
+// goes); a row whose sum would underflow under that shift has its S rebuilt
+// from shared memory and is redone with its exact maximum.  O is normalised by
+// the sum of the bf16 weights P holds, which 12 more UMMAs of P against a
+// tile of ones leave beside O.
+// TMEM: two step buffers of 256 columns (S: 192 fp32, P: first 96, O: 96..96+D,
+// row sums: 16 columns after O).
 // Every wait is bounded; a timeout unwinds the CTA cleanly.
 #pragma once
 

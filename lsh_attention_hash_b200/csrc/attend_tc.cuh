@@ -28,7 +28,7 @@
 //              128-row slots (warp w copies rows 64w..64w+63 of a slot); they
 //              also prefetch the rows of the fill two steps ahead into L2;
 //   warp 2     TMEM owner; its lane 0 issues the S UMMAs, lane 0 of warp 3
-//              the PV UMMAs, each sleeping on one barrier at a time;
+//              the PV UMMAs, each waiting on one barrier at a time;
 //   warps 4-7  softmax + epilogue of the even steps, warps 8-11 of the odd
 //              steps (one query row per thread), so that one step's softmax
 //              overlaps the other step's UMMAs, loads and stores.
@@ -124,13 +124,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Single-thread bounded wait for an UMMA issuer: sleeps in the barrier wait,
-// gives up on abort or after kWaitNs.
+// Single-thread bounded wait for an UMMA issuer (the barrier wait's own short
+// suspend; a longer suspend-time hint woke the issuers late): gives up on
+// abort or after kWaitNs.
 __device__ __forceinline__ bool issuer_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (tc::mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = tc::globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (tc::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (tc::mbar_try_wait(bar, parity)) return true;
     if ((i & 7u) == 0) {
       if (*abort_flag) return false;
       if (tc::globaltimer() - t0 > tc::kWaitNs) {
@@ -524,9 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ UMMA issuers
-    // warp 2 lane 0 issues the S UMMAs, warp 3 lane 0 the PV UMMAs; each blocks
-    // on one barrier at a time (the thread sleeps in the barrier wait instead
-    // of polling).  tcgen05.commit tracks the issuing thread's own UMMAs.
+    // warp 2 lane 0 issues the S UMMAs, warp 3 lane 0 the PV UMMAs; each waits
+    // on one barrier at a time.  tcgen05.commit tracks the issuing thread's own
+    // UMMAs.
     if (lane == 0) {
       const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK);
       const uint32_t v0 = tc::smem_u32(smem + Lay::kV);

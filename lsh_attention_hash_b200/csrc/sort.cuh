@@ -154,21 +154,24 @@ sort_scatter_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
 }
 
 // Whole-segment sort in one CTA (L <= 65536, n_buckets <= 1024): each of the
-// 16 warps counts a contiguous range of the segment into its own histogram, the
+// 32 warps counts a contiguous range of the segment into its own histogram, the
 // CTA turns the (bucket, warp) counts into exclusive offsets (bucket-major, so
 // warp ranges stay in position order inside a bucket), and each warp then
 // places its range in order with the warp-match ranking of
-// sort_scatter_kernel.  The permutation is built in shared memory as uint16
-// (positions < 65536) and written out with coalesced stores; the inverse is
-// written directly (its writes are already in position order).
-constexpr int kSegWarps = 16;
+// sort_scatter_kernel.  Counts, offsets and sorted slots are all below 65536,
+// so the histograms are uint16 (two buckets per 32-bit word for the counting
+// atomics; a warp counts at most 2048 ids, so no carry crosses into the
+// neighbour).  The permutation is built in shared memory as uint16 (positions
+// < 65536) and written out with coalesced stores; the inverse is written
+// directly (its writes are already in position order).
+constexpr int kSegWarps = 32;
 constexpr int kSegMaxL = 65536;
 constexpr int kSegMaxBuckets = 1024;
 
 __host__ __device__ inline size_t sort_segment_smem(int L, int n_buckets) {
-  return (size_t)kSegWarps * n_buckets * 4      // per-warp histograms / offsets
+  return (size_t)kSegWarps * ((n_buckets + 1) & ~1) * 2  // per-warp histograms / offsets, uint16
          + (size_t)kSegMaxBuckets * 4           // bucket totals / bases
-         + 32 * 4                               // warp sums of the scan
+         + 48 * 4                               // warp sums of the scan, count of invalid ids
          + (((size_t)L * 2 + 15) & ~(size_t)15);  // the permutation, uint16
 }
 
@@ -176,20 +179,23 @@ __global__ void __launch_bounds__(kSegWarps * 32)
 sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, int32_t* __restrict__ perm,
                     int32_t* __restrict__ inv) {
   extern __shared__ uint32_t sm_u32[];
-  uint32_t* hist = sm_u32;                          // [kSegWarps][n_buckets]
-  uint32_t* tot = hist + kSegWarps * n_buckets;     // [n_buckets]
-  uint32_t* ws = tot + kSegMaxBuckets;              // [32]
-  uint16_t* pm = reinterpret_cast<uint16_t*>(ws + 32);  // [L] sorted slot -> position
+  const int nbp = (n_buckets + 1) & ~1;             // row pitch (even: rows start on a 32-bit word)
+  uint16_t* hist = reinterpret_cast<uint16_t*>(sm_u32);  // [kSegWarps][nbp]
+  uint32_t* tot = sm_u32 + kSegWarps * nbp / 2;     // [n_buckets]
+  uint32_t* ws = tot + kSegMaxBuckets;              // [32] warp sums, [32] invalid ids
+  uint16_t* pm = reinterpret_cast<uint16_t*>(ws + 48);  // [L] sorted slot -> position
   const long long seg = blockIdx.x;
   const int32_t* src = buckets + seg * L;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int per_warp = (((L + kSegWarps - 1) / kSegWarps) + 31) & ~31;
   const int lo = min(L, warp * per_warp), hi = min(L, lo + per_warp);
 
-  for (int i = threadIdx.x; i < kSegWarps * n_buckets; i += blockDim.x) hist[i] = 0;
+  for (int i = threadIdx.x; i < kSegWarps * nbp / 2; i += blockDim.x) sm_u32[i] = 0;
+  if (threadIdx.x == 0) ws[32] = 0;
   __syncthreads();
   // 1. per-warp counts of a contiguous range (out-of-range ids are skipped)
-  uint32_t* my = hist + warp * n_buckets;
+  uint16_t* my = hist + warp * nbp;
+  uint32_t* my_words = sm_u32 + warp * nbp / 2;
   for (int base = lo; base < hi; base += 128) {
     int bq[4];
 #pragma unroll
@@ -201,8 +207,12 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
     for (int k = 0; k < 4; ++k) {
       if (base + 32 * k + lane >= hi) continue;
       const int b = bq[k];
-      if ((unsigned)b >= (unsigned)n_buckets) record_error(LSH_ERR_INVALID_ARG);
-      else atomicAdd(&my[b], 1u);
+      if ((unsigned)b >= (unsigned)n_buckets) {
+        record_error(LSH_ERR_INVALID_ARG);
+        atomicAdd(&ws[32], 1u);
+      } else {
+        atomicAdd(&my_words[b >> 1], 1u << (16 * (b & 1)));
+      }
     }
   }
   __syncthreads();
@@ -210,18 +220,17 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
   for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
     uint32_t run = 0;
     for (int w = 0; w < kSegWarps; ++w) {
-      const uint32_t c = hist[w * n_buckets + b];
-      hist[w * n_buckets + b] = run;
+      const uint32_t c = hist[w * nbp + b];
+      hist[w * nbp + b] = (uint16_t)run;  // < 65536: at most L - (this warp's count)
       run += c;
     }
     tot[b] = run;
   }
   __syncthreads();
-  // 2b. exclusive scan of the bucket totals (two buckets per thread)
+  // 2b. exclusive scan of the bucket totals (one bucket per thread)
   {
-    const int b0 = 2 * threadIdx.x;
-    const uint32_t t0 = b0 < n_buckets ? tot[b0] : 0u, t1 = b0 + 1 < n_buckets ? tot[b0 + 1] : 0u;
-    const uint32_t local = t0 + t1;
+    const int b0 = threadIdx.x;
+    const uint32_t local = b0 < n_buckets ? tot[b0] : 0u;
     uint32_t incl = local;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -243,13 +252,12 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
     __syncthreads();
     const uint32_t excl = ws[warp] + incl - local;
     if (b0 < n_buckets) tot[b0] = excl;
-    if (b0 + 1 < n_buckets) tot[b0 + 1] = excl + t0;
   }
   __syncthreads();
   // 2c. first sorted slot of (bucket, warp)
   for (int b = threadIdx.x; b < n_buckets; b += blockDim.x) {
     const uint32_t base = tot[b];
-    for (int w = 0; w < kSegWarps; ++w) hist[w * n_buckets + b] += base;
+    for (int w = 0; w < kSegWarps; ++w) hist[w * nbp + b] = (uint16_t)(hist[w * nbp + b] + base);  // a slot < L
   }
   __syncthreads();
   // 3. stable placement of the warp's range (ids re-read, now from L2, four groups
@@ -276,7 +284,7 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
         slot = my[b] + __popc(peers & lt_mask);
       }
       __syncwarp();
-      if (valid && (peers & lt_mask) == 0) my[b] += __popc(peers);
+      if (valid && (peers & lt_mask) == 0) my[b] = (uint16_t)(my[b] + __popc(peers));
       __syncwarp();
       if (valid) {
         pm[slot] = (uint16_t)i;
@@ -285,10 +293,9 @@ sort_segment_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, i
     }
   }
   __syncthreads();
-  // 4. coalesced write of the permutation.  After placement the last warp's
-  //    offset of the last bucket is the end of that bucket, i.e. the number of
-  //    valid ids; slots past it (left by out-of-range ids) stay as they were.
-  const uint32_t n_valid = hist[(kSegWarps - 1) * n_buckets + n_buckets - 1];
+  // 4. coalesced write of the permutation: the valid ids fill slots [0, n_valid);
+  //    slots past it (left by out-of-range ids) stay as they were.
+  const uint32_t n_valid = (uint32_t)L - ws[32];
   int32_t* dst = perm + seg * L;
   for (int s = threadIdx.x; s < L; s += blockDim.x)
     if ((uint32_t)s < n_valid) dst[s] = pm[s];

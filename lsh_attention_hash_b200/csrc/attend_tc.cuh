@@ -338,13 +338,15 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
     uint32_t(&cur)[32] = (g & 1) ? rb : ra;
     uint32_t(&nxt)[32] = (g & 1) ? ra : rb;
     if (g < 3) tc::tmem_ld32(sbuf + scol + 32 * (g + 1), nxt);
-    const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
+    // key multipliers as 16-byte loads (each group's 32 floats start on a 16-byte boundary)
+    const float4* cm4 = reinterpret_cast<const float4*>(g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2));
     const bool dead = g < g_first;
     uint32_t w16[16];
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-      float v0 = __uint_as_float(cur[e]) * cm[e];
-      float v1 = __uint_as_float(cur[e + 1]) * cm[e + 1];
+      const float4 c4 = cm4[e >> 2];
+      float v0 = __uint_as_float(cur[e]) * ((e & 2) ? c4.z : c4.x);
+      float v1 = __uint_as_float(cur[e + 1]) * ((e & 2) ? c4.w : c4.y);
       if (g == g_self && self_mask) {
         if (e == lane) v0 = -INFINITY;
         if (e + 1 == lane) v1 = -INFINITY;

@@ -226,11 +226,11 @@ def run_ours(args, w, rank, world, local_rank):
     import torch.distributed as dist
 
     import lsh_attention_hash_b200 as lsh
-    from lsh_attention_hash_b200 import binding, synth
+    from lsh_attention_hash_b200 import binding, multi, synth
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    qk_h, v_h, R_h = synth.make_inputs(w, seed=rank, pin=True)
+    qk_h, v_h, R_h = synth.make_inputs(w, seed=multi.rank_seed(0, rank), pin=True)
     qk = qk_h.to(dev)
     v = v_h.to(dev)
     R = R_h.to(dev)
@@ -304,10 +304,7 @@ def run_ours(args, w, rank, world, local_rank):
     barrier()
     e2e_ms = e_start.elapsed_time(e_end)
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, e2e_ms = t.tolist()
+    elapsed_ms, e2e_ms = multi.max_over_ranks([elapsed_ms, e2e_ms], device=dev)
 
     if rank != 0:
         return

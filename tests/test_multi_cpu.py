@@ -1,0 +1,72 @@
+"""The N > 1 host logic on CPU: two gloo ranks (no GPU), as bench.py runs it under
+torchrun with one rank per GPU.  The data path has no collective (every (b, h)
+slice is independent); the ranks only agree on the step time, the maximum of
+their own timings."""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from lsh_attention_hash_b200 import multi, synth
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # the step time of the run is the maximum of the ranks' own timings
+        got = multi.max_over_ranks([10.0 + rank, 5.0 - rank])
+        # weak scaling: each rank generates its own batch
+        w = synth.small_workload("multi", 1, 1, 256, 64, "bf16", 16, 64, 1)
+        qk, _, _ = synth.make_inputs(w, seed=multi.rank_seed(0, rank))
+        digest = float(qk.float().sum())
+        digests = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(digests, torch.tensor([digest], dtype=torch.float64))
+        out[rank] = (got, [float(d) for d in digests])
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_max_timing_and_draw_distinct_batches():
+    world = 2
+    manager = mp.get_context("spawn").Manager()
+    out = manager.dict()
+    mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, start_method="spawn", join=True)
+    assert sorted(out.keys()) == [0, 1]
+    for rank in range(world):
+        got, digests = out[rank]
+        assert got == [11.0, 5.0]                # max over ranks of (10 + r, 5 - r)
+        assert digests[0] != digests[1]          # the ranks' inputs differ
+    assert out[0][1] == out[1][1]
+
+
+def test_max_over_ranks_without_process_group_is_identity():
+    assert multi.max_over_ranks([1.5, 2.0]) == [1.5, 2.0]
+
+
+@pytest.mark.parametrize("B,H,world", [(8, 8, 2), (8, 8, 3), (1, 8, 4), (3, 5, 8), (1, 1, 2)])
+def test_slice_shards_cover_every_slice_once(B, H, world):
+    seen = []
+    sizes = []
+    for rank in range(world):
+        sl = multi.shard_slices(B, H, rank, world)
+        sizes.append(len(sl))
+        seen += sl
+    assert sorted(seen) == [(b, h) for b in range(B) for h in range(H)]
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_slice_shard_rejects_bad_rank():
+    with pytest.raises(ValueError):
+        multi.slice_shard(8, 8, 2, 2)

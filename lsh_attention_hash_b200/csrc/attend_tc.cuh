@@ -329,10 +329,10 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
 template <int D>
 __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint32_t pcol, const float* cm_lo,
                                              const float* cm_hi, int g_first, int g_self, int lane, int self_mask,
-                                             float m, float& l) {
+                                             float m, float& l, const uint32_t (&g0)[32]) {
   uint32_t ra[32], rb[32];
-  tc::tmem_ld32(sbuf + scol, ra);
-  tc::tmem_wait_ld_regs(ra);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) ra[e] = g0[e];  // group 0, loaded by the caller
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
     uint32_t(&cur)[32] = (g & 1) ? rb : ra;
@@ -616,12 +616,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
         if (!low) colmul[sp * kRows + r] = row_colmul<D>(smem + Lay::kQK + sp * Lay::kSlotBytes, r, p.colscale);
         tc::mbar_arrive(&cm_full[sp]);
       }
-      // own key multiplier from the diagonal of S (||k_r||^2 at key 64 + r % 64)
+      // own key multiplier from the diagonal of S (||k_r||^2 at key 64 + r % 64); the
+      // pass's first S group is loaded at the same time, so its latency hides
+      // behind the key-multiplier exchange
       float diag;
+      uint32_t sg0[32];
       {
         uint32_t raw[32];
         tc::tmem_ld32(sbuf + scol + 32 * g_self, raw);
-        tc::tmem_wait_ld();
+        tc::tmem_ld32(sbuf + scol, sg0);
+        tc::tmem_wait_ld_regs(raw);
+        tc::tmem_wait_ld_regs(sg0);
         diag = 0.f;
 #pragma unroll
         for (int e = 0; e < 32; ++e) diag = (e == lane) ? __uint_as_float(raw[e]) : diag;
@@ -641,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       float m = diag * cm_own;
       float l = 0.f;  // sum of the weights (log-sum-exp); O is normalised by the rounded weights' sum
       const uint32_t pcol = low ? 0 : 32;  // P column of the row's first key
-      softmax_pass<D>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l);
+      softmax_pass<D>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0);
       if (__any_sync(0xffffffffu, !(l > 1e-30f))) {
         // the bound was too loose for some row of the warp (long query rows): S is
         // rebuilt in TMEM from the rows in shared memory (P has overwritten part of
@@ -649,7 +654,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
         restore_s<D>(smem, sbuf, scol, sp, sc, r, low);
         m = exact_row_max(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask);
         l = 0.f;
-        softmax_pass<D>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l);
+        tc::tmem_ld32(sbuf + scol, sg0);
+        tc::tmem_wait_ld_regs(sg0);
+        softmax_pass<D>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0);
       }
       {
         uint32_t z[32];

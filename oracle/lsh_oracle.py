@@ -27,7 +27,7 @@ Sources (the pages this follows, by title and section):
   section "Разделение на блоки (Chunking)": fixed-size blocks of the sorted
   sequence, each element attends inside its block and the neighbouring one.
 
-Readings where the pages are silent or garbled (each also listed in the design doc):
+Readings where the pages are silent or garbled:
 
 * chunk 0 has no previous chunk (no wrap-around); the window is a *set* of
   sorted slots, so a single chunk covering the sequence is not duplicated;

@@ -14,7 +14,8 @@
 //   S[128 x 192] = Q K^T        two UMMAs (N = 64 for chunk 2j-1, N = 128 for
 //                                the pair itself, whose rows are also Q)
 //   row r sees keys [64*(r>=64), 64*(r>=64) + 128); its own key is 64 + r%64
-//   P = exp2(S * s_j - max) in bf16, written back over the head of S in TMEM
+//   P = exp2(S * s_j - m) in bf16 (m a per-row shift), written back over the
+//                                head of S in TMEM
 //   O[128 x D] = P V            UMMA with A = P from TMEM, B = V (MN-major),
 //                                accumulated behind P in the same TMEM buffer
 // and the rows go back to their original positions perm[s].

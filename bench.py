@@ -337,7 +337,7 @@ def run_ours(args, w, rank, world, local_rank):
     else:
         sort_launches = 3 + (1 if w.n_buckets > 16384 else 0)  # count, scan, scatter (+ counter clear)
     launches_per_step = 3 + sort_launches                  # hash, sort, attend, combine
-    sample_slices = 1
+    sample_slices = 2  # about 10 s of float64 CPU work at the 64K workload
     c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

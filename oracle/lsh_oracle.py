@@ -36,6 +36,11 @@ Readings where the pages are silent or garbled:
 * queries stay raw, keys are unit-normalised, logit scale defaults to
   1/sqrt(D);
 * a token does not attend to itself unless it is the only key in its window;
+* causal variant (the pages' character-level language model, ai-scholar.tech
+  article, results on enwik8-64K; masking in the twgreatdaily article, "1 LSH
+  Attention"): a key whose original position is after the query's is not
+  admissible; the self rule then applies to what remains, so a query with no
+  earlier key in its window sees only itself;
 * rounds are merged by their per-query log-sum-exp weights;
 * argmax ties go to the lowest index; a hash is "near-tie" when the top two
   values of [p, -p] differ by less than ``TIE_REL`` relative to the top.
@@ -132,8 +137,12 @@ def _window_slots(k: int, chunk: int) -> np.ndarray:
     return np.arange(max(k - 1, 0) * chunk, (k + 1) * chunk)
 
 
-def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale):
+def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale, causal=False):
     """Outputs of the queries of sorted chunk k of one (b, h, round) segment.
+
+    causal: a key whose original position is after the query's is not
+    admissible (the language-model reading of the window).  The self entry is
+    dropped while the query has another admissible key.
 
     Returns (orig positions [c], o [c, D], lse [c]).
     """
@@ -142,8 +151,14 @@ def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale):
     qi = perm_seg[q_slots]
     kj = perm_seg[w_slots]
     logits = (x[qi] @ k_hat[kj].T) * scale  # [c, |W|]
-    if self_mask and len(w_slots) > 1:
-        logits[q_slots[:, None] == w_slots[None, :]] = -np.inf
+    adm = np.ones(logits.shape, dtype=bool)
+    if causal:
+        adm &= kj[None, :] <= qi[:, None]
+    if self_mask:
+        is_self = q_slots[:, None] == w_slots[None, :]
+        others = np.any(adm & ~is_self, axis=1, keepdims=True)
+        adm &= ~(is_self & others)
+    logits[~adm] = -np.inf
     m = np.max(logits, axis=1, keepdims=True)
     lse = m[:, 0] + np.log(np.sum(np.exp(logits - m), axis=1))
     weights = np.exp(logits - lse[:, None])
@@ -157,10 +172,12 @@ def _prep_slice(qk_bh, v_bh):
     return x, x / np.maximum(norms, 1e-12), vv
 
 
-def oracle_attend(qk, v, perm, chunk: int, self_mask: bool = True, scale: float | None = None):
+def oracle_attend(qk, v, perm, chunk: int, self_mask: bool = True, scale: float | None = None,
+                  causal: bool = False):
     """Per-round LSH attention outputs in original token order.
 
-    qk, v: [B, H, L, D]; perm: [B, H, n_rounds, L].
+    qk, v: [B, H, L, D]; perm: [B, H, n_rounds, L].  causal: keys after the
+    query's position are not admissible.
     Returns (o [B, H, n_rounds, L, D] float64, lse [B, H, n_rounds, L] float64).
     """
     B, H, L, D = qk.shape
@@ -177,14 +194,14 @@ def oracle_attend(qk, v, perm, chunk: int, self_mask: bool = True, scale: float 
             x, k_hat, vv = _prep_slice(qk[b, h], v[b, h])
             for r in range(n_rounds):
                 for k in range(L // chunk):
-                    qi, ob, lb = _attend_chunk(x, k_hat, vv, perm[b, h, r], k, chunk, self_mask, scale)
+                    qi, ob, lb = _attend_chunk(x, k_hat, vv, perm[b, h, r], k, chunk, self_mask, scale, causal)
                     o[b, h, r, qi] = ob
                     lse[b, h, r, qi] = lb
     return o, lse
 
 
 def oracle_attend_slots(qk_bh, v_bh, perm_seg, chunk: int, slots, self_mask: bool = True,
-                        scale: float | None = None):
+                        scale: float | None = None, causal: bool = False):
     """Outputs of selected sorted slots of ONE (b, h, round) segment.
 
     For checks at sizes where a whole segment is too slow: qk_bh, v_bh are
@@ -205,7 +222,7 @@ def oracle_attend_slots(qk_bh, v_bh, perm_seg, chunk: int, slots, self_mask: boo
     for n, s in enumerate(slots):
         k = int(s) // chunk
         if k not in cache:
-            cache[k] = _attend_chunk(x, k_hat, vv, np.asarray(perm_seg), k, chunk, self_mask, scale)
+            cache[k] = _attend_chunk(x, k_hat, vv, np.asarray(perm_seg), k, chunk, self_mask, scale, causal)
         qi, ob, lb = cache[k]
         j = int(s) - k * chunk
         out_pos[n], out_o[n], out_l[n] = qi[j], ob[j], lb[j]
@@ -233,11 +250,11 @@ def oracle_combine(o, lse):
 
 
 def oracle_lsh_attention(qk, v, R, n_buckets: int, chunk: int, self_mask: bool = True,
-                         scale: float | None = None):
+                         scale: float | None = None, causal: bool = False):
     """All four steps end to end.  Returns a dict of every intermediate."""
     buckets, near = oracle_hash(qk, R, n_buckets)
     perm = oracle_sort(buckets)
-    o, lse = oracle_attend(_f64(qk), _f64(v), perm, chunk, self_mask, scale)
+    o, lse = oracle_attend(_f64(qk), _f64(v), perm, chunk, self_mask, scale, causal)
     out, lse_out = oracle_combine(o, lse)
     return {"buckets": buckets, "near_tie": near, "perm": perm, "o_rounds": o,
             "lse_rounds": lse, "out": out, "lse": lse_out}

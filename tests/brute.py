@@ -41,20 +41,23 @@ def brute_hash_row(x, R_round):
     return best, ordered[0], ordered[1]
 
 
-def admissible_slots(s, L, chunk, self_mask):
+def admissible_slots(s, L, chunk, self_mask, perm=None, causal=False):
     """Sorted slots that the query at sorted slot s may attend to.
 
     Enumerated over every slot of the sequence: slot t is admissible when its
-    chunk is the query's chunk or the one just before it.
+    chunk is the query's chunk or the one just before it (and, causal, when
+    its original position perm[t] is not after the query's perm[s]).
     """
     k = s // chunk
     W = [t for t in range(L) if t // chunk == k or t // chunk == k - 1]
+    if causal:
+        W = [t for t in W if perm[t] <= perm[s]]
     if self_mask and len(W) > 1:
         W = [t for t in W if t != s]
     return W
 
 
-def brute_attend_round(qk, v, perm, chunk, self_mask, scale):
+def brute_attend_round(qk, v, perm, chunk, self_mask, scale, causal=False):
     """Per-position (o, lse) of one round, as dicts keyed by original position.
 
     qk, v: L lists of D floats; perm: list, perm[s] = original position.
@@ -65,7 +68,7 @@ def brute_attend_round(qk, v, perm, chunk, self_mask, scale):
     for s in range(L):
         i = perm[s]
         logits = []
-        for t in admissible_slots(s, L, chunk, self_mask):
+        for t in admissible_slots(s, L, chunk, self_mask, perm, causal):
             j = perm[t]
             nj = math.sqrt(dot(qk[j], qk[j]))
             logits.append((dot(qk[i], qk[j]) / nj * scale if nj > 0 else 0.0, j))

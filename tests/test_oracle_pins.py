@@ -357,3 +357,67 @@ def test_end_to_end_matches_brute_force_pipeline():
     for i in range(L):
         assert np.allclose(res["out"][0, 0, i], bo[i], atol=1e-12)
         assert abs(res["lse"][0, 0, i] - bl[i]) < 1e-12
+
+
+# ---------------------------------------------------------------- causal variant
+@pytest.mark.parametrize("L,chunk,self_mask", [(24, 4, True), (24, 4, False), (16, 16, True), (12, 3, True),
+                                               (8, 1, True)])
+def test_attend_causal_matches_admissible_set_enumeration(L, chunk, self_mask):
+    """causal: keys after the query's original position are not admissible (brute force)."""
+    rng = np.random.default_rng(L * 17 + chunk)
+    D, nr = 5, 2
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, nr)[None, None]
+    scale = 0.41
+    o, lse = oracle_attend(qk, v, perm, chunk, self_mask, scale, causal=True)
+    for r in range(nr):
+        bo, bl = brute.brute_attend_round(qk[0, 0].tolist(), v[0, 0].tolist(), perm[0, 0, r].tolist(), chunk,
+                                          self_mask, scale, causal=True)
+        for i in range(L):
+            assert np.allclose(o[0, 0, r, i], bo[i], rtol=0, atol=1e-12)
+            assert abs(lse[0, 0, r, i] - bl[i]) < 1e-12
+
+
+def test_attend_causal_single_chunk_equals_dense_causal_softmax():
+    """chunk == L, causal: dense attention of position i over positions j < i (normalised keys);
+    position 0 has no earlier key and sees only itself, whatever the permutation."""
+    rng = np.random.default_rng(21)
+    L, D, nr = 24, 6, 3
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, nr)[None, None]
+    o, lse = oracle_attend(qk, v, perm, L, True, causal=True)
+    x = qk[0, 0]
+    kh = x / np.linalg.norm(x, axis=1, keepdims=True)
+    S = (x @ kh.T) / math.sqrt(D)
+    S[np.triu_indices(L, 0)] = -np.inf          # keys j >= i out (self too)
+    S[0, 0] = x[0] @ kh[0] / math.sqrt(D)       # position 0: only itself
+    Z = np.exp(S).sum(1)
+    dense = (np.exp(S) / Z[:, None]) @ v[0, 0]
+    for r in range(nr):
+        assert np.allclose(o[0, 0, r], dense, atol=1e-12)
+        assert np.allclose(lse[0, 0, r], np.log(Z), atol=1e-12)
+    assert np.allclose(o[0, 0, 0, 0], v[0, 0, 0])
+
+
+def test_attend_causal_constant_values_and_future_independence():
+    """V == 1 gives 1; changing only the rows of positions after i leaves position i unchanged
+    in a single-chunk window (causal), while it does change without the mask."""
+    rng = np.random.default_rng(23)
+    L, D = 16, 4
+    qk = rng.standard_normal((1, 1, L, D))
+    perm = _random_perm(rng, L, 1)[None, None]
+    o1, _ = oracle_attend(qk, np.ones((1, 1, L, D)), perm, 8, causal=True)
+    assert np.allclose(o1, 1.0, atol=1e-12)
+    v = rng.standard_normal((1, 1, L, D))
+    o, _ = oracle_attend(qk, v, perm, L, causal=True)
+    i = 9
+    qk2, v2 = qk.copy(), v.copy()
+    qk2[0, 0, i + 1:] += rng.standard_normal((L - i - 1, D))
+    v2[0, 0, i + 1:] += 5.0
+    o2, _ = oracle_attend(qk2, v2, perm, L, causal=True)
+    assert np.allclose(o[0, 0, 0, :i + 1], o2[0, 0, 0, :i + 1], atol=1e-12)
+    o3, _ = oracle_attend(qk, v, perm, L, causal=False)
+    o4, _ = oracle_attend(qk2, v2, perm, L, causal=False)
+    assert not np.allclose(o3[0, 0, 0, i], o4[0, 0, 0, i])

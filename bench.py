@@ -157,7 +157,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
-def oracle_sample(w, slices=1, seed=0):
+def oracle_sample(w, slices=1, seed=0, causal=False):
     """Runs the float64 oracle on `slices` (b, h) slices of the workload, all rounds.
 
     Returns (seconds, tokens, threads).
@@ -176,7 +176,7 @@ def oracle_sample(w, slices=1, seed=0):
         qk = qk_s[None, None]
         v = v_s[None, None]
         t0 = time.perf_counter()
-        oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk)
+        oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, causal=causal)
         secs += time.perf_counter() - t0
         tokens += w.L
     info = threadpoolctl.threadpool_info()
@@ -188,10 +188,10 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     for _ in range(args.warmup):
-        oracle_sample(w, 1)
+        oracle_sample(w, 1, causal=args.causal)
     secs, tokens, threads = 0.0, 0, 1
     for _ in range(args.steps):
-        s, t, threads = oracle_sample(w, 1)
+        s, t, threads = oracle_sample(w, 1, causal=args.causal)
         secs += s
         tokens += t
     value = tokens / secs
@@ -249,7 +249,7 @@ def run_ours(args, w, rank, world, local_rank):
         if record:
             ev[2].record(stream)
         lsh.lsh_chunk_attend(qk, v, bufs["perm"], w.chunk, out_rounds=bufs["out_rounds"],
-                             lse=bufs["lse_rounds"], stream=stream)
+                             lse=bufs["lse_rounds"], causal=args.causal, stream=stream)
         if record:
             ev[3].record(stream)
         lsh.lsh_combine_rounds(bufs["out_rounds"], bufs["lse_rounds"], out=bufs["out"], want_lse=False,
@@ -297,7 +297,7 @@ def run_ours(args, w, rank, world, local_rank):
         qk.copy_(qk_h, non_blocking=True)
         v.copy_(v_h, non_blocking=True)
         R.copy_(R_h, non_blocking=True)
-        lsh.lsh_attention(qk, v, R, w.n_buckets, w.chunk, stream=stream, bufs=bufs)
+        lsh.lsh_attention(qk, v, R, w.n_buckets, w.chunk, causal=args.causal, stream=stream, bufs=bufs)
         out_h.copy_(bufs["out"], non_blocking=True)
     e_end.record(stream)
     torch.cuda.synchronize()
@@ -338,12 +338,12 @@ def run_ours(args, w, rank, world, local_rank):
         sort_launches = 3 + (1 if w.n_buckets > 16384 else 0)  # count, scan, scatter (+ counter clear)
     launches_per_step = 3 + sort_launches                  # hash, sort, attend, combine
     sample_slices = 2  # about 10 s of float64 CPU work at the 64K workload
-    c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices)
+    c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices, causal=args.causal)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": workload_config(w),
+        "config": dict(workload_config(w), **({"mask": "causal"} if args.causal else {})),
         "roofline": {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": recorded_traffic(dominant, args.workload),
                      "peak_source": peak_src + (", sustained tensor peak" if bound == "tensor" else "")},
@@ -372,6 +372,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="64k")
+    ap.add_argument("--causal", action="store_true",
+                    help="causal window (keys after the query's position masked; CUDA-core attention path)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

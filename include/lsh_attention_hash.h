@@ -66,6 +66,12 @@ typedef enum lsh_status {
 
 typedef enum lsh_dtype { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
 
+/* Mask bits of lsh_chunk_attend. */
+typedef enum lsh_mask {
+  LSH_MASK_SELF = 1,   /* a slot does not see itself unless it is its only key */
+  LSH_MASK_CAUSAL = 2  /* a key after the query's original position is not admissible */
+} lsh_mask;
+
 /* Version of this ABI (incremented on any signature change). */
 LSH_API int lsh_abi_version(void);
 
@@ -177,7 +183,13 @@ LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H
  *   chunk      chunk length c, L % c == 0.  Chunk k = sorted slots
  *              [k c, (k+1) c); its queries see the slots of chunk k-1 (none
  *              for k = 0: no wrap-around) and of chunk k
- *   self_mask  1: a slot does not see itself unless it is its only key; 0: it does
+ *   mask       bits of lsh_mask: LSH_MASK_SELF (1): a slot does not see itself
+ *              unless it is its only key; LSH_MASK_CAUSAL (2): a key whose
+ *              original position perm[t] is after the query's perm[s] is not
+ *              admissible (the pages' character-level language model; the self
+ *              rule then applies to what remains, so a query with no earlier key
+ *              in its window sees only itself).  The tensor-core path serves
+ *              masks 0 and 1; causal runs on the CUDA-core path
  *   scale      logit scale; <= 0 selects 1/sqrt(D).  logit(s, t) =
  *              scale * qk[perm[s]] . qk[perm[t]] / ||qk[perm[t]]||
  *   out_rounds [B, H, n_rounds, L, D] out_dtype  out: per-round softmax-weighted
@@ -191,7 +203,7 @@ LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H
 LSH_API lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int H, int L,
                             int D, int n_rounds, const int32_t* perm,
                             const void* qk_sorted, const void* v_sorted, int chunk,
-                            int self_mask, float scale, void* out_rounds, int out_dtype,
+                            int mask, float scale, void* out_rounds, int out_dtype,
                             float* lse, void* stream);
 
 /*

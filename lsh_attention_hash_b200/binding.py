@@ -190,9 +190,12 @@ def lsh_sort_permute_noalloc(buckets, n_buckets, *, perm=None, inv=None, want_in
     return perm, inv
 
 
-def lsh_chunk_attend(qk, v, perm, chunk, *, self_mask=True, scale=None, qk_sorted=None, v_sorted=None,
-                     out_dtype=None, out_rounds=None, lse=None, stream=None):
-    """Per-round outputs [B,H,n_rounds,L,D] and log-sum-exp [B,H,n_rounds,L] in original order."""
+def lsh_chunk_attend(qk, v, perm, chunk, *, self_mask=True, causal=False, scale=None, qk_sorted=None,
+                     v_sorted=None, out_dtype=None, out_rounds=None, lse=None, stream=None):
+    """Per-round outputs [B,H,n_rounds,L,D] and log-sum-exp [B,H,n_rounds,L] in original order.
+
+    ``causal``: keys after the query's original position are not admissible.
+    """
     lib = load_library()
     _need(qk, "qk")
     _need(v, "v", qk.dtype, qk.shape)
@@ -212,7 +215,8 @@ def lsh_chunk_attend(qk, v, perm, chunk, *, self_mask=True, scale=None, qk_sorte
     _need(lse, "lse", torch.float32, (B, H, n_rounds, L))
     sc = 0.0 if scale is None else float(scale)
     _check(lib.lsh_chunk_attend(_ptr(qk), _ptr(v), _dt(qk), B, H, L, D, n_rounds, _ptr(perm),
-                                _ptr(qk_sorted), _ptr(v_sorted), int(chunk), 1 if self_mask else 0, sc,
+                                _ptr(qk_sorted), _ptr(v_sorted), int(chunk),
+                                (1 if self_mask else 0) | (2 if causal else 0), sc,
                                 _ptr(out_rounds), _DT[out_dtype], _ptr(lse), _stream(stream)),
            "lsh_chunk_attend")
     return out_rounds, lse
@@ -244,7 +248,7 @@ def lsh_get_device_status(stream=None) -> int:
     return int(load_library().lsh_get_device_status(_stream(stream)))
 
 
-def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, scale=None, stream=None,
+def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, causal=False, scale=None, stream=None,
                   return_all=False, bufs=None):
     """The whole forward pass: hash, sort, chunk attention, round merge (four C-ABI calls).
 
@@ -256,7 +260,7 @@ def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, scale=None, str
                              with_near_tie=return_all or "near_tie" in b, stream=stream)
     perm, _, _, _ = lsh_sort_permute(buckets, n_buckets, perm=b.get("perm"), workspace=b.get("workspace"),
                                      stream=stream)
-    o, lse = lsh_chunk_attend(qk, v, perm, chunk, self_mask=self_mask, scale=scale,
+    o, lse = lsh_chunk_attend(qk, v, perm, chunk, self_mask=self_mask, causal=causal, scale=scale,
                               out_rounds=b.get("out_rounds"), lse=b.get("lse_rounds"), stream=stream)
     out, lse_out = lsh_combine_rounds(o, lse, out=b.get("out"), lse_out=b.get("lse"),
                                       want_lse=return_all or "lse" in b, stream=stream)

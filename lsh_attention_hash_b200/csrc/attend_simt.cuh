@@ -5,6 +5,9 @@
 // divided by the partition function; with Q = K the keys are length-normalised;
 // after sorting, chunk k looks back one chunk (no wrap-around for chunk 0).
 // A query does not see its own slot unless that slot is its only key.
+// Causal variant (the pages' character-level language model): a key whose
+// original position is after the query's is not admissible; a query left with
+// no key but itself sees only itself (output v_self, lse = scale * ||q||).
 //
 // One CTA takes up to 32 queries of one chunk of one (b, h, round) segment and
 // streams the chunk's window (chunks k-1 and k) in blocks of 32 keys, keeping
@@ -25,7 +28,7 @@ template <typename T, typename TO>
 __global__ void __launch_bounds__(kAttWarps * 32)
 attend_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int32_t* __restrict__ perm,
                    const T* __restrict__ qk_sorted, const T* __restrict__ v_sorted, int L, int D,
-                   int n_rounds, int chunk, int self_mask, float scale, TO* __restrict__ out,
+                   int n_rounds, int chunk, int self_mask, int causal, float scale, TO* __restrict__ out,
                    float* __restrict__ lse) {
   extern __shared__ float sm[];
   const int DP = D + 1;                 // padded row pitch (conflict-free column reads)
@@ -94,6 +97,7 @@ attend_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int3
       }
     }
     __syncthreads();
+    const int kpos = (causal && lane < nk) ? pseg[kb + lane] : 0;  // original position of lane's key
 #pragma unroll
     for (int a = 0; a < QW; ++a) {
       const int qi = warp * QW + a;
@@ -104,7 +108,11 @@ attend_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int3
       for (int d = 0; d < D; ++d) dotv = fmaf(qs[qi * DP + d], ks[lane * DP + d], dotv);
       float logit = dotv * kinv[lane] * scale;
       const int kslot = kb + lane;
-      if (lane >= nk || (self_mask && kslot == qslot && !only_self_possible)) logit = -INFINITY;
+      // self is dropped here while other keys may remain (non-causal: unless the window is
+      // the query alone); a causal query left with no key falls back to itself below
+      if (lane >= nk || (self_mask && kslot == qslot && (causal || !only_self_possible)) ||
+          (causal && kpos > pseg[qslot]))
+        logit = -INFINITY;
       float bm = logit;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
@@ -130,11 +138,22 @@ attend_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int3
 
 #pragma unroll
   for (int a = 0; a < QW; ++a) {
-    const int qslot = q0 + warp * QW + a;
+    const int qi = warp * QW + a;
+    const int qslot = q0 + qi;
     if (qslot >= q1) continue;
     const long long pos = pseg[qslot];
-    const float inv_l = 1.f / l[a];
     TO* dst = out + (seg * L + pos) * (long long)D;
+    if (m[a] == -INFINITY) {  // no admissible key but itself (causal): the query sees only itself
+      float ss = 0.f;
+      for (int d = lane; d < D; d += 32) ss = fmaf(qs[qi * DP + d], qs[qi * DP + d], ss);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const T* vrow = row_v(qslot);
+      for (int d = lane; d < D; d += 32) dst[d] = from_f32<TO>(to_f32(vrow[d]));
+      if (lane == 0) lse[seg * L + pos] = sqrtf(ss) * scale;
+      continue;
+    }
+    const float inv_l = 1.f / l[a];
 #pragma unroll
     for (int e = 0; e < kAttMaxDL; ++e)
       if (e < DL && lane + 32 * e < D) dst[lane + 32 * e] = from_f32<TO>(o[a][e] * inv_l);

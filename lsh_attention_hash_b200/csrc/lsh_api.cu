@@ -378,14 +378,16 @@ lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H, int L,
 
 lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int H, int L, int D,
                             int n_rounds, const int32_t* perm, const void* qk_sorted,
-                            const void* v_sorted, int chunk, int self_mask, float scale,
+                            const void* v_sorted, int chunk, int mask, float scale,
                             void* out_rounds, int out_dtype, float* lse, void* stream) {
   if (!valid_dtype(dtype) || !valid_dtype(out_dtype)) return LSH_ERR_DTYPE;
   lsh_status st = check_bhld(B, H, L, D);
   if (st != LSH_OK) return st;
   if (n_rounds < 1 || !index_space_ok(B, H, L, n_rounds)) return LSH_ERR_SHAPE;
   if (chunk < 1 || (L > 0 && (chunk > L || L % chunk != 0))) return LSH_ERR_SHAPE;
-  if (self_mask != 0 && self_mask != 1) return LSH_ERR_INVALID_ARG;
+  if (mask < 0 || mask > (LSH_MASK_SELF | LSH_MASK_CAUSAL)) return LSH_ERR_INVALID_ARG;
+  const int self_mask = (mask & LSH_MASK_SELF) ? 1 : 0;
+  const int causal = (mask & LSH_MASK_CAUSAL) ? 1 : 0;
   if (!qk || !v || !perm || !out_rounds || !lse) return LSH_ERR_INVALID_ARG;
   if ((qk_sorted == nullptr) != (v_sorted == nullptr)) return LSH_ERR_INVALID_ARG;
   if (!aligned16(qk) || !aligned16(v) || !aligned16(perm) || !aligned16(out_rounds) ||
@@ -398,7 +400,7 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
   cudaStream_t s = as_stream(stream);
 
   const DevInfo di = dev_info();
-  if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && di.major == 10) {
+  if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && !causal && di.major == 10) {
 #define LSH_ATT_TC(DD, TO)                                                                            \
   return launch_attend_tc<DD, TO>(qk, v, qk_sorted, v_sorted, perm, B, H, L, n_rounds, self_mask, scale, \
                                   out_rounds, lse, s, di.sms)
@@ -419,7 +421,7 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
     auto kfn = lsh::attend_simt_kernel<T, TO>;                                                   \
     if (smem > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     kfn<<<grid, threads, smem, s>>>((const T*)qk, (const T*)v, perm, (const T*)qk_sorted,        \
-                                    (const T*)v_sorted, L, D, n_rounds, chunk, self_mask, scale, \
+                                    (const T*)v_sorted, L, D, n_rounds, chunk, self_mask, causal, scale, \
                                     (TO*)out_rounds, lse);                                       \
   } while (0)
   if (dtype == LSH_F32) {

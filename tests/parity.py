@@ -46,8 +46,8 @@ def check_sort(g_buckets, g_perm):
     assert np.array_equal(o_p, np_(g_perm)), "perm differs from the oracle's sort of the same buckets"
 
 
-def check_attend(qk, v, g_perm, chunk, self_mask, scale, g_o, g_lse, dtype):
-    o, lse = oracle_attend(f64(qk), f64(v), np_(g_perm), chunk, self_mask, scale)
+def check_attend(qk, v, g_perm, chunk, self_mask, scale, g_o, g_lse, dtype, causal=False):
+    o, lse = oracle_attend(f64(qk), f64(v), np_(g_perm), chunk, self_mask, scale, causal)
     err_o = float(np.max(np.abs(o - f64(g_o)))) if o.size else 0.0
     err_l = float(np.max(np.abs(lse - f64(g_lse)))) if lse.size else 0.0
     tol = TOL[dtype]

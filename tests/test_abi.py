@@ -97,7 +97,8 @@ def test_attend_rejects_bad_arguments_before_launch(lib):
     assert call(chunk=48) == SHAPE        # 1024 % 48 != 0
     assert call(chunk=0) == SHAPE
     assert call(chunk=2048) == SHAPE      # chunk > L
-    assert call(mask=2) == INVALID
+    assert call(mask=4) == INVALID        # bits beyond LSH_MASK_SELF | LSH_MASK_CAUSAL
+    assert call(mask=-1) == INVALID
     assert call(out_dtype=5) == DTYPE
     assert call(qs=A) == INVALID          # sorted qk without sorted v
     assert call(lse=None) == INVALID

@@ -232,3 +232,33 @@ def test_64k_workload_sampled_slices():
 def test_1m_workload_sampled_slices():
     w = synth.WORKLOADS["1m"]
     _sampled_slices(w, [(0, 0), (0, 6)], row_sample=4096, slot_sample=2048)
+
+
+# ---------------------------------------------------------------- causal variant
+@pytest.mark.parametrize("name,shape", [
+    ("causal_tiny", (1, 1, 1024, 64, "f32", 16, 64, 1)),
+    ("causal_bf16", (2, 2, 2048, 128, "bf16", 32, 64, 2)),
+    ("causal_dense", (1, 2, 256, 128, "bf16", 16, 256, 2)),    # chunk = L: dense causal attention
+    ("causal_chunk1", (1, 1, 64, 32, "f32", 8, 1, 1)),          # every window has two slots
+    ("causal_ragged", (1, 3, 320, 64, "bf16", 8, 32, 3)),
+])
+def test_causal_attention_end_to_end(name, shape):
+    """Keys after the query's original position are not admissible; a query with no earlier key in
+    its window sees only itself.  Checked stage by stage and end to end against the oracle."""
+    w = synth.small_workload(name, *shape)
+    qk, v, R = synth.make_inputs(w, seed=zlib.crc32(name.encode()) % 1000)
+    qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
+    res = lsh.lsh_attention(qk_d, v_d, R_d, w.n_buckets, w.chunk, causal=True, return_all=True)
+    torch.cuda.synchronize()
+    assert lsh.lsh_get_device_status() == 0
+    mism, _ = parity.check_hash(qk, R, w.n_buckets, res["buckets"], res["near_tie"], 1e-3)
+    parity.check_sort(res["buckets"], res["perm"])
+    parity.check_attend(qk, v, res["perm"], w.chunk, True, None, res["o_rounds"], res["lse_rounds"],
+                        w.torch_dtype, causal=True)
+    parity.check_combine(res["o_rounds"], res["lse_rounds"], res["out"], res["lse"], w.torch_dtype)
+    if mism == 0:
+        from oracle import oracle_lsh_attention
+
+        ref = oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, causal=True)
+        err = float(np.max(np.abs(ref["out"] - parity.f64(res["out"]))))
+        assert err <= parity.TOL[w.torch_dtype], err

@@ -188,8 +188,8 @@ LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H
  *              original position perm[t] is after the query's perm[s] is not
  *              admissible (the pages' character-level language model; the self
  *              rule then applies to what remains, so a query with no earlier key
- *              in its window sees only itself).  The tensor-core path serves
- *              masks 0 and 1; causal runs on the CUDA-core path
+ *              in its window sees only itself).  Every mask runs on both the
+ *              tensor-core and the CUDA-core path
  *   scale      logit scale; <= 0 selects 1/sqrt(D).  logit(s, t) =
  *              scale * qk[perm[s]] . qk[perm[t]] / ||qk[perm[t]]||
  *   out_rounds [B, H, n_rounds, L, D] out_dtype  out: per-round softmax-weighted

@@ -324,13 +324,17 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
 
 // One pass of the softmax over a row's 128 keys (four groups of 32 S columns,
 // the next group's TMEM load in flight while the current one is processed):
-// w = 2^(S * colmul - m) in fp32 (self masked, a missing previous chunk dead),
-// l += w, and the weights go to P as bf16 pairs right away: P's group g lands
-// on S columns whose values this row has already consumed.
-template <int D>
+// w = 2^(S * colmul - m) in fp32 (self masked, a missing previous chunk dead,
+// with CAUSAL a key after the query's original position masked), l += w, and
+// the weights go to P as bf16 pairs right away: P's group g lands on S columns
+// whose values this row has already consumed.  With CAUSAL, `earlier` counts
+// the admissible keys other than self and `self_w` keeps the P words of the
+// self group (for the self-only fix-up).
+template <int D, bool CAUSAL>
 __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint32_t pcol, const float* cm_lo,
                                              const float* cm_hi, int g_first, int g_self, int lane, int self_mask,
-                                             float m, float& l, const uint32_t (&g0)[32]) {
+                                             float m, float& l, const uint32_t (&g0)[32], const int32_t* kp_lo,
+                                             const int32_t* kp_hi, int qpos, int& earlier, uint32_t (&self_w)[16]) {
   uint32_t ra[32], rb[32];
 #pragma unroll
   for (int e = 0; e < 32; ++e) ra[e] = g0[e];  // group 0, loaded by the caller
@@ -341,6 +345,7 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
     if (g < 3) tc::tmem_ld32(sbuf + scol + 32 * (g + 1), nxt);
     // key multipliers as 16-byte loads (each group's 32 floats start on a 16-byte boundary)
     const float4* cm4 = reinterpret_cast<const float4*>(g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2));
+    const int4* kp4 = reinterpret_cast<const int4*>(g < 2 ? kp_lo + 32 * g : kp_hi + 32 * (g - 2));
     const bool dead = g < g_first;
     uint32_t w16[16];
 #pragma unroll
@@ -348,6 +353,13 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
       const float4 c4 = cm4[e >> 2];
       float v0 = __uint_as_float(cur[e]) * ((e & 2) ? c4.z : c4.x);
       float v1 = __uint_as_float(cur[e + 1]) * ((e & 2) ? c4.w : c4.y);
+      if (CAUSAL) {  // keys are distinct tokens: position == qpos only for self
+        const int4 k4 = kp4[e >> 2];
+        const int p0 = (e & 2) ? k4.z : k4.x, p1 = (e & 2) ? k4.w : k4.y;
+        if (p0 > qpos) v0 = -INFINITY;
+        if (p1 > qpos) v1 = -INFINITY;
+        if (!dead) earlier += (p0 < qpos) + (p1 < qpos);
+      }
       if (g == g_self && self_mask) {
         if (e == lane) v0 = -INFINITY;
         if (e + 1 == lane) v1 = -INFINITY;
@@ -358,13 +370,36 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
       w16[e >> 1] = tc::pack_bf16x2(a, c);
     }
     tc::tmem_st16(sbuf + pcol + 16 * g, w16);
+    if (CAUSAL && g >= 2 && g == g_self) {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) self_w[k] = w16[k];
+    }
     if (g < 3) tc::tmem_wait_ld_regs(nxt);
   }
 }
 
-// Exact maximum of a row's scaled logits (self excluded while it has other keys).
+// Causal rows with no earlier key in their window see only themselves: their P
+// becomes one-hot at the own key (bf16 1.0 at element `lane` of the self group)
+// and their weight sum 1 (the shift m is their own logit).  The whole warp
+// rewrites the self group, the other rows with the words they already had.
+__device__ __forceinline__ void causal_self_only(uint32_t sbuf, uint32_t pcol, int g_self, int lane, int earlier,
+                                                 const uint32_t (&self_w)[16], float& l) {
+  const bool only = earlier == 0;
+  if (!__any_sync(0xffffffffu, only)) return;
+  uint32_t w16[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    w16[k] = !only ? self_w[k] : (k == (lane >> 1) ? ((lane & 1) ? 0x3F800000u : 0x00003F80u) : 0u);
+  tc::tmem_st16(sbuf + pcol + 16 * g_self, w16);
+  if (only) l = 1.f;
+}
+
+// Exact maximum of a row's scaled logits (self excluded while it has other keys;
+// with CAUSAL, keys after the query's position excluded).
+template <bool CAUSAL>
 __device__ __forceinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const float* cm_lo, const float* cm_hi,
-                                               int g_first, int g_self, int lane, int self_mask) {
+                                               int g_first, int g_self, int lane, int self_mask,
+                                               const int32_t* kp_lo, const int32_t* kp_hi, int qpos) {
   float m = -INFINITY;
 #pragma unroll 1
   for (int g = 0; g < 4; ++g) {
@@ -373,9 +408,11 @@ __device__ __forceinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, con
     tc::tmem_wait_ld_regs(raw);
     if (g < g_first) continue;
     const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
+    const int32_t* kp = g < 2 ? kp_lo + 32 * g : kp_hi + 32 * (g - 2);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       float v = __uint_as_float(raw[e]) * cm[e];
+      if (CAUSAL && kp[e] > qpos) v = -INFINITY;
       if (g == g_self && self_mask && e == lane) v = -INFINITY;
       m = fmaxf(m, v);
     }
@@ -421,7 +458,7 @@ __device__ __noinline__ void restore_s(const uint8_t* smem, uint32_t sbuf, uint3
   tc::tmem_wait_st();
 }
 
-template <int D, typename TO>
+template <int D, typename TO, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) {
   using Lay = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -642,22 +679,33 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       if (!ok) break;
       const float* cm_lo = low ? colmul + sp * kRows + 64 : colmul + sc * kRows;  // keys 0..63 of the row
       const float* cm_hi = low ? colmul + sc * kRows : colmul + sc * kRows + 64;  // keys 64..127
+      const int32_t* kp_lo = low ? perm_s + sp * kRows + 64 : perm_s + sc * kRows;  // their positions
+      const int32_t* kp_hi = low ? perm_s + sc * kRows : perm_s + sc * kRows + 64;
+      int earlier = 0;
+      uint32_t self_w[16];
       const int g_first = (low && it.j == 0) ? 2 : 0;  // chunk 0 has no previous chunk
       // shift: ||q|| * scale * log2(e) bounds every logit of the row (log2 domain)
       float m = diag * cm_own;
       float l = 0.f;  // sum of the weights (log-sum-exp); O is normalised by the rounded weights' sum
       const uint32_t pcol = low ? 0 : 32;  // P column of the row's first key
-      softmax_pass<D>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0);
+      softmax_pass<D, CAUSAL>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0, kp_lo,
+                              kp_hi, pos, earlier, self_w);
+      if (CAUSAL) causal_self_only(sbuf, pcol, g_self, lane, earlier, self_w, l);
       if (__any_sync(0xffffffffu, !(l > 1e-30f))) {
         // the bound was too loose for some row of the warp (long query rows): S is
         // rebuilt in TMEM from the rows in shared memory (P has overwritten part of
         // it) and the warp's rows are redone with their exact maxima
         restore_s<D>(smem, sbuf, scol, sp, sc, r, low);
-        m = exact_row_max(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask);
+        const float m_cs = m;
+        m = exact_row_max<CAUSAL>(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, kp_lo, kp_hi, pos);
+        if (CAUSAL && m == -INFINITY) m = m_cs;  // self-only row: its own logit is the shift
         l = 0.f;
+        earlier = 0;
         tc::tmem_ld32(sbuf + scol, sg0);
         tc::tmem_wait_ld_regs(sg0);
-        softmax_pass<D>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0);
+        softmax_pass<D, CAUSAL>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0,
+                                kp_lo, kp_hi, pos, earlier, self_w);
+        if (CAUSAL) causal_self_only(sbuf, pcol, g_self, lane, earlier, self_w, l);
       }
       {
         uint32_t z[32];

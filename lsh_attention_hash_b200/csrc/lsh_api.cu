@@ -149,7 +149,7 @@ lsh_status dispatch_hash_tc(const void* qk, const void* R, int B, int H, int L, 
 }
 
 // Tensor-core chunk attention (bf16, chunk 64, D 64 or 128) on sm_100.
-template <int D, typename TO>
+template <int D, typename TO, bool CAUSAL>
 lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted, const void* v_sorted,
                             const int32_t* perm, int B, int H, int L, int n_rounds, int self_mask, float scale,
                             void* out, float* lse, cudaStream_t s, int sms) {
@@ -174,7 +174,7 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
   p.v = (const uint8_t*)(sorted ? v_sorted : v);
   p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   const unsigned grid = (unsigned)std::min<long long>(p.n_units, sms);
-  auto kfn = attend_tc_kernel<D, TO>;
+  auto kfn = attend_tc_kernel<D, TO, CAUSAL>;
   const int smem = (int)Layout<D>::kSmem;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LSH_ERR_CUDA;
@@ -400,9 +400,11 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
   cudaStream_t s = as_stream(stream);
 
   const DevInfo di = dev_info();
-  if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && !causal && di.major == 10) {
+  if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && di.major == 10) {
 #define LSH_ATT_TC(DD, TO)                                                                            \
-  return launch_attend_tc<DD, TO>(qk, v, qk_sorted, v_sorted, perm, B, H, L, n_rounds, self_mask, scale, \
+  return causal ? launch_attend_tc<DD, TO, true>(qk, v, qk_sorted, v_sorted, perm, B, H, L, n_rounds, self_mask, \
+                                                  scale, out_rounds, lse, s, di.sms)                         \
+                : launch_attend_tc<DD, TO, false>(qk, v, qk_sorted, v_sorted, perm, B, H, L, n_rounds, self_mask, scale, \
                                   out_rounds, lse, s, di.sms)
     if (D == 128) {
       if (out_dtype == LSH_BF16) LSH_ATT_TC(128, __nv_bfloat16); else LSH_ATT_TC(128, float);

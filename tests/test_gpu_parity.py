@@ -241,6 +241,7 @@ def test_1m_workload_sampled_slices():
     ("causal_dense", (1, 2, 256, 128, "bf16", 16, 256, 2)),    # chunk = L: dense causal attention
     ("causal_chunk1", (1, 1, 64, 32, "f32", 8, 1, 1)),          # every window has two slots
     ("causal_ragged", (1, 3, 320, 64, "bf16", 8, 32, 3)),
+    ("causal_tc_d64_odd", (1, 2, 8256, 64, "bf16", 128, 64, 2)),   # tensor-core path, odd chunk count
 ])
 def test_causal_attention_end_to_end(name, shape):
     """Keys after the query's original position are not admissible; a query with no earlier key in
@@ -262,3 +263,19 @@ def test_causal_attention_end_to_end(name, shape):
         ref = oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, causal=True)
         err = float(np.max(np.abs(ref["out"] - parity.f64(res["out"]))))
         assert err <= parity.TOL[w.torch_dtype], err
+
+
+@pytest.mark.parametrize("scale", [None, 6.0, 40.0])
+def test_causal_tensor_core_attention_scales(scale):
+    """The tensor-core attention with the causal mask (bf16, chunk 64): rows with no earlier key see
+    only themselves; at scale 40 the Cauchy-Schwarz shift underflows and the exact-maximum path
+    (with the causal mask) takes over."""
+    w = synth.small_workload("causal_tc", 2, 2, 4096, 128, "bf16", 64, 64, 2)
+    qk, v, R = synth.make_inputs(w, seed=31)
+    qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
+    b, _ = lsh.lsh_hash(qk_d, R_d, w.n_buckets)
+    perm, _, _, _ = lsh.lsh_sort_permute(b, w.n_buckets)
+    o, l = lsh.lsh_chunk_attend(qk_d, v_d, perm, w.chunk, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert lsh.lsh_get_device_status() == 0
+    parity.check_attend(qk, v, perm, w.chunk, True, scale, o, l, w.torch_dtype, causal=True)

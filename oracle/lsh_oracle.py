@@ -36,6 +36,18 @@ Readings where the pages are silent or garbled:
 * queries stay raw, keys are unit-normalised, logit scale defaults to
   1/sqrt(D);
 * a token does not attend to itself unless it is the only key in its window;
+* bucket-equality variant (twgreatdaily article, "1 LSH Attention": the
+  admissible set of a query is the keys of its own bucket, batched by chunks):
+  inside the chunk window a key is admissible only when it shares the query's
+  bucket in that round; the self rule then applies to what remains;
+* multi-round union variant (twgreatdaily article, "1 LSH Attention": the
+  admissible set over several rounds is the union of the rounds' sets, with a
+  per-pair correction whose formula the page lost in extraction): read as the
+  original paper's duplicate count, each admissible logit of a round is lowered
+  by log N_ij, N_ij = the number of rounds whose hash puts i and j in the same
+  bucket (the self pair shares every round); used with the bucket-equality
+  mask, the log-sum-exp merge then counts each key of the union once whenever
+  each shared bucket lies inside the query's window;
 * causal variant (the pages' character-level language model, ai-scholar.tech
   article, results on enwik8-64K; masking in the twgreatdaily article, "1 LSH
   Attention"): a key whose original position is after the query's is not
@@ -137,12 +149,18 @@ def _window_slots(k: int, chunk: int) -> np.ndarray:
     return np.arange(max(k - 1, 0) * chunk, (k + 1) * chunk)
 
 
-def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale, causal=False):
+def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale, causal=False, bucket_seg=None,
+                  union_buckets=None):
     """Outputs of the queries of sorted chunk k of one (b, h, round) segment.
 
     causal: a key whose original position is after the query's is not
-    admissible (the language-model reading of the window).  The self entry is
-    dropped while the query has another admissible key.
+    admissible (the language-model reading of the window).  bucket_seg (the
+    round's bucket of every original position), when given: a key in another
+    bucket than the query's is not admissible.  The self entry is dropped while
+    the query has another admissible key.  union_buckets ([n_rounds, L], every
+    round's bucket by original position), when given: each admissible logit is
+    lowered by log N, N = the number of rounds whose hash puts query and key in
+    the same bucket (the self pair: every round).
 
     Returns (orig positions [c], o [c, D], lse [c]).
     """
@@ -154,10 +172,16 @@ def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale, causal=Fals
     adm = np.ones(logits.shape, dtype=bool)
     if causal:
         adm &= kj[None, :] <= qi[:, None]
+    if bucket_seg is not None:
+        adm &= bucket_seg[kj][None, :] == bucket_seg[qi][:, None]
     if self_mask:
         is_self = q_slots[:, None] == w_slots[None, :]
         others = np.any(adm & ~is_self, axis=1, keepdims=True)
         adm &= ~(is_self & others)
+    if union_buckets is not None:
+        ub = np.asarray(union_buckets)
+        n_shared = np.sum(ub[:, kj][:, None, :] == ub[:, qi][:, :, None], axis=0)  # [c, |W|]
+        logits[adm] -= np.log(n_shared[adm])
     logits[~adm] = -np.inf
     m = np.max(logits, axis=1, keepdims=True)
     lse = m[:, 0] + np.log(np.sum(np.exp(logits - m), axis=1))
@@ -173,11 +197,16 @@ def _prep_slice(qk_bh, v_bh):
 
 
 def oracle_attend(qk, v, perm, chunk: int, self_mask: bool = True, scale: float | None = None,
-                  causal: bool = False):
+                  causal: bool = False, buckets=None, union: bool = False):
     """Per-round LSH attention outputs in original token order.
 
     qk, v: [B, H, L, D]; perm: [B, H, n_rounds, L].  causal: keys after the
-    query's position are not admissible.
+    query's position are not admissible.  buckets ([B, H, n_rounds, L], by
+    original position), when given: keys outside the query's bucket are not
+    admissible (the pages' bucket-equality mask inside the window).  union
+    (needs buckets): every admissible logit is lowered by the log of the number
+    of rounds in which query and key share a bucket, so that the rounds merged
+    by their log-sum-exp count each shared key once.
     Returns (o [B, H, n_rounds, L, D] float64, lse [B, H, n_rounds, L] float64).
     """
     B, H, L, D = qk.shape
@@ -185,8 +214,11 @@ def oracle_attend(qk, v, perm, chunk: int, self_mask: bool = True, scale: float 
     n_rounds = perm.shape[2]
     if L % chunk:
         raise ValueError("L must be a multiple of chunk")
+    if union and buckets is None:
+        raise ValueError("the union correction needs the bucket-equality mask")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    bk = None if buckets is None else np.asarray(buckets)
     o = np.empty((B, H, n_rounds, L, D))
     lse = np.empty((B, H, n_rounds, L))
     for b in range(B):
@@ -194,19 +226,24 @@ def oracle_attend(qk, v, perm, chunk: int, self_mask: bool = True, scale: float 
             x, k_hat, vv = _prep_slice(qk[b, h], v[b, h])
             for r in range(n_rounds):
                 for k in range(L // chunk):
-                    qi, ob, lb = _attend_chunk(x, k_hat, vv, perm[b, h, r], k, chunk, self_mask, scale, causal)
+                    qi, ob, lb = _attend_chunk(x, k_hat, vv, perm[b, h, r], k, chunk, self_mask, scale, causal,
+                                               None if bk is None else bk[b, h, r],
+                                               bk[b, h] if union else None)
                     o[b, h, r, qi] = ob
                     lse[b, h, r, qi] = lb
     return o, lse
 
 
 def oracle_attend_slots(qk_bh, v_bh, perm_seg, chunk: int, slots, self_mask: bool = True,
-                        scale: float | None = None, causal: bool = False):
+                        scale: float | None = None, causal: bool = False, bucket_seg=None,
+                        union_buckets=None):
     """Outputs of selected sorted slots of ONE (b, h, round) segment.
 
     For checks at sizes where a whole segment is too slow: qk_bh, v_bh are
     [L, D]; perm_seg is [L]; slots are sorted-slot indices.  The chunk of each
-    slot is evaluated in full and the requested rows are returned.
+    slot is evaluated in full and the requested rows are returned.  bucket_seg
+    ([L], this round's buckets) and union_buckets ([n_rounds, L], every round's)
+    select the bucket-equality mask and the union correction.
 
     Returns (orig positions [n], o [n, D], lse [n]).
     """
@@ -222,7 +259,8 @@ def oracle_attend_slots(qk_bh, v_bh, perm_seg, chunk: int, slots, self_mask: boo
     for n, s in enumerate(slots):
         k = int(s) // chunk
         if k not in cache:
-            cache[k] = _attend_chunk(x, k_hat, vv, np.asarray(perm_seg), k, chunk, self_mask, scale, causal)
+            cache[k] = _attend_chunk(x, k_hat, vv, np.asarray(perm_seg), k, chunk, self_mask, scale, causal,
+                                     None if bucket_seg is None else np.asarray(bucket_seg), union_buckets)
         qi, ob, lb = cache[k]
         j = int(s) - k * chunk
         out_pos[n], out_o[n], out_l[n] = qi[j], ob[j], lb[j]
@@ -250,11 +288,13 @@ def oracle_combine(o, lse):
 
 
 def oracle_lsh_attention(qk, v, R, n_buckets: int, chunk: int, self_mask: bool = True,
-                         scale: float | None = None, causal: bool = False):
+                         scale: float | None = None, causal: bool = False, bucket_mask: bool = False,
+                         union: bool = False):
     """All four steps end to end.  Returns a dict of every intermediate."""
     buckets, near = oracle_hash(qk, R, n_buckets)
     perm = oracle_sort(buckets)
-    o, lse = oracle_attend(_f64(qk), _f64(v), perm, chunk, self_mask, scale, causal)
+    o, lse = oracle_attend(_f64(qk), _f64(v), perm, chunk, self_mask, scale, causal,
+                           buckets if bucket_mask else None, union)
     out, lse_out = oracle_combine(o, lse)
     return {"buckets": buckets, "near_tie": near, "perm": perm, "o_rounds": o,
             "lse_rounds": lse, "out": out, "lse": lse_out}

@@ -41,26 +41,33 @@ def brute_hash_row(x, R_round):
     return best, ordered[0], ordered[1]
 
 
-def admissible_slots(s, L, chunk, self_mask, perm=None, causal=False):
+def admissible_slots(s, L, chunk, self_mask, perm=None, causal=False, bucket=None):
     """Sorted slots that the query at sorted slot s may attend to.
 
     Enumerated over every slot of the sequence: slot t is admissible when its
     chunk is the query's chunk or the one just before it (and, causal, when
-    its original position perm[t] is not after the query's perm[s]).
+    its original position perm[t] is not after the query's perm[s]; and, with
+    bucket (by original position), when bucket[perm[t]] == bucket[perm[s]]).
     """
     k = s // chunk
     W = [t for t in range(L) if t // chunk == k or t // chunk == k - 1]
     if causal:
         W = [t for t in W if perm[t] <= perm[s]]
+    if bucket is not None:
+        W = [t for t in W if bucket[perm[t]] == bucket[perm[s]]]
     if self_mask and len(W) > 1:
         W = [t for t in W if t != s]
     return W
 
 
-def brute_attend_round(qk, v, perm, chunk, self_mask, scale, causal=False):
+def brute_attend_round(qk, v, perm, chunk, self_mask, scale, causal=False, bucket=None,
+                       all_buckets=None):
     """Per-position (o, lse) of one round, as dicts keyed by original position.
 
     qk, v: L lists of D floats; perm: list, perm[s] = original position.
+    all_buckets (a list of every round's bucket list), when given: the weight
+    of key j for query i is divided by the number of rounds in which
+    all_buckets[r][j] == all_buckets[r][i].
     """
     L = len(perm)
     D = len(qk[0])
@@ -68,10 +75,13 @@ def brute_attend_round(qk, v, perm, chunk, self_mask, scale, causal=False):
     for s in range(L):
         i = perm[s]
         logits = []
-        for t in admissible_slots(s, L, chunk, self_mask, perm, causal):
+        for t in admissible_slots(s, L, chunk, self_mask, perm, causal, bucket):
             j = perm[t]
             nj = math.sqrt(dot(qk[j], qk[j]))
-            logits.append((dot(qk[i], qk[j]) / nj * scale if nj > 0 else 0.0, j))
+            lg = dot(qk[i], qk[j]) / nj * scale if nj > 0 else 0.0
+            if all_buckets is not None:
+                lg -= math.log(sum(1 for rb in all_buckets if rb[j] == rb[i]))
+            logits.append((lg, j))
         Z = sum(math.exp(l) for l, _ in logits)
         out_o[i] = [sum(math.exp(l) * v[j][d] for l, j in logits) / Z for d in range(D)]
         out_lse[i] = math.log(Z)

@@ -421,3 +421,141 @@ def test_attend_causal_constant_values_and_future_independence():
     o3, _ = oracle_attend(qk, v, perm, L, causal=False)
     o4, _ = oracle_attend(qk2, v2, perm, L, causal=False)
     assert not np.allclose(o3[0, 0, 0, i], o4[0, 0, 0, i])
+
+
+# ------------------------------------------------- bucket-equality mask and union
+def _bucketed(rng, L, nr, nb, sorted_perm):
+    """Random buckets [nr, L] and a permutation per round: the stable sort by
+    bucket when sorted_perm, else an unrelated random permutation."""
+    bk = rng.integers(0, nb, size=(nr, L)).astype(np.int32)
+    if sorted_perm:
+        perm = np.stack([np.argsort(bk[r], kind="stable") for r in range(nr)]).astype(np.int32)
+    else:
+        perm = _random_perm(rng, L, nr)
+    return bk, perm
+
+
+@pytest.mark.parametrize("L,chunk,self_mask,causal,union,sorted_perm", [
+    (24, 4, True, False, False, True), (24, 4, False, False, False, False), (16, 16, True, False, False, True),
+    (12, 3, True, True, False, True), (8, 1, True, False, False, True), (24, 4, True, False, True, True),
+    (24, 6, True, True, True, False), (16, 8, False, False, True, True),
+])
+def test_attend_bucket_mask_matches_admissible_set_enumeration(L, chunk, self_mask, causal, union, sorted_perm):
+    """bucket mask: a key outside the query's bucket is not admissible; union: each logit is
+    lowered by log(#rounds sharing the bucket) (brute force over the admissible slots)."""
+    rng = np.random.default_rng(L * 13 + chunk * 3 + union)
+    D, nr, nb = 5, 3, 3
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    bk, perm = _bucketed(rng, L, nr, nb, sorted_perm)
+    scale = 0.53
+    o, lse = oracle_attend(qk, v, perm[None, None], chunk, self_mask, scale, causal=causal,
+                           buckets=bk[None, None], union=union)
+    allb = [bk[r].tolist() for r in range(nr)] if union else None
+    for r in range(nr):
+        bo, bl = brute.brute_attend_round(qk[0, 0].tolist(), v[0, 0].tolist(), perm[r].tolist(), chunk,
+                                          self_mask, scale, causal=causal, bucket=bk[r].tolist(),
+                                          all_buckets=allb)
+        for i in range(L):
+            assert np.allclose(o[0, 0, r, i], bo[i], rtol=0, atol=1e-12)
+            assert abs(lse[0, 0, r, i] - bl[i]) < 1e-12
+
+
+def _dense_logits(x, D):
+    kh = x / np.linalg.norm(x, axis=1, keepdims=True)
+    return (x @ kh.T) / math.sqrt(D)
+
+
+def test_attend_bucket_mask_single_chunk_equals_dense_same_bucket_softmax():
+    """chunk == L, bucket mask: round r is dense attention of i over the other members of its
+    bucket b_r(i); a query alone in its bucket sees only itself."""
+    rng = np.random.default_rng(31)
+    L, D, nr, nb = 24, 6, 3, 5
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    bk, perm = _bucketed(rng, L, nr, nb, True)
+    bk[0, 7] = nb  # position 7 alone in its bucket in round 0
+    perm[0] = np.argsort(bk[0], kind="stable")
+    o, lse = oracle_attend(qk, v, perm[None, None], L, True, buckets=bk[None, None])
+    S0 = _dense_logits(qk[0, 0], D)
+    for r in range(nr):
+        S = S0.copy()
+        same = bk[r][:, None] == bk[r][None, :]
+        alone = same.sum(1) == 1
+        S[~same] = -np.inf
+        S[np.diag_indices(L)] = np.where(alone, np.diag(S0), -np.inf)
+        Z = np.exp(S).sum(1)
+        assert np.allclose(o[0, 0, r], (np.exp(S) / Z[:, None]) @ v[0, 0], atol=1e-12)
+        assert np.allclose(lse[0, 0, r], np.log(Z), atol=1e-12)
+    assert np.allclose(o[0, 0, 0, 7], v[0, 0, 7])
+
+
+def test_union_single_chunk_merge_equals_softmax_over_set_union():
+    """chunk == L, bucket mask and union, no query alone in any round: the rounds merged by
+    their log-sum-exp give softmax attention over U_i = {j != i : b_r(j) == b_r(i) for some r},
+    each key once; the plain merge (no correction) does not."""
+    rng = np.random.default_rng(37)
+    L, D, nr, nb = 32, 5, 4, 3
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    bk, perm = _bucketed(rng, L, nr, nb, True)
+    for r in range(nr):
+        assert np.all(np.bincount(bk[r], minlength=nb) >= 2)  # nobody alone
+    o, lse = oracle_attend(qk, v, perm[None, None], L, True, buckets=bk[None, None], union=True)
+    out, big = oracle_combine(o, lse)
+    S = _dense_logits(qk[0, 0], D)
+    U = np.zeros((L, L), dtype=bool)
+    for r in range(nr):
+        U |= bk[r][:, None] == bk[r][None, :]
+    np.fill_diagonal(U, False)
+    assert not np.all(U)  # the union is a proper subset of the sequence
+    S[~U] = -np.inf
+    Z = np.exp(S).sum(1)
+    assert np.allclose(out[0, 0], (np.exp(S) / Z[:, None]) @ v[0, 0], atol=1e-12)
+    assert np.allclose(big[0, 0], np.log(Z), atol=1e-12)
+    o2, lse2 = oracle_attend(qk, v, perm[None, None], L, True, buckets=bk[None, None], union=False)
+    out2, _ = oracle_combine(o2, lse2)
+    assert not np.allclose(out2[0, 0], out[0, 0], atol=1e-6)
+
+
+def test_union_identical_rounds_collapse_to_one_round():
+    """n identical rounds with the union correction: every pair shares all n, so each round's
+    lse is the single round's minus log n and the merged LSE equals the single round's."""
+    rng = np.random.default_rng(41)
+    L, D, chunk, n = 24, 4, 6, 4
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    bk1, perm1 = _bucketed(rng, L, 1, 3, True)
+    bk, perm = np.repeat(bk1, n, axis=0), np.repeat(perm1, n, axis=0)
+    o1, l1 = oracle_attend(qk, v, perm1[None, None], chunk, True, buckets=bk1[None, None])
+    o, lse = oracle_attend(qk, v, perm[None, None], chunk, True, buckets=bk[None, None], union=True)
+    assert np.allclose(lse, l1 - math.log(n), atol=1e-12)
+    out, big = oracle_combine(o, lse)
+    assert np.allclose(out, o1[:, :, 0], atol=1e-12)
+    assert np.allclose(big, l1[:, :, 0], atol=1e-12)
+
+
+def test_union_needs_bucket_mask():
+    qk = np.ones((1, 1, 4, 2))
+    with pytest.raises(ValueError):
+        oracle_attend(qk, qk, np.zeros((1, 1, 1, 4), dtype=np.int32) + np.arange(4), 2, union=True)
+
+
+def test_bucket_mask_end_to_end_matches_brute_force_pipeline():
+    """hash -> sort -> bucket-masked attention with the union correction, brute force per round."""
+    rng = np.random.default_rng(43)
+    L, D, nb, chunk, nr = 24, 4, 4, 4, 3
+    qk = rng.standard_normal((1, 1, L, D))
+    v = rng.standard_normal((1, 1, L, D))
+    R = rng.standard_normal((nr, D, nb // 2))
+    res = oracle_lsh_attention(qk, v, R, nb, chunk, bucket_mask=True, union=True)
+    X = qk[0, 0].tolist()
+    bks = [[brute.brute_hash_row(X[i], R[r].tolist())[0] for i in range(L)] for r in range(nr)]
+    for r in range(nr):
+        assert bks[r] == res["buckets"][0, 0, r].tolist()
+        perm = brute.brute_sort(bks[r])
+        bo, bl = brute.brute_attend_round(X, v[0, 0].tolist(), perm, chunk, True, 1 / math.sqrt(D),
+                                          bucket=bks[r], all_buckets=bks)
+        for i in range(L):
+            assert np.allclose(res["o_rounds"][0, 0, r, i], bo[i], atol=1e-12)
+            assert abs(res["lse_rounds"][0, 0, r, i] - bl[i]) < 1e-12

@@ -157,7 +157,19 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
-def oracle_sample(w, slices=1, seed=0, causal=False):
+def mask_options(args):
+    """Keyword arguments of the attention masks the command line selects."""
+    return {"causal": args.causal, "bucket_mask": args.bucket_mask or args.union, "union": args.union}
+
+
+def mask_config(args):
+    """The "mask" entry of the JSON config (absent for the plain window)."""
+    names = [n for n, on in (("causal", args.causal), ("bucket", args.bucket_mask or args.union),
+                             ("union", args.union)) if on]
+    return {"mask": "+".join(names)} if names else {}
+
+
+def oracle_sample(w, slices=1, seed=0, masks=None):
     """Runs the float64 oracle on `slices` (b, h) slices of the workload, all rounds.
 
     Returns (seconds, tokens, threads).
@@ -176,7 +188,7 @@ def oracle_sample(w, slices=1, seed=0, causal=False):
         qk = qk_s[None, None]
         v = v_s[None, None]
         t0 = time.perf_counter()
-        oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, causal=causal)
+        oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, **(masks or {}))
         secs += time.perf_counter() - t0
         tokens += w.L
     info = threadpoolctl.threadpool_info()
@@ -188,10 +200,10 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     for _ in range(args.warmup):
-        oracle_sample(w, 1, causal=args.causal)
+        oracle_sample(w, 1, masks=mask_options(args))
     secs, tokens, threads = 0.0, 0, 1
     for _ in range(args.steps):
-        s, t, threads = oracle_sample(w, 1, causal=args.causal)
+        s, t, threads = oracle_sample(w, 1, masks=mask_options(args))
         secs += s
         tokens += t
     value = tokens / secs
@@ -200,7 +212,7 @@ def run_reference(args, w, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic", "config": dict(workload_config(w), **mask_config(args)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -228,6 +240,7 @@ def run_ours(args, w, rank, world, local_rank):
     import lsh_attention_hash_b200 as lsh
     from lsh_attention_hash_b200 import binding, multi, synth
 
+    masks = mask_options(args)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     qk_h, v_h, R_h = synth.make_inputs(w, seed=multi.rank_seed(0, rank), pin=True)
@@ -249,7 +262,7 @@ def run_ours(args, w, rank, world, local_rank):
         if record:
             ev[2].record(stream)
         lsh.lsh_chunk_attend(qk, v, bufs["perm"], w.chunk, out_rounds=bufs["out_rounds"],
-                             lse=bufs["lse_rounds"], causal=args.causal, stream=stream)
+                             lse=bufs["lse_rounds"], buckets=bufs["buckets"], stream=stream, **masks)
         if record:
             ev[3].record(stream)
         lsh.lsh_combine_rounds(bufs["out_rounds"], bufs["lse_rounds"], out=bufs["out"], want_lse=False,
@@ -297,7 +310,7 @@ def run_ours(args, w, rank, world, local_rank):
         qk.copy_(qk_h, non_blocking=True)
         v.copy_(v_h, non_blocking=True)
         R.copy_(R_h, non_blocking=True)
-        lsh.lsh_attention(qk, v, R, w.n_buckets, w.chunk, causal=args.causal, stream=stream, bufs=bufs)
+        lsh.lsh_attention(qk, v, R, w.n_buckets, w.chunk, stream=stream, bufs=bufs, **masks)
         out_h.copy_(bufs["out"], non_blocking=True)
     e_end.record(stream)
     torch.cuda.synchronize()
@@ -338,12 +351,12 @@ def run_ours(args, w, rank, world, local_rank):
         sort_launches = 3 + (1 if w.n_buckets > 16384 else 0)  # count, scan, scatter (+ counter clear)
     launches_per_step = 3 + sort_launches                  # hash, sort, attend, combine
     sample_slices = 2  # about 10 s of float64 CPU work at the 64K workload
-    c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices, causal=args.causal)
+    c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices, masks=masks)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": dict(workload_config(w), **({"mask": "causal"} if args.causal else {})),
+        "config": dict(workload_config(w), **mask_config(args)),
         "roofline": {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": recorded_traffic(dominant, args.workload),
                      "peak_source": peak_src + (", sustained tensor peak" if bound == "tensor" else "")},
@@ -373,7 +386,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="64k")
     ap.add_argument("--causal", action="store_true",
-                    help="causal window (keys after the query's position masked; CUDA-core attention path)")
+                    help="causal window: keys after the query's position are masked")
+    ap.add_argument("--bucket-mask", action="store_true",
+                    help="keys outside the query's bucket are masked (CUDA-core attention path)")
+    ap.add_argument("--union", action="store_true",
+                    help="multi-round union correction (implies --bucket-mask; CUDA-core attention path)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

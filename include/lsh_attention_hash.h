@@ -68,8 +68,10 @@ typedef enum lsh_dtype { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
 
 /* Mask bits of lsh_chunk_attend. */
 typedef enum lsh_mask {
-  LSH_MASK_SELF = 1,   /* a slot does not see itself unless it is its only key */
-  LSH_MASK_CAUSAL = 2  /* a key after the query's original position is not admissible */
+  LSH_MASK_SELF = 1,    /* a slot does not see itself unless it is its only key */
+  LSH_MASK_CAUSAL = 2,  /* a key after the query's original position is not admissible */
+  LSH_MASK_BUCKET = 4,  /* a key in another bucket than the query's (this round) is not admissible */
+  LSH_MASK_UNION = 8    /* lower each logit by log(#rounds sharing the bucket); needs LSH_MASK_BUCKET */
 } lsh_mask;
 
 /* Version of this ABI (incremented on any signature change). */
@@ -178,6 +180,8 @@ LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H
  *
  *   qk, v      [B, H, L, D] dtype          in: shared query/key rows and values
  *   perm       [B, H, n_rounds, L] int32   in: from lsh_sort_permute
+ *   buckets    [B, H, n_rounds, L] int32   in, nullable: from lsh_hash (by original
+ *              position); required by LSH_MASK_BUCKET and LSH_MASK_UNION, else unread
  *   qk_sorted, v_sorted  nullable [B, H, n_rounds, L, D] dtype: when given, the
  *              rows are read in sorted order from them instead of through perm
  *   chunk      chunk length c, L % c == 0.  Chunk k = sorted slots
@@ -188,8 +192,15 @@ LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H
  *              original position perm[t] is after the query's perm[s] is not
  *              admissible (the pages' character-level language model; the self
  *              rule then applies to what remains, so a query with no earlier key
- *              in its window sees only itself).  Every mask runs on both the
- *              tensor-core and the CUDA-core path
+ *              in its window sees only itself); LSH_MASK_BUCKET (4): a key whose
+ *              bucket buckets[r][perm[t]] differs from the query's is not
+ *              admissible (the article's admissible set: the query's own bucket,
+ *              batched by chunks; self rule as for causal); LSH_MASK_UNION (8,
+ *              only with 4): each admissible logit is lowered by log N, N = the
+ *              number of rounds r' with buckets[r'][i] == buckets[r'][j] (the
+ *              article's multi-round union: lsh_combine_rounds then counts each
+ *              shared key once).  SELF and CAUSAL run on the tensor-core and the
+ *              CUDA-core path; BUCKET and UNION on the CUDA-core path
  *   scale      logit scale; <= 0 selects 1/sqrt(D).  logit(s, t) =
  *              scale * qk[perm[s]] . qk[perm[t]] / ||qk[perm[t]]||
  *   out_rounds [B, H, n_rounds, L, D] out_dtype  out: per-round softmax-weighted
@@ -201,7 +212,7 @@ LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H
  * 8 <= D <= 256, 1 <= chunk <= L.
  */
 LSH_API lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int H, int L,
-                            int D, int n_rounds, const int32_t* perm,
+                            int D, int n_rounds, const int32_t* perm, const int32_t* buckets,
                             const void* qk_sorted, const void* v_sorted, int chunk,
                             int mask, float scale, void* out_rounds, int out_dtype,
                             float* lse, void* stream);

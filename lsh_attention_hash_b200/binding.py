@@ -45,7 +45,7 @@ _SIGS = {
                                   _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp]),
     "lsh_sort_permute_noalloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "lsh_chunk_attend": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp,
-                                  _vp, _c_int, _c_int, _c_float, _vp, _c_int, _vp, _vp]),
+                                  _vp, _vp, _c_int, _c_int, _c_float, _vp, _c_int, _vp, _vp]),
     "lsh_combine_rounds": (_c_int, [_vp, _c_int, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp,
                                     _c_int, _vp, _vp]),
     "lsh_get_device_status": (_c_int, [_vp]),
@@ -190,11 +190,15 @@ def lsh_sort_permute_noalloc(buckets, n_buckets, *, perm=None, inv=None, want_in
     return perm, inv
 
 
-def lsh_chunk_attend(qk, v, perm, chunk, *, self_mask=True, causal=False, scale=None, qk_sorted=None,
-                     v_sorted=None, out_dtype=None, out_rounds=None, lse=None, stream=None):
+def lsh_chunk_attend(qk, v, perm, chunk, *, self_mask=True, causal=False, buckets=None, bucket_mask=False,
+                     union=False, scale=None, qk_sorted=None, v_sorted=None, out_dtype=None, out_rounds=None,
+                     lse=None, stream=None):
     """Per-round outputs [B,H,n_rounds,L,D] and log-sum-exp [B,H,n_rounds,L] in original order.
 
     ``causal``: keys after the query's original position are not admissible.
+    ``bucket_mask`` (needs ``buckets`` from ``lsh_hash``): keys outside the query's bucket
+    are not admissible.  ``union`` (with ``bucket_mask``): each logit is lowered by the log
+    of the number of rounds in which query and key share a bucket.
     """
     lib = load_library()
     _need(qk, "qk")
@@ -203,6 +207,12 @@ def lsh_chunk_attend(qk, v, perm, chunk, *, self_mask=True, causal=False, scale=
     _need(perm, "perm", torch.int32)
     n_rounds = perm.shape[2]
     _need(perm, "perm", torch.int32, (B, H, n_rounds, L))
+    if union and not bucket_mask:
+        raise ValueError("union needs bucket_mask")
+    if bucket_mask:
+        if buckets is None:
+            raise ValueError("bucket_mask needs buckets")
+        _need(buckets, "buckets", torch.int32, (B, H, n_rounds, L))
     if qk_sorted is not None or v_sorted is not None:
         _need(qk_sorted, "qk_sorted", qk.dtype, (B, H, n_rounds, L, D))
         _need(v_sorted, "v_sorted", qk.dtype, (B, H, n_rounds, L, D))
@@ -214,9 +224,10 @@ def lsh_chunk_attend(qk, v, perm, chunk, *, self_mask=True, causal=False, scale=
         lse = torch.empty((B, H, n_rounds, L), dtype=torch.float32, device=qk.device)
     _need(lse, "lse", torch.float32, (B, H, n_rounds, L))
     sc = 0.0 if scale is None else float(scale)
+    mask = (1 if self_mask else 0) | (2 if causal else 0) | (4 if bucket_mask else 0) | (8 if union else 0)
     _check(lib.lsh_chunk_attend(_ptr(qk), _ptr(v), _dt(qk), B, H, L, D, n_rounds, _ptr(perm),
-                                _ptr(qk_sorted), _ptr(v_sorted), int(chunk),
-                                (1 if self_mask else 0) | (2 if causal else 0), sc,
+                                _ptr(buckets) if bucket_mask else None, _ptr(qk_sorted), _ptr(v_sorted),
+                                int(chunk), mask, sc,
                                 _ptr(out_rounds), _DT[out_dtype], _ptr(lse), _stream(stream)),
            "lsh_chunk_attend")
     return out_rounds, lse
@@ -248,8 +259,8 @@ def lsh_get_device_status(stream=None) -> int:
     return int(load_library().lsh_get_device_status(_stream(stream)))
 
 
-def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, causal=False, scale=None, stream=None,
-                  return_all=False, bufs=None):
+def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, causal=False, bucket_mask=False, union=False,
+                  scale=None, stream=None, return_all=False, bufs=None):
     """The whole forward pass: hash, sort, chunk attention, round merge (four C-ABI calls).
 
     ``bufs`` may hold preallocated outputs (keys: buckets, near_tie, perm, workspace,
@@ -260,7 +271,8 @@ def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, causal=False, s
                              with_near_tie=return_all or "near_tie" in b, stream=stream)
     perm, _, _, _ = lsh_sort_permute(buckets, n_buckets, perm=b.get("perm"), workspace=b.get("workspace"),
                                      stream=stream)
-    o, lse = lsh_chunk_attend(qk, v, perm, chunk, self_mask=self_mask, causal=causal, scale=scale,
+    o, lse = lsh_chunk_attend(qk, v, perm, chunk, self_mask=self_mask, causal=causal, buckets=buckets,
+                              bucket_mask=bucket_mask, union=union, scale=scale,
                               out_rounds=b.get("out_rounds"), lse=b.get("lse_rounds"), stream=stream)
     out, lse_out = lsh_combine_rounds(o, lse, out=b.get("out"), lse_out=b.get("lse"),
                                       want_lse=return_all or "lse" in b, stream=stream)

@@ -186,7 +186,7 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
 
 extern "C" {
 
-int lsh_abi_version(void) { return 1; }
+int lsh_abi_version(void) { return 2; }
 
 const char* lsh_status_string(int s) {
   switch (s) {
@@ -377,17 +377,23 @@ lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H, int L,
 }
 
 lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int H, int L, int D,
-                            int n_rounds, const int32_t* perm, const void* qk_sorted,
-                            const void* v_sorted, int chunk, int mask, float scale,
+                            int n_rounds, const int32_t* perm, const int32_t* buckets,
+                            const void* qk_sorted, const void* v_sorted, int chunk, int mask, float scale,
                             void* out_rounds, int out_dtype, float* lse, void* stream) {
   if (!valid_dtype(dtype) || !valid_dtype(out_dtype)) return LSH_ERR_DTYPE;
   lsh_status st = check_bhld(B, H, L, D);
   if (st != LSH_OK) return st;
   if (n_rounds < 1 || !index_space_ok(B, H, L, n_rounds)) return LSH_ERR_SHAPE;
   if (chunk < 1 || (L > 0 && (chunk > L || L % chunk != 0))) return LSH_ERR_SHAPE;
-  if (mask < 0 || mask > (LSH_MASK_SELF | LSH_MASK_CAUSAL)) return LSH_ERR_INVALID_ARG;
+  if (mask < 0 || mask > (LSH_MASK_SELF | LSH_MASK_CAUSAL | LSH_MASK_BUCKET | LSH_MASK_UNION))
+    return LSH_ERR_INVALID_ARG;
   const int self_mask = (mask & LSH_MASK_SELF) ? 1 : 0;
   const int causal = (mask & LSH_MASK_CAUSAL) ? 1 : 0;
+  const int bucket_mask = (mask & LSH_MASK_BUCKET) ? 1 : 0;
+  const int union_count = (mask & LSH_MASK_UNION) ? 1 : 0;
+  if (union_count && !bucket_mask) return LSH_ERR_INVALID_ARG;
+  if (bucket_mask && !buckets) return LSH_ERR_INVALID_ARG;
+  if (buckets && !aligned16(buckets)) return LSH_ERR_ALIGN;
   if (!qk || !v || !perm || !out_rounds || !lse) return LSH_ERR_INVALID_ARG;
   if ((qk_sorted == nullptr) != (v_sorted == nullptr)) return LSH_ERR_INVALID_ARG;
   if (!aligned16(qk) || !aligned16(v) || !aligned16(perm) || !aligned16(out_rounds) ||
@@ -400,7 +406,8 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
   cudaStream_t s = as_stream(stream);
 
   const DevInfo di = dev_info();
-  if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && di.major == 10) {
+  if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && di.major == 10 &&
+      !bucket_mask) {
 #define LSH_ATT_TC(DD, TO)                                                                            \
   return causal ? launch_attend_tc<DD, TO, true>(qk, v, qk_sorted, v_sorted, perm, B, H, L, n_rounds, self_mask, \
                                                   scale, out_rounds, lse, s, di.sms)                         \
@@ -416,15 +423,17 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
 
   const int qb_per_chunk = (chunk + lsh::kAttQ - 1) / lsh::kAttQ;
   dim3 grid((unsigned)((L / chunk) * qb_per_chunk), (unsigned)segs);
-  const size_t smem = ((size_t)lsh::kAttQ * (D + 1) + lsh::kAttK * (D + 1) + lsh::kAttK * D + lsh::kAttK) * 4;
+  const size_t smem = ((size_t)lsh::kAttQ * (D + 1) + lsh::kAttK * (D + 1) + lsh::kAttK * D + lsh::kAttK +
+                        (union_count ? (size_t)n_rounds * (lsh::kAttK + lsh::kAttQ) : 0)) * 4;
+  if (smem > (size_t)227 * 1024) return LSH_ERR_UNSUPPORTED;  // union with very many rounds
   const int threads = lsh::kAttWarps * 32;
 #define LSH_ATT(T, TO)                                                                          \
   do {                                                                                           \
     auto kfn = lsh::attend_simt_kernel<T, TO>;                                                   \
     if (smem > 48 * 1024) cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-    kfn<<<grid, threads, smem, s>>>((const T*)qk, (const T*)v, perm, (const T*)qk_sorted,        \
-                                    (const T*)v_sorted, L, D, n_rounds, chunk, self_mask, causal, scale, \
-                                    (TO*)out_rounds, lse);                                       \
+    kfn<<<grid, threads, smem, s>>>((const T*)qk, (const T*)v, perm, buckets, (const T*)qk_sorted, \
+                                    (const T*)v_sorted, L, D, n_rounds, chunk, self_mask, causal,  \
+                                    bucket_mask, union_count, scale, (TO*)out_rounds, lse);      \
   } while (0)
   if (dtype == LSH_F32) {
     if (out_dtype == LSH_F32) LSH_ATT(float, float); else LSH_ATT(float, __nv_bfloat16);

@@ -46,8 +46,11 @@ def check_sort(g_buckets, g_perm):
     assert np.array_equal(o_p, np_(g_perm)), "perm differs from the oracle's sort of the same buckets"
 
 
-def check_attend(qk, v, g_perm, chunk, self_mask, scale, g_o, g_lse, dtype, causal=False):
-    o, lse = oracle_attend(f64(qk), f64(v), np_(g_perm), chunk, self_mask, scale, causal)
+def check_attend(qk, v, g_perm, chunk, self_mask, scale, g_o, g_lse, dtype, causal=False, g_buckets=None,
+                 union=False):
+    """g_buckets (the GPU's buckets), when given, selects the bucket-equality mask."""
+    o, lse = oracle_attend(f64(qk), f64(v), np_(g_perm), chunk, self_mask, scale, causal,
+                           None if g_buckets is None else np_(g_buckets), union)
     err_o = float(np.max(np.abs(o - f64(g_o)))) if o.size else 0.0
     err_l = float(np.max(np.abs(lse - f64(g_lse)))) if lse.size else 0.0
     tol = TOL[dtype]
@@ -68,13 +71,18 @@ def check_combine(g_o, g_lse, g_out, g_lse_out, dtype):
 
 
 def check_slice_rounds(qk_bh, v_bh, g_perm_bh, chunk, self_mask, scale, g_o_bh, g_lse_bh, dtype,
-                       slots=None):
-    """Per-round attention of one (b, h) slice at full size (all rounds, optional slot sample)."""
+                       slots=None, g_buckets_bh=None, union=False):
+    """Per-round attention of one (b, h) slice at full size (all rounds, optional slot sample).
+
+    g_buckets_bh ([n_rounds, L], the GPU's), when given, selects the bucket-equality mask."""
     n_rounds, L = g_perm_bh.shape
+    bk = None if g_buckets_bh is None else np_(g_buckets_bh)
     worst = 0.0
     for r in range(n_rounds):
         ss = np.arange(L) if slots is None else np.asarray(slots)
-        pos, o, lse = oracle_attend_slots(f64(qk_bh), f64(v_bh), np_(g_perm_bh[r]), chunk, ss, self_mask, scale)
+        pos, o, lse = oracle_attend_slots(f64(qk_bh), f64(v_bh), np_(g_perm_bh[r]), chunk, ss, self_mask, scale,
+                                          bucket_seg=None if bk is None else bk[r],
+                                          union_buckets=bk if union else None)
         go = f64(g_o_bh[r])[pos]
         gl = f64(g_lse_bh[r])[pos]
         e = max(float(np.max(np.abs(o - go))), float(np.max(np.abs(lse - gl))))

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(lib):
     assert len(names) >= 8
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.lsh_abi_version() == 1
+    assert lib.lsh_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -84,11 +84,11 @@ def test_sort_rejects_bad_arguments_before_launch(lib):
 
 def test_attend_rejects_bad_arguments_before_launch(lib):
     f = lib.lsh_chunk_attend
-    args = [A, A, BF16, 1, 1, 1024, 64, 1, A, None, None, 64, 1, 0.0, A, BF16, A, None]
+    args = [A, A, BF16, 1, 1, 1024, 64, 1, A, None, None, None, 64, 1, 0.0, A, BF16, A, None]
 
     def call(**kw):
         a = list(args)
-        names = ["qk", "v", "dtype", "B", "H", "L", "D", "nr", "perm", "qs", "vs", "chunk", "mask",
+        names = ["qk", "v", "dtype", "B", "H", "L", "D", "nr", "perm", "bk", "qs", "vs", "chunk", "mask",
                  "scale", "out", "out_dtype", "lse", "stream"]
         for k, val in kw.items():
             a[names.index(k)] = val
@@ -97,8 +97,12 @@ def test_attend_rejects_bad_arguments_before_launch(lib):
     assert call(chunk=48) == SHAPE        # 1024 % 48 != 0
     assert call(chunk=0) == SHAPE
     assert call(chunk=2048) == SHAPE      # chunk > L
-    assert call(mask=4) == INVALID        # bits beyond LSH_MASK_SELF | LSH_MASK_CAUSAL
+    assert call(mask=16) == INVALID       # bits beyond the four of lsh_mask
     assert call(mask=-1) == INVALID
+    assert call(mask=1 | 4) == INVALID    # bucket mask without buckets
+    assert call(mask=1 | 8, bk=A) == INVALID  # union without the bucket mask
+    assert call(mask=1 | 4, bk=A + 4) == ALIGN
+    assert call(mask=1 | 4 | 8, bk=A, L=0) == OK
     assert call(out_dtype=5) == DTYPE
     assert call(qs=A) == INVALID          # sorted qk without sorted v
     assert call(lse=None) == INVALID

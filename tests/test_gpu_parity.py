@@ -21,10 +21,10 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def run_gpu(w, qk, v, R, self_mask=True, scale=None, out_dtype=None):
+def run_gpu(w, qk, v, R, self_mask=True, scale=None, out_dtype=None, **masks):
     qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
     res = lsh.lsh_attention(qk_d, v_d, R_d, w.n_buckets, w.chunk, self_mask=self_mask, scale=scale,
-                            return_all=True)
+                            return_all=True, **masks)
     torch.cuda.synchronize()
     assert lsh.lsh_get_device_status() == 0
     return res
@@ -192,9 +192,9 @@ def test_out_of_range_bucket_is_recorded_not_faulted():
     assert p[:1022].tolist() == [i for i in range(1024) if i not in (10, 11)]
 
 
-def _sampled_slices(w, slices, row_sample=None, slot_sample=None):
+def _sampled_slices(w, slices, row_sample=None, slot_sample=None, bucket_mask=False, union=False):
     qk, v, R = synth.make_inputs(w)
-    res = run_gpu(w, qk, v, R)
+    res = run_gpu(w, qk, v, R, bucket_mask=bucket_mask, union=union)
     for (b, h) in slices:
         qk_bh, v_bh = qk[b, h], v[b, h]
         rows = np.arange(w.L) if row_sample is None else np.sort(
@@ -208,7 +208,7 @@ def _sampled_slices(w, slices, row_sample=None, slot_sample=None):
             np.random.default_rng(b * 7 + h).choice(w.L, slot_sample, replace=False))
         parity.check_slice_rounds(qk_bh, v_bh, res["perm"][b, h].cpu(), w.chunk, True, None,
                                   res["o_rounds"][b, h].cpu(), res["lse_rounds"][b, h].cpu(), w.torch_dtype,
-                                  slots)
+                                  slots, g_b if bucket_mask else None, union)
         parity.check_combine(res["o_rounds"][b, h][None, None], res["lse_rounds"][b, h][None, None],
                              res["out"][b, h][None, None], res["lse"][b, h][None, None], w.torch_dtype)
     return res
@@ -279,3 +279,59 @@ def test_causal_tensor_core_attention_scales(scale):
     torch.cuda.synchronize()
     assert lsh.lsh_get_device_status() == 0
     parity.check_attend(qk, v, perm, w.chunk, True, scale, o, l, w.torch_dtype, causal=True)
+
+
+# ------------------------------------------------- bucket-equality mask and union
+@pytest.mark.parametrize("name,shape,causal,union", [
+    ("bucket_tiny", (1, 1, 64, 32, "f32", 8, 8, 2), False, False),
+    ("bucket_union_f32", (1, 2, 512, 64, "f32", 4, 32, 8), False, True),     # few buckets: many shared rounds
+    ("bucket_union_bf16", (2, 2, 2048, 128, "bf16", 32, 64, 4), False, True),
+    ("bucket_dense", (1, 2, 256, 64, "bf16", 16, 256, 2), False, False),     # chunk = L
+    ("bucket_chunk1", (1, 1, 64, 32, "f32", 8, 1, 2), False, True),          # every window has two slots
+    ("bucket_union_causal", (1, 3, 320, 64, "bf16", 8, 32, 3), True, True),
+    ("bucket_many", (1, 1, 4096, 128, "bf16", 1024, 64, 2), False, True),    # most buckets split or alone
+])
+def test_bucket_mask_attention_end_to_end(name, shape, causal, union):
+    """Keys outside the query's bucket are not admissible (a query alone in its bucket sees only
+    itself); with the union correction each logit is lowered by log(#rounds sharing the bucket).
+    Checked stage by stage and end to end against the oracle."""
+    w = synth.small_workload(name, *shape)
+    qk, v, R = synth.make_inputs(w, seed=zlib.crc32(name.encode()) % 1000)
+    qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
+    res = lsh.lsh_attention(qk_d, v_d, R_d, w.n_buckets, w.chunk, causal=causal, bucket_mask=True, union=union,
+                            return_all=True)
+    torch.cuda.synchronize()
+    assert lsh.lsh_get_device_status() == 0
+    mism, _ = parity.check_hash(qk, R, w.n_buckets, res["buckets"], res["near_tie"], 1e-3)
+    parity.check_sort(res["buckets"], res["perm"])
+    parity.check_attend(qk, v, res["perm"], w.chunk, True, None, res["o_rounds"], res["lse_rounds"],
+                        w.torch_dtype, causal=causal, g_buckets=res["buckets"], union=union)
+    parity.check_combine(res["o_rounds"], res["lse_rounds"], res["out"], res["lse"], w.torch_dtype)
+    if mism == 0:
+        from oracle import oracle_lsh_attention
+
+        ref = oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, causal=causal, bucket_mask=True, union=union)
+        err = float(np.max(np.abs(ref["out"] - parity.f64(res["out"]))))
+        assert err <= parity.TOL[w.torch_dtype], err
+
+
+def test_bucket_mask_without_self_mask_and_custom_scale():
+    """self_mask off: a query always sees itself (it shares its own bucket); scale 3."""
+    w = synth.small_workload("bucket_noself", 1, 2, 1024, 64, "f32", 16, 32, 3)
+    qk, v, R = synth.make_inputs(w, seed=5)
+    qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
+    b, _ = lsh.lsh_hash(qk_d, R_d, w.n_buckets)
+    perm, _, _, _ = lsh.lsh_sort_permute(b, w.n_buckets)
+    o, l = lsh.lsh_chunk_attend(qk_d, v_d, perm, w.chunk, self_mask=False, buckets=b, bucket_mask=True,
+                                union=True, scale=3.0)
+    torch.cuda.synchronize()
+    assert lsh.lsh_get_device_status() == 0
+    parity.check_attend(qk, v, perm, w.chunk, False, 3.0, o, l, w.torch_dtype, g_buckets=b, union=True)
+
+
+@pytest.mark.slow
+def test_64k_workload_bucket_union_sampled_slices():
+    """The full-size launch (B 8, H 8, L 65536, D 128, bf16, 1024 buckets, chunk 64, 8 rounds) with
+    the bucket mask and the union correction, on sampled slots of two slices."""
+    w = synth.WORKLOADS["64k"]
+    _sampled_slices(w, [(0, 0), (7, 7)], slot_sample=2048, bucket_mask=True, union=True)

@@ -63,6 +63,10 @@ constexpr uint32_t kOOff = 96;      // O columns inside a step buffer
 template <int D>
 __host__ __device__ constexpr uint32_t lr_col() { return kOOff + D; }
 
+// Compile-time masks of an instantiation (besides the self mask, a runtime flag).
+constexpr int kMaskCausal = 1;  // a key after the query's original position is not admissible
+constexpr int kMaskBucket = 2;  // a key in another bucket than the query's is not admissible
+
 template <int D>
 struct Layout {
   static constexpr int kHalves = D / 64;
@@ -73,7 +77,8 @@ struct Layout {
   static constexpr uint32_t kOnes = 2 * kSlots * kSlotBytes;        // 16 x 128 B of bf16 1.0 (row sums)
   static constexpr uint32_t kPerm = kOnes + 16 * 128;               // int32 [kSlots][128]
   static constexpr uint32_t kColMul = kPerm + kSlots * kRows * 4;   // float [kSlots][128]
-  static constexpr uint32_t kBar = kColMul + kSlots * kRows * 4;
+  static constexpr uint32_t kBk = kColMul + kSlots * kRows * 4;     // int32 [kSlots][128] (bucket mask)
+  static constexpr uint32_t kBar = kBk + kSlots * kRows * 4;
   // full[3] empty[3] cm_full[3] s_full[2] p_ready[2] o_full[2] buf_empty[2] done
   static constexpr int kNumBars = 18;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;   // tmem base, abort flag
@@ -83,6 +88,7 @@ struct Layout {
 
 struct Params {
   const int32_t* perm;   // [segs][L]
+  const int32_t* buckets;  // [segs][L] by original position (bucket mask only)
   void* out;             // [segs][L][D]
   float* lse;            // [segs][L]
   int L;
@@ -267,7 +273,7 @@ __device__ __forceinline__ void fill_positions(const Params& p, const Fill& f, i
 // and its 16-byte piece c at ((c ^ (r % 8)) * 16), the 128-byte swizzle the
 // UMMA descriptors expect.  Every producer lane then arrives on `full_bar`
 // when its copies have landed.
-template <int D>
+template <int D, bool BUCKET>
 __device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, uint64_t* full_bar, int slot,
                                               const Fill& f, int pw, const int (&pos)[2]) {
   using Lay = Layout<D>;
@@ -284,6 +290,8 @@ __device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, ui
       const int i = base + 32 * k + lane;
       const int chunk = (i - f.row0) < 64 ? f.cA : f.cB;
       perm_s[i] = pos[k];
+      if (BUCKET)  // the row's bucket lands with the row (same cp.async group, same barrier)
+        tc::cp_async4(tc::smem_u32(smem + Lay::kBk) + (slot * kRows + i) * 4, p.buckets + f.seg * p.L + pos[k]);
       grow[k] = p.sorted_input ? f.seg * p.L + chunk * kC + (i & 63) : (f.seg / p.n_rounds) * p.L + pos[k];
     }
     const uint32_t qk_dst = tc::smem_u32(smem + Lay::kQK + slot * Lay::kSlotBytes);
@@ -325,16 +333,20 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
 // One pass of the softmax over a row's 128 keys (four groups of 32 S columns,
 // the next group's TMEM load in flight while the current one is processed):
 // w = 2^(S * colmul - m) in fp32 (self masked, a missing previous chunk dead,
-// with CAUSAL a key after the query's original position masked), l += w, and
+// with CAUSAL a key after the query's original position masked, with BUCKET a
+// key outside the query's bucket masked), l += w, and
 // the weights go to P as bf16 pairs right away: P's group g lands on S columns
-// whose values this row has already consumed.  With CAUSAL, `earlier` counts
-// the admissible keys other than self and `self_w` keeps the P words of the
+// whose values this row has already consumed.  With MASK bits, `others`
+// counts the admissible keys (CAUSAL: the earlier ones; BUCKET alone: those of
+// the query's bucket, self included) and `self_w` keeps the P words of the
 // self group (for the self-only fix-up).
-template <int D, bool CAUSAL>
+template <int D, int MASK>
 __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint32_t pcol, const float* cm_lo,
                                              const float* cm_hi, int g_first, int g_self, int lane, int self_mask,
                                              float m, float& l, const uint32_t (&g0)[32], const int32_t* kp_lo,
-                                             const int32_t* kp_hi, int qpos, int& earlier, uint32_t (&self_w)[16]) {
+                                             const int32_t* kp_hi, int qpos, const int32_t* kb_lo,
+                                             const int32_t* kb_hi, int qb, int& others, uint32_t (&self_w)[16]) {
+  constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
   uint32_t ra[32], rb[32];
 #pragma unroll
   for (int e = 0; e < 32; ++e) ra[e] = g0[e];  // group 0, loaded by the caller
@@ -346,6 +358,7 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
     // key multipliers as 16-byte loads (each group's 32 floats start on a 16-byte boundary)
     const float4* cm4 = reinterpret_cast<const float4*>(g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2));
     const int4* kp4 = reinterpret_cast<const int4*>(g < 2 ? kp_lo + 32 * g : kp_hi + 32 * (g - 2));
+    const int4* kb4 = reinterpret_cast<const int4*>(g < 2 ? kb_lo + 32 * g : kb_hi + 32 * (g - 2));
     const bool dead = g < g_first;
     uint32_t w16[16];
 #pragma unroll
@@ -353,12 +366,25 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
       const float4 c4 = cm4[e >> 2];
       float v0 = __uint_as_float(cur[e]) * ((e & 2) ? c4.z : c4.x);
       float v1 = __uint_as_float(cur[e + 1]) * ((e & 2) ? c4.w : c4.y);
-      if (CAUSAL) {  // keys are distinct tokens: position == qpos only for self
-        const int4 k4 = kp4[e >> 2];
-        const int p0 = (e & 2) ? k4.z : k4.x, p1 = (e & 2) ? k4.w : k4.y;
-        if (p0 > qpos) v0 = -INFINITY;
-        if (p1 > qpos) v1 = -INFINITY;
-        if (!dead) earlier += (p0 < qpos) + (p1 < qpos);
+      if (CAUSAL || BUCKET) {  // keys are distinct tokens: position == qpos only for self
+        bool c0 = true, c1 = true;  // counted: admissible and (CAUSAL) not self
+        if (CAUSAL) {
+          const int4 k4 = kp4[e >> 2];
+          const int p0 = (e & 2) ? k4.z : k4.x, p1 = (e & 2) ? k4.w : k4.y;
+          if (p0 > qpos) v0 = -INFINITY;
+          if (p1 > qpos) v1 = -INFINITY;
+          c0 = p0 < qpos;
+          c1 = p1 < qpos;
+        }
+        if (BUCKET) {
+          const int4 b4 = kb4[e >> 2];
+          const int b0 = (e & 2) ? b4.z : b4.x, b1 = (e & 2) ? b4.w : b4.y;
+          if (b0 != qb) v0 = -INFINITY;
+          if (b1 != qb) v1 = -INFINITY;
+          c0 = c0 && b0 == qb;
+          c1 = c1 && b1 == qb;
+        }
+        if (!dead) others += (int)c0 + (int)c1;
       }
       if (g == g_self && self_mask) {
         if (e == lane) v0 = -INFINITY;
@@ -370,7 +396,7 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
       w16[e >> 1] = tc::pack_bf16x2(a, c);
     }
     tc::tmem_st16(sbuf + pcol + 16 * g, w16);
-    if (CAUSAL && g >= 2 && g == g_self) {
+    if ((CAUSAL || BUCKET) && g >= 2 && g == g_self) {
 #pragma unroll
       for (int k = 0; k < 16; ++k) self_w[k] = w16[k];
     }
@@ -378,13 +404,16 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
   }
 }
 
-// Causal rows with no earlier key in their window see only themselves: their P
-// becomes one-hot at the own key (bf16 1.0 at element `lane` of the self group)
-// and their weight sum 1 (the shift m is their own logit).  The whole warp
-// rewrites the self group, the other rows with the words they already had.
-__device__ __forceinline__ void causal_self_only(uint32_t sbuf, uint32_t pcol, int g_self, int lane, int earlier,
-                                                 const uint32_t (&self_w)[16], float& l) {
-  const bool only = earlier == 0;
+// Rows with no admissible key but themselves (causal: no earlier key; bucket:
+// alone in their bucket inside the window) see only themselves: their P becomes
+// one-hot at the own key (bf16 1.0 at element `lane` of the self group) and
+// their weight sum 1 (the shift m is their own logit).  The whole warp rewrites
+// the self group, the other rows with the words they already had.  `others`
+// counts self too when only the bucket mask is on.
+template <int MASK>
+__device__ __forceinline__ void self_only_fixup(uint32_t sbuf, uint32_t pcol, int g_self, int lane, int others,
+                                                const uint32_t (&self_w)[16], float& l) {
+  const bool only = (MASK & kMaskCausal) ? others == 0 : others <= 1;
   if (!__any_sync(0xffffffffu, only)) return;
   uint32_t w16[16];
 #pragma unroll
@@ -395,11 +424,13 @@ __device__ __forceinline__ void causal_self_only(uint32_t sbuf, uint32_t pcol, i
 }
 
 // Exact maximum of a row's scaled logits (self excluded while it has other keys;
-// with CAUSAL, keys after the query's position excluded).
-template <bool CAUSAL>
+// with MASK bits, keys after the query's position / outside its bucket excluded).
+template <int MASK>
 __device__ __forceinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const float* cm_lo, const float* cm_hi,
                                                int g_first, int g_self, int lane, int self_mask,
-                                               const int32_t* kp_lo, const int32_t* kp_hi, int qpos) {
+                                               const int32_t* kp_lo, const int32_t* kp_hi, int qpos,
+                                               const int32_t* kb_lo, const int32_t* kb_hi, int qb) {
+  constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
   float m = -INFINITY;
 #pragma unroll 1
   for (int g = 0; g < 4; ++g) {
@@ -409,10 +440,12 @@ __device__ __forceinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, con
     if (g < g_first) continue;
     const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
     const int32_t* kp = g < 2 ? kp_lo + 32 * g : kp_hi + 32 * (g - 2);
+    const int32_t* kb = g < 2 ? kb_lo + 32 * g : kb_hi + 32 * (g - 2);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       float v = __uint_as_float(raw[e]) * cm[e];
       if (CAUSAL && kp[e] > qpos) v = -INFINITY;
+      if (BUCKET && kb[e] != qb) v = -INFINITY;
       if (g == g_self && self_mask && e == lane) v = -INFINITY;
       m = fmaxf(m, v);
     }
@@ -458,9 +491,10 @@ __device__ __noinline__ void restore_s(const uint8_t* smem, uint32_t sbuf, uint3
   tc::tmem_wait_st();
 }
 
-template <int D, typename TO, bool CAUSAL>
+template <int D, typename TO, int MASK>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) {
   using Lay = Layout<D>;
+  constexpr bool MASKED = MASK != 0;  // a self-only fix-up may be needed
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
@@ -476,6 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
   float* colmul = reinterpret_cast<float*>(smem + Lay::kColMul);
   const int32_t* perm_s = reinterpret_cast<const int32_t*>(smem + Lay::kPerm);
+  const int32_t* bk_s = reinterpret_cast<const int32_t*>(smem + Lay::kBk);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -548,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       const Fill cur = it0.get(p);
       const int slot = f % kSlots;
       if (!warp_wait(&empty[slot], ((f / kSlots) & 1) ^ 1, abort_flag)) break;
-      producer_fill<D>(p, smem, &full[slot], slot, cur, pw, pos0);
+      producer_fill<D, (MASK & kMaskBucket) != 0>(p, smem, &full[slot], slot, cur, pw, pos0);
       ++f;
       it0 = it1;
       it1 = it2;
@@ -681,31 +716,35 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       const float* cm_hi = low ? colmul + sc * kRows : colmul + sc * kRows + 64;  // keys 64..127
       const int32_t* kp_lo = low ? perm_s + sp * kRows + 64 : perm_s + sc * kRows;  // their positions
       const int32_t* kp_hi = low ? perm_s + sc * kRows : perm_s + sc * kRows + 64;
-      int earlier = 0;
+      const int32_t* kb_lo = low ? bk_s + sp * kRows + 64 : bk_s + sc * kRows;      // their buckets
+      const int32_t* kb_hi = low ? bk_s + sc * kRows : bk_s + sc * kRows + 64;
+      const int qb = (MASK & kMaskBucket) ? bk_s[sc * kRows + r] : 0;
+      int others = 0;
       uint32_t self_w[16];
       const int g_first = (low && it.j == 0) ? 2 : 0;  // chunk 0 has no previous chunk
       // shift: ||q|| * scale * log2(e) bounds every logit of the row (log2 domain)
       float m = diag * cm_own;
       float l = 0.f;  // sum of the weights (log-sum-exp); O is normalised by the rounded weights' sum
       const uint32_t pcol = low ? 0 : 32;  // P column of the row's first key
-      softmax_pass<D, CAUSAL>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0, kp_lo,
-                              kp_hi, pos, earlier, self_w);
-      if (CAUSAL) causal_self_only(sbuf, pcol, g_self, lane, earlier, self_w, l);
+      softmax_pass<D, MASK>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0, kp_lo,
+                            kp_hi, pos, kb_lo, kb_hi, qb, others, self_w);
+      if (MASKED) self_only_fixup<MASK>(sbuf, pcol, g_self, lane, others, self_w, l);
       if (__any_sync(0xffffffffu, !(l > 1e-30f))) {
         // the bound was too loose for some row of the warp (long query rows): S is
         // rebuilt in TMEM from the rows in shared memory (P has overwritten part of
         // it) and the warp's rows are redone with their exact maxima
         restore_s<D>(smem, sbuf, scol, sp, sc, r, low);
         const float m_cs = m;
-        m = exact_row_max<CAUSAL>(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, kp_lo, kp_hi, pos);
-        if (CAUSAL && m == -INFINITY) m = m_cs;  // self-only row: its own logit is the shift
+        m = exact_row_max<MASK>(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, kp_lo, kp_hi, pos,
+                                kb_lo, kb_hi, qb);
+        if (MASKED && m == -INFINITY) m = m_cs;  // self-only row: its own logit is the shift
         l = 0.f;
-        earlier = 0;
+        others = 0;
         tc::tmem_ld32(sbuf + scol, sg0);
         tc::tmem_wait_ld_regs(sg0);
-        softmax_pass<D, CAUSAL>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0,
-                                kp_lo, kp_hi, pos, earlier, self_w);
-        if (CAUSAL) causal_self_only(sbuf, pcol, g_self, lane, earlier, self_w, l);
+        softmax_pass<D, MASK>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0,
+                              kp_lo, kp_hi, pos, kb_lo, kb_hi, qb, others, self_w);
+        if (MASKED) self_only_fixup<MASK>(sbuf, pcol, g_self, lane, others, self_w, l);
       }
       {
         uint32_t z[32];

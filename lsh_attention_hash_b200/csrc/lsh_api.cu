@@ -149,15 +149,16 @@ lsh_status dispatch_hash_tc(const void* qk, const void* R, int B, int H, int L, 
 }
 
 // Tensor-core chunk attention (bf16, chunk 64, D 64 or 128) on sm_100.
-template <int D, typename TO, bool CAUSAL>
+template <int D, typename TO, int MASK>
 lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted, const void* v_sorted,
-                            const int32_t* perm, int B, int H, int L, int n_rounds, int self_mask, float scale,
-                            void* out, float* lse, cudaStream_t s, int sms) {
+                            const int32_t* perm, const int32_t* buckets, int B, int H, int L, int n_rounds,
+                            int self_mask, float scale, void* out, float* lse, cudaStream_t s, int sms) {
   using namespace lsh::att_tc;
   const long long segs = (long long)B * H * n_rounds;
   const bool sorted = qk_sorted != nullptr;
   Params p;
   p.perm = perm;
+  p.buckets = buckets;
   p.out = out;
   p.lse = lse;
   p.L = L;
@@ -174,7 +175,7 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
   p.v = (const uint8_t*)(sorted ? v_sorted : v);
   p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   const unsigned grid = (unsigned)std::min<long long>(p.n_units, sms);
-  auto kfn = attend_tc_kernel<D, TO, CAUSAL>;
+  auto kfn = attend_tc_kernel<D, TO, MASK>;
   const int smem = (int)Layout<D>::kSmem;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LSH_ERR_CUDA;
@@ -407,18 +408,26 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
 
   const DevInfo di = dev_info();
   if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && di.major == 10 &&
-      !bucket_mask) {
-#define LSH_ATT_TC(DD, TO)                                                                            \
-  return causal ? launch_attend_tc<DD, TO, true>(qk, v, qk_sorted, v_sorted, perm, B, H, L, n_rounds, self_mask, \
-                                                  scale, out_rounds, lse, s, di.sms)                         \
-                : launch_attend_tc<DD, TO, false>(qk, v, qk_sorted, v_sorted, perm, B, H, L, n_rounds, self_mask, scale, \
-                                  out_rounds, lse, s, di.sms)
+      !union_count) {
+    using lsh::att_tc::kMaskBucket;
+    using lsh::att_tc::kMaskCausal;
+#define LSH_ATT_TC_M(DD, TO, MM)                                                                            \
+  return launch_attend_tc<DD, TO, MM>(qk, v, qk_sorted, v_sorted, perm, buckets, B, H, L, n_rounds, self_mask, \
+                                      scale, out_rounds, lse, s, di.sms)
+#define LSH_ATT_TC(DD, TO)                                                              \
+  do {                                                                                  \
+    if (causal && bucket_mask) LSH_ATT_TC_M(DD, TO, kMaskCausal | kMaskBucket);         \
+    if (causal) LSH_ATT_TC_M(DD, TO, kMaskCausal);                                      \
+    if (bucket_mask) LSH_ATT_TC_M(DD, TO, kMaskBucket);                                 \
+    LSH_ATT_TC_M(DD, TO, 0);                                                            \
+  } while (0)
     if (D == 128) {
       if (out_dtype == LSH_BF16) LSH_ATT_TC(128, __nv_bfloat16); else LSH_ATT_TC(128, float);
     } else {
       if (out_dtype == LSH_BF16) LSH_ATT_TC(64, __nv_bfloat16); else LSH_ATT_TC(64, float);
     }
 #undef LSH_ATT_TC
+#undef LSH_ATT_TC_M
   }
 
   const int qb_per_chunk = (chunk + lsh::kAttQ - 1) / lsh::kAttQ;

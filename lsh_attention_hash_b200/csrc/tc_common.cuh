@@ -106,6 +106,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 
+__device__ __forceinline__ void cp_async4(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+
 // Arrives on `bar` once every cp.async this thread issued so far has landed
 // (the arrival counts toward the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {

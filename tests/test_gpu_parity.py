@@ -290,6 +290,11 @@ def test_causal_tensor_core_attention_scales(scale):
     ("bucket_chunk1", (1, 1, 64, 32, "f32", 8, 1, 2), False, True),          # every window has two slots
     ("bucket_union_causal", (1, 3, 320, 64, "bf16", 8, 32, 3), True, True),
     ("bucket_many", (1, 1, 4096, 128, "bf16", 1024, 64, 2), False, True),    # most buckets split or alone
+    # tensor-core path (bf16, chunk 64, D 64 / 128, no union)
+    ("bucket_tc", (2, 2, 4096, 128, "bf16", 64, 64, 2), False, False),
+    ("bucket_tc_many", (1, 2, 4096, 128, "bf16", 1024, 64, 2), False, False),  # many rows alone
+    ("bucket_tc_causal_d64_odd", (1, 2, 8256, 64, "bf16", 128, 64, 2), True, False),
+    ("bucket_tc_3heads", (1, 3, 2048, 64, "bf16", 32, 64, 3), False, False),
 ])
 def test_bucket_mask_attention_end_to_end(name, shape, causal, union):
     """Keys outside the query's bucket are not admissible (a query alone in its bucket sees only
@@ -335,3 +340,27 @@ def test_64k_workload_bucket_union_sampled_slices():
     the bucket mask and the union correction, on sampled slots of two slices."""
     w = synth.WORKLOADS["64k"]
     _sampled_slices(w, [(0, 0), (7, 7)], slot_sample=2048, bucket_mask=True, union=True)
+
+
+@pytest.mark.parametrize("scale,self_mask", [(None, False), (6.0, True), (40.0, True)])
+def test_bucket_mask_tensor_core_attention_scales(scale, self_mask):
+    """The tensor-core attention with the bucket mask (bf16, chunk 64): rows alone in their bucket
+    see only themselves; at scale 40 the Cauchy-Schwarz shift underflows and the exact-maximum path
+    (with the bucket mask) takes over."""
+    w = synth.small_workload("bucket_tc_scale", 2, 2, 4096, 128, "bf16", 256, 64, 2)
+    qk, v, R = synth.make_inputs(w, seed=33)
+    qk_d, v_d, R_d = qk.to(DEV), v.to(DEV), R.to(DEV)
+    b, _ = lsh.lsh_hash(qk_d, R_d, w.n_buckets)
+    perm, _, _, _ = lsh.lsh_sort_permute(b, w.n_buckets)
+    o, l = lsh.lsh_chunk_attend(qk_d, v_d, perm, w.chunk, self_mask=self_mask, buckets=b, bucket_mask=True,
+                                scale=scale)
+    torch.cuda.synchronize()
+    assert lsh.lsh_get_device_status() == 0
+    parity.check_attend(qk, v, perm, w.chunk, self_mask, scale, o, l, w.torch_dtype, g_buckets=b)
+
+
+@pytest.mark.slow
+def test_64k_workload_bucket_mask_sampled_slices():
+    """The full-size launch with the bucket mask alone (tensor-core path), sampled slots of two slices."""
+    w = synth.WORKLOADS["64k"]
+    _sampled_slices(w, [(0, 0), (7, 7)], slot_sample=2048, bucket_mask=True)

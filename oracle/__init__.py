@@ -20,4 +20,5 @@ from .lsh_oracle import (  # noqa: F401
     oracle_attend_slots,
     oracle_combine,
     oracle_lsh_attention,
+    oracle_attend_backward,
 )

@@ -149,9 +149,11 @@ def _window_slots(k: int, chunk: int) -> np.ndarray:
     return np.arange(max(k - 1, 0) * chunk, (k + 1) * chunk)
 
 
-def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale, causal=False, bucket_seg=None,
+def _chunk_logits(x, k_hat, perm_seg, k, chunk, self_mask, scale, causal=False, bucket_seg=None,
                   union_buckets=None):
-    """Outputs of the queries of sorted chunk k of one (b, h, round) segment.
+    """Logits of the queries of sorted chunk k against its window, -inf where not admissible.
+
+    Returns (qi [c] original positions of the queries, kj [|W|] of the keys, logits [c, |W|]).
 
     causal: a key whose original position is after the query's is not
     admissible (the language-model reading of the window).  bucket_seg (the
@@ -161,8 +163,6 @@ def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale, causal=Fals
     round's bucket by original position), when given: each admissible logit is
     lowered by log N, N = the number of rounds whose hash puts query and key in
     the same bucket (the self pair: every round).
-
-    Returns (orig positions [c], o [c, D], lse [c]).
     """
     q_slots = np.arange(k * chunk, (k + 1) * chunk)
     w_slots = _window_slots(k, chunk)
@@ -183,6 +183,15 @@ def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale, causal=Fals
         n_shared = np.sum(ub[:, kj][:, None, :] == ub[:, qi][:, :, None], axis=0)  # [c, |W|]
         logits[adm] -= np.log(n_shared[adm])
     logits[~adm] = -np.inf
+    return qi, kj, logits
+
+
+def _attend_chunk(x, k_hat, v, perm_seg, k, chunk, self_mask, scale, causal=False, bucket_seg=None,
+                  union_buckets=None):
+    """Outputs of the queries of sorted chunk k of one (b, h, round) segment (masks as in
+    ``_chunk_logits``).  Returns (orig positions [c], o [c, D], lse [c])."""
+    qi, kj, logits = _chunk_logits(x, k_hat, perm_seg, k, chunk, self_mask, scale, causal, bucket_seg,
+                                   union_buckets)
     m = np.max(logits, axis=1, keepdims=True)
     lse = m[:, 0] + np.log(np.sum(np.exp(logits - m), axis=1))
     weights = np.exp(logits - lse[:, None])
@@ -285,6 +294,68 @@ def oracle_combine(o, lse):
     w = np.exp(lse - big[:, :, None, :])
     out = np.sum(w[..., None] * o, axis=2)
     return out, big
+
+
+# ----------------------------------------------------------------------------
+# backward  [the forward above, differentiated by the chain rule with the hash,
+#            the sort and the masks held fixed (a bucket is a piecewise-constant
+#            function of x); GLOSSARY / ZH-ICLR: training through LSH attention
+#            recomputes from the stored buckets]
+# ----------------------------------------------------------------------------
+def oracle_attend_backward(qk, v, perm, chunk: int, dout, self_mask: bool = True, scale: float | None = None,
+                           causal: bool = False, buckets=None, union: bool = False):
+    """Gradients (dqk, dv) [B, H, L, D] float64 of sum(dout * out) for the merged output.
+
+    The forward is recomputed here: per-round (o_r, lse_r), then out and LSE.  Chain rule:
+
+      merge: out = sum_r w_r o_r, w_r = exp(lse_r - LSE)
+             d o_r = w_r dout;  d lse_r = w_r (dout . o_r - dout . out)
+      round: o = sum_j p_j v_j, p_j = exp(z_j - lse), lse = log sum_j exp(z_j)
+             d v_j += p_j d o;  d z_j = p_j (d o . v_j - d o . o) + p_j d lse
+      logit: z_ij = scale * x_i . k_j (less log N under the union correction, a constant),
+             k_j = x_j / max(||x_j||, 1e-12)
+             d x_i += scale * sum_j dz_ij k_j                          (query role)
+             d k_j  = scale * sum_i dz_ij x_i
+             d x_j += (d k_j - (d k_j . k_j) k_j) / ||x_j||            (key role; the clamp's
+                      linear branch d k_j / 1e-12 when ||x_j|| < 1e-12)
+    """
+    qk = _f64(qk)
+    v = _f64(v)
+    dout = _f64(dout)
+    B, H, L, D = qk.shape
+    perm = np.asarray(perm)
+    n_rounds = perm.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o, lse = oracle_attend(qk, v, perm, chunk, self_mask, scale, causal, buckets, union)
+    out, big = oracle_combine(o, lse)
+    w = np.exp(lse - big[:, :, None, :])                                    # [B, H, R, L]
+    d_o = w[..., None] * dout[:, :, None]                                   # [B, H, R, L, D]
+    d_lse = w * (np.sum(dout[:, :, None] * o, axis=-1) - np.sum(dout * out, axis=-1)[:, :, None])
+    bk = None if buckets is None else np.asarray(buckets)
+    dqk = np.zeros((B, H, L, D))
+    dv = np.zeros((B, H, L, D))
+    for b in range(B):
+        for h in range(H):
+            x, k_hat, vv = _prep_slice(qk[b, h], v[b, h])
+            norms = np.sqrt(np.sum(x * x, axis=1))
+            dk_hat = np.zeros((L, D))
+            for r in range(n_rounds):
+                for k in range(L // chunk):
+                    qi, kj, z = _chunk_logits(x, k_hat, perm[b, h, r], k, chunk, self_mask, scale, causal,
+                                              None if bk is None else bk[b, h, r], bk[b, h] if union else None)
+                    p = np.exp(z - lse[b, h, r, qi][:, None])                   # [c, |W|]
+                    g = d_o[b, h, r, qi]                                        # [c, D]
+                    dv[b, h, kj] += p.T @ g
+                    dz = p * (g @ vv[kj].T - np.sum(g * o[b, h, r, qi], axis=1)[:, None]) \
+                        + p * d_lse[b, h, r, qi][:, None]
+                    dqk[b, h, qi] += scale * dz @ k_hat[kj]
+                    dk_hat[kj] += scale * dz.T @ x[qi]
+            small = norms < 1e-12
+            proj = np.sum(dk_hat * k_hat, axis=1, keepdims=True) * k_hat
+            dqk[b, h] += np.where(small[:, None], dk_hat / 1e-12,
+                                  (dk_hat - proj) / np.maximum(norms, 1e-12)[:, None])
+    return dqk, dv
 
 
 def oracle_lsh_attention(qk, v, R, n_buckets: int, chunk: int, self_mask: bool = True,

@@ -317,7 +317,39 @@ def run_ours(args, w, rank, world, local_rank):
     barrier()
     e2e_ms = e_start.elapsed_time(e_end)
 
-    elapsed_ms, e2e_ms = multi.max_over_ranks([elapsed_ms, e2e_ms], device=dev)
+    # backward of the step (optional): gradients of sum(dout * out) from the forward's merged
+    # output and LSE, inputs resident; timed on its own after the forward line's region
+    bwd_ms, bwd_steps = 0.0, 0
+    if args.backward:
+        lse_m = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+        lsh.lsh_attention(qk, v, R, w.n_buckets, w.chunk, stream=stream, bufs=dict(bufs, lse=lse_m), **masks)
+        gen = torch.Generator(device=dev).manual_seed(multi.rank_seed(1, rank))
+        dout = torch.randn((w.B, w.H, w.L, w.D), generator=gen, device=dev).to(w.torch_dtype)
+        dqk = torch.empty((w.B, w.H, w.L, w.D), dtype=torch.float32, device=dev)
+        dvv = torch.empty_like(dqk)
+
+        def backward():
+            lsh.lsh_chunk_attend_backward(qk, v, bufs["perm"], w.chunk, bufs["out"], lse_m, dout,
+                                          buckets=bufs["buckets"], dqk=dqk, dv=dvv, stream=stream, **masks)
+
+        backward()
+        torch.cuda.synchronize()
+        bwd_steps = max(1, min(args.steps, 3))
+        b_start = torch.cuda.Event(enable_timing=True)
+        b_end = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        b_start.record(stream)
+        for _ in range(bwd_steps):
+            backward()
+        b_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        assert lsh.lsh_get_device_status(stream) == 0
+        bwd_ms = b_start.elapsed_time(b_end)
+        del dout, dqk, dvv
+
+    elapsed_ms, e2e_ms, bwd_ms = multi.max_over_ranks([elapsed_ms, e2e_ms, bwd_ms], device=dev)
 
     if rank != 0:
         return
@@ -375,6 +407,11 @@ def run_ours(args, w, rank, world, local_rank):
                          "sample": f"{sample_slices} (b,h) slice(s) of the workload ({c_tokens} tokens, all "
                                    f"{w.n_rounds} rounds), float64 NumPy oracle, {c_secs:.1f} s"},
     }
+    if args.backward:
+        line["backward"] = {
+            "ms": bwd_ms / bwd_steps, "value": world * w.tokens / (bwd_ms / bwd_steps / 1e3), "unit": UNIT,
+            "steps": bwd_steps, "gpu_launches": w.n_rounds * bwd_steps,
+            "note": "lsh_chunk_attend_backward alone (CUDA-core kernels, one launch per round), inputs resident"}
     print(json.dumps(line), flush=True)
 
 
@@ -388,7 +425,9 @@ def main():
     ap.add_argument("--causal", action="store_true",
                     help="causal window: keys after the query's position are masked")
     ap.add_argument("--bucket-mask", action="store_true",
-                    help="keys outside the query's bucket are masked (CUDA-core attention path)")
+                    help="keys outside the query's bucket are masked")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward call (gradients w.r.t. the shared rows and the values)")
     ap.add_argument("--union", action="store_true",
                     help="multi-round union correction (implies --bucket-mask; CUDA-core attention path)")
     args = ap.parse_args()

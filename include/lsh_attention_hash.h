@@ -235,6 +235,33 @@ LSH_API lsh_status lsh_combine_rounds(const void* out_rounds, int in_dtype, cons
                               int out_dtype, float* lse_out, void* stream);
 
 /*
+ * lsh_chunk_attend_backward -- gradients of sum(dout * out) with respect to the
+ * shared rows and the values, where out is lsh_combine_rounds' merge of
+ * lsh_chunk_attend's rounds.  (Training through LSH attention recomputes from
+ * the stored hash: twgreatdaily ICLR 2020 Reformer article, "1 LSH Attention";
+ * Ultralytics glossary "Reformer", "Atencao LSH".)  The hash, the sort and the
+ * masks are held fixed; per admissible pair (i, j) of every round, with
+ * p~ = exp(logit - LSE_i):
+ *     dv_j += p~ dout_i,  dz = p~ (dout_i . v_j - dout_i . out_i),
+ *     dqk_i += scale dz k_j,  and through k_j = qk_j / ||qk_j|| the key side.
+ *
+ *   qk, v, perm, buckets, chunk, mask, scale   as given to lsh_chunk_attend
+ *   out        [B, H, L, D] out_dtype   in: the merged output (lsh_combine_rounds)
+ *   lse        [B, H, L] float          in: its LSE (lse_out of lsh_combine_rounds)
+ *   dout       [B, H, L, D] out_dtype   in: gradient of the loss w.r.t. out
+ *   dqk, dv    [B, H, L, D] float       out: overwritten (zeroed, then accumulated
+ *                                       over the rounds in order; deterministic)
+ *
+ * Every mask runs (CUDA-core kernels, one launch per round).  A key row of zero
+ * length takes the clamp's linear branch (its gradient is scaled by 1e12).
+ * Requires what lsh_chunk_attend requires and B * H <= 65535.
+ */
+LSH_API lsh_status lsh_chunk_attend_backward(const void* qk, const void* v, int dtype, int B, int H, int L,
+                                     int D, int n_rounds, const int32_t* perm, const int32_t* buckets,
+                                     int chunk, int mask, float scale, const void* out, const float* lse,
+                                     const void* dout, int out_dtype, float* dqk, float* dv, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word (LSH_OK when no kernel recorded an error).  Returns LSH_ERR_CUDA if the
  * synchronisation itself fails.

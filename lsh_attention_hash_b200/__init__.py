@@ -1,4 +1,4 @@
-"""B200-native shared-QK LSH attention (Reformer), forward pass.
+"""B200-native shared-QK LSH attention (Reformer): forward pass and its backward.
 
 The compute path lives in ``liblsh_attention_hash.so`` (hand-written sm_100a
 CUDA kernels behind a C ABI declared in ``include/lsh_attention_hash.h``).  This
@@ -16,6 +16,7 @@ from .binding import (  # noqa: F401
     lsh_sort_workspace_bytes,
     lsh_chunk_attend,
     lsh_combine_rounds,
+    lsh_chunk_attend_backward,
     lsh_get_device_status,
     lsh_attention,
     library_path,

@@ -48,6 +48,8 @@ _SIGS = {
                                   _vp, _vp, _c_int, _c_int, _c_float, _vp, _c_int, _vp, _vp]),
     "lsh_combine_rounds": (_c_int, [_vp, _c_int, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp,
                                     _c_int, _vp, _vp]),
+    "lsh_chunk_attend_backward": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp,
+                                           _c_int, _c_int, _c_float, _vp, _vp, _vp, _c_int, _vp, _vp, _vp]),
     "lsh_get_device_status": (_c_int, [_vp]),
 }
 
@@ -252,6 +254,44 @@ def lsh_combine_rounds(out_rounds, lse, *, out_dtype=None, out=None, lse_out=Non
                                   _ptr(out), _DT[out_dtype], _ptr(lse_out), _stream(stream)),
            "lsh_combine_rounds")
     return out, lse_out
+
+
+def lsh_chunk_attend_backward(qk, v, perm, chunk, out, lse, dout, *, self_mask=True, causal=False, buckets=None,
+                              bucket_mask=False, union=False, scale=None, dqk=None, dv=None, stream=None):
+    """Gradients (dqk, dv) [B,H,L,D] float32 of sum(dout * out) for the merged output.
+
+    ``out`` and ``lse`` are the merged output and LSE of the forward (``lsh_combine_rounds``);
+    ``perm``, ``buckets``, the masks and ``scale`` must be the forward's.
+    """
+    lib = load_library()
+    _need(qk, "qk")
+    _need(v, "v", qk.dtype, qk.shape)
+    B, H, L, D = qk.shape
+    _need(perm, "perm", torch.int32)
+    n_rounds = perm.shape[2]
+    _need(perm, "perm", torch.int32, (B, H, n_rounds, L))
+    _need(out, "out", None, (B, H, L, D))
+    _need(dout, "dout", out.dtype, (B, H, L, D))
+    _need(lse, "lse", torch.float32, (B, H, L))
+    if union and not bucket_mask:
+        raise ValueError("union needs bucket_mask")
+    if bucket_mask:
+        if buckets is None:
+            raise ValueError("bucket_mask needs buckets")
+        _need(buckets, "buckets", torch.int32, (B, H, n_rounds, L))
+    if dqk is None:
+        dqk = torch.empty((B, H, L, D), dtype=torch.float32, device=qk.device)
+    if dv is None:
+        dv = torch.empty((B, H, L, D), dtype=torch.float32, device=qk.device)
+    _need(dqk, "dqk", torch.float32, (B, H, L, D))
+    _need(dv, "dv", torch.float32, (B, H, L, D))
+    mask = (1 if self_mask else 0) | (2 if causal else 0) | (4 if bucket_mask else 0) | (8 if union else 0)
+    sc = 0.0 if scale is None else float(scale)
+    _check(lib.lsh_chunk_attend_backward(_ptr(qk), _ptr(v), _dt(qk), B, H, L, D, n_rounds, _ptr(perm),
+                                         _ptr(buckets) if bucket_mask else None, int(chunk), mask, sc, _ptr(out),
+                                         _ptr(lse), _ptr(dout), _dt(out), _ptr(dqk), _ptr(dv), _stream(stream)),
+           "lsh_chunk_attend_backward")
+    return dqk, dv
 
 
 def lsh_get_device_status(stream=None) -> int:

@@ -8,6 +8,7 @@
 
 #include <cudaTypedefs.h>
 
+#include "attend_bwd_simt.cuh"
 #include "attend_simt.cuh"
 #include "attend_tc.cuh"
 #include "combine.cuh"
@@ -450,6 +451,60 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
     if (out_dtype == LSH_F32) LSH_ATT(__nv_bfloat16, float); else LSH_ATT(__nv_bfloat16, __nv_bfloat16);
   }
 #undef LSH_ATT
+  return launch_status();
+}
+
+lsh_status lsh_chunk_attend_backward(const void* qk, const void* v, int dtype, int B, int H, int L, int D,
+                                     int n_rounds, const int32_t* perm, const int32_t* buckets, int chunk,
+                                     int mask, float scale, const void* out, const float* lse,
+                                     const void* dout, int out_dtype, float* dqk, float* dv, void* stream) {
+  if (!valid_dtype(dtype) || !valid_dtype(out_dtype)) return LSH_ERR_DTYPE;
+  lsh_status st = check_bhld(B, H, L, D);
+  if (st != LSH_OK) return st;
+  if (n_rounds < 1 || !index_space_ok(B, H, L, n_rounds)) return LSH_ERR_SHAPE;
+  if (chunk < 1 || (L > 0 && (chunk > L || L % chunk != 0))) return LSH_ERR_SHAPE;
+  if (mask < 0 || mask > (LSH_MASK_SELF | LSH_MASK_CAUSAL | LSH_MASK_BUCKET | LSH_MASK_UNION))
+    return LSH_ERR_INVALID_ARG;
+  const int self_mask = (mask & LSH_MASK_SELF) ? 1 : 0;
+  const int causal = (mask & LSH_MASK_CAUSAL) ? 1 : 0;
+  const int bucket_mask = (mask & LSH_MASK_BUCKET) ? 1 : 0;
+  const int union_count = (mask & LSH_MASK_UNION) ? 1 : 0;
+  if (union_count && !bucket_mask) return LSH_ERR_INVALID_ARG;
+  if (bucket_mask && !buckets) return LSH_ERR_INVALID_ARG;
+  if (!qk || !v || !perm || !out || !lse || !dout || !dqk || !dv) return LSH_ERR_INVALID_ARG;
+  if (!aligned16(qk) || !aligned16(v) || !aligned16(perm) || !aligned16(out) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(dqk) || !aligned16(dv) || (buckets && !aligned16(buckets)))
+    return LSH_ERR_ALIGN;
+  const long long bhs = (long long)B * H;
+  if (bhs == 0 || L == 0) return LSH_OK;
+  if (bhs > 65535) return LSH_ERR_UNSUPPORTED;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)D);
+  const size_t smem = lsh::bwd_smem_words(D, n_rounds, union_count) * 4;
+  if (smem > (size_t)227 * 1024) return LSH_ERR_UNSUPPORTED;  // union with very many rounds
+  cudaStream_t s = as_stream(stream);
+  const size_t grad_bytes = (size_t)bhs * L * D * sizeof(float);
+  if (cudaMemsetAsync(dqk, 0, grad_bytes, s) != cudaSuccess || cudaMemsetAsync(dv, 0, grad_bytes, s) != cudaSuccess)
+    return LSH_ERR_CUDA;
+  const int blocks_per_chunk = (chunk + lsh::kBwdB - 1) / lsh::kBwdB;
+  dim3 grid((unsigned)((L / chunk) * blocks_per_chunk), (unsigned)bhs);
+  const int threads = lsh::kBwdWarps * 32;
+#define LSH_BWD(T, TO)                                                                                   \
+  do {                                                                                                    \
+    auto kfn = lsh::attend_bwd_simt_kernel<T, TO>;                                                        \
+    if (smem > 48 * 1024 &&                                                                               \
+        cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)  \
+      return LSH_ERR_CUDA;                                                                                \
+    for (int r = 0; r < n_rounds; ++r) /* rounds in order: every token has one writer per launch */      \
+      kfn<<<grid, threads, smem, s>>>((const T*)qk, (const T*)v, perm, buckets, (const TO*)out, lse,      \
+                                      (const TO*)dout, L, D, n_rounds, r, chunk, self_mask, causal,       \
+                                      bucket_mask, union_count, scale, dqk, dv);                          \
+  } while (0)
+  if (dtype == LSH_F32) {
+    if (out_dtype == LSH_F32) LSH_BWD(float, float); else LSH_BWD(float, __nv_bfloat16);
+  } else {
+    if (out_dtype == LSH_F32) LSH_BWD(__nv_bfloat16, float); else LSH_BWD(__nv_bfloat16, __nv_bfloat16);
+  }
+#undef LSH_BWD
   return launch_status();
 }
 

@@ -110,6 +110,34 @@ def test_attend_rejects_bad_arguments_before_launch(lib):
     assert call(L=0) == OK
 
 
+def test_backward_rejects_bad_arguments_before_launch(lib):
+    f = lib.lsh_chunk_attend_backward
+    args = [A, A, BF16, 1, 1, 1024, 64, 2, A, None, 64, 1, 0.0, A, A, A, BF16, A, A, None]
+    names = ["qk", "v", "dtype", "B", "H", "L", "D", "nr", "perm", "bk", "chunk", "mask", "scale", "out",
+             "lse", "dout", "out_dtype", "dqk", "dv", "stream"]
+
+    def call(**kw):
+        a = list(args)
+        for k, val in kw.items():
+            a[names.index(k)] = val
+        return f(*a)
+
+    assert call(dtype=3) == DTYPE
+    assert call(out_dtype=3) == DTYPE
+    assert call(chunk=48) == SHAPE
+    assert call(D=60) == SHAPE
+    assert call(nr=0) == SHAPE
+    assert call(mask=16) == INVALID
+    assert call(mask=1 | 4) == INVALID        # bucket mask without buckets
+    assert call(mask=1 | 8, bk=A) == INVALID  # union without the bucket mask
+    assert call(dout=None) == INVALID
+    assert call(dqk=None) == INVALID
+    assert call(lse=A + 4) == ALIGN
+    assert call(dv=A + 8) == ALIGN
+    assert call(B=0) == OK                    # empty: no launch
+    assert call(L=0) == OK
+
+
 def test_combine_rejects_bad_arguments_before_launch(lib):
     c = lib.lsh_combine_rounds
     assert c(A, 9, A, 1, 1, 64, 64, 2, A, BF16, None, None) == DTYPE

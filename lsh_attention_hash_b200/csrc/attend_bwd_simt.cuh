@@ -20,6 +20,8 @@
 // the owned tokens' rows of dqk and dv, which no other CTA of the launch
 // touches (perm is a permutation), so there are no atomics and the result is
 // deterministic.  Each pair's p~ and dz are computed by both CTAs involved.
+// The pair step reads 16-byte pieces of the staged rows (one key piece serves
+// four queries); the gradients of a warp's four rows stay in registers.
 #pragma once
 
 #include "common.cuh"
@@ -27,38 +29,40 @@
 namespace lsh {
 
 constexpr int kBwdB = 32;      // slots per block (queries or keys)
-constexpr int kBwdWarps = 8;   // 4 queries per warp in the pair step
+constexpr int kBwdWarps = 8;   // 4 queries (pair step, query role) or 4 keys (key role) per warp
+
+// Row stride of the staged rows: D + 4 words keeps every row 16-byte aligned and,
+// as D % 8 == 0, makes it an odd multiple of 4 words, so eight lanes reading
+// float4s of eight different rows hit 32 different banks.
+__host__ __device__ inline int bwd_row_stride(int D) { return D + 4; }
 
 // Shared memory of attend_bwd_simt_kernel, in 4-byte words.
 __host__ __device__ inline size_t bwd_smem_words(int D, int n_rounds, int union_count) {
-  const size_t DP = (size_t)D + 1;
-  return 4 * kBwdB * DP                       // qs, gs, ks, vs
-         + 3 * kBwdB * (kBwdB + 1)            // p~, dz, x_i . k_j
-         + 2 * (size_t)kBwdB * D              // two accumulators
-         + 6 * kBwdB                          // lse, delta, kinv, kproj, ck, pad
-         + 7 * kBwdB                          // q_pos, q_slot, q_bk, q_alone, k_pos, k_slot, k_bk
+  return 4 * (size_t)kBwdB * bwd_row_stride(D)  // qs, gs, ks, vs
+         + 3 * kBwdB * (kBwdB + 1)              // p~, dz, x_i . k_j
+         + 6 * kBwdB                            // lse, delta, kinv, kproj, ck, pad
+         + 7 * kBwdB                            // q_pos, q_slot, q_bk, q_alone, k_pos, k_slot, k_bk
          + (union_count ? 2 * (size_t)n_rounds * kBwdB : 0);
 }
 
-template <typename T, typename TO>
-__global__ void __launch_bounds__(kBwdWarps * 32)
+// MDL: columns per lane (D <= 32 * MDL); 4 (D <= 128) leaves room for two CTAs per SM.
+template <typename T, typename TO, int MDL>
+__global__ void __launch_bounds__(kBwdWarps * 32, MDL <= 4 ? 2 : 1)
 attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const int32_t* __restrict__ perm,
                        const int32_t* __restrict__ buckets, const TO* __restrict__ out,
                        const float* __restrict__ lse, const TO* __restrict__ dout, int L, int D, int n_rounds,
                        int round, int chunk, int self_mask, int causal, int bucket_mask, int union_count,
                        float scale, float* __restrict__ dqk, float* __restrict__ dv) {
-  extern __shared__ float sm[];
-  const int DP = D + 1;
-  float* qs = sm;                          // [32][DP] query rows x_i
-  float* gs = qs + kBwdB * DP;             // [32][DP] their dout rows
-  float* ks = gs + kBwdB * DP;             // [32][DP] key rows x_j
-  float* vs = ks + kBwdB * DP;             // [32][DP] their values
-  float* pm = vs + kBwdB * DP;             // [32][33] p~
+  extern __shared__ __align__(16) float bwd_sm[];
+  const int DS = bwd_row_stride(D);
+  float* qs = bwd_sm;                        // [32][DS] query rows x_i
+  float* gs = qs + kBwdB * DS;             // [32][DS] their dout rows
+  float* ks = gs + kBwdB * DS;             // [32][DS] key rows x_j
+  float* vs = ks + kBwdB * DS;             // [32][DS] their values
+  float* pm = vs + kBwdB * DS;             // [32][33] p~
   float* dz = pm + kBwdB * (kBwdB + 1);    // [32][33] dz
   float* zq = dz + kBwdB * (kBwdB + 1);    // [32][33] x_i . k_j
-  float* acc1 = zq + kBwdB * (kBwdB + 1);  // [32][D] query role: dx; key role: dk
-  float* acc2 = acc1 + kBwdB * D;          // [32][D] key role: dv
-  float* q_lse = acc2 + kBwdB * D;         // [32]
+  float* q_lse = zq + kBwdB * (kBwdB + 1); // [32]
   float* q_delta = q_lse + kBwdB;          // [32] dout_i . out_i
   float* kinv = q_delta + kBwdB;           // [32] 1 / max(||x_j||, 1e-12)
   float* kproj = kinv + kBwdB;             // [32] 1 when ||x_j|| >= 1e-12 (projection term), else 0
@@ -91,6 +95,7 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
   float* dqk_bh = dqk + bh * (long long)L * D;
   float* dv_bh = dv + bh * (long long)L * D;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r0 = warp * 4;                 // this warp's 4 rows (queries or keys) of a block
   constexpr int kThreads = kBwdWarps * 32;
 
   // Whether the query at sorted slot s has no admissible key but itself (the
@@ -135,8 +140,8 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
         x = to_f32(qk_bh[row + d]);
         g = to_f32(dout_bh[row + d]);
       }
-      qs[j * DP + d] = x;
-      gs[j * DP + d] = g;
+      qs[j * DS + d] = x;
+      gs[j * DS + d] = g;
     }
     for (int i = warp; i < kBwdB; i += kBwdWarps) {  // delta_i = dout_i . out_i
       float acc = 0.f;
@@ -150,7 +155,7 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
     }
   };
 
-  // Key block: slots [a, a + n).
+  // Key block: slots [a, a + n); ends with a barrier and the key lengths.
   auto load_keys = [&](int a, int n) {
     for (int i = tid; i < kBwdB; i += kThreads) {
       const int pos = i < n ? pseg[a + i] : 0;
@@ -171,13 +176,13 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
         x = to_f32(qk_bh[row + d]);
         y = to_f32(v_bh[row + d]);
       }
-      ks[j * DP + d] = x;
-      vs[j * DP + d] = y;
+      ks[j * DS + d] = x;
+      vs[j * DS + d] = y;
     }
     __syncthreads();
     for (int j = warp; j < kBwdB; j += kBwdWarps) {
       float ss = 0.f;
-      for (int d = lane; d < D; d += 32) ss = fmaf(ks[j * DP + d], ks[j * DP + d], ss);
+      for (int d = lane; d < D; d += 32) ss = fmaf(ks[j * DS + d], ks[j * DS + d], ss);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
       if (lane == 0) {
@@ -188,21 +193,31 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
     }
   };
 
-  // p~, dz and x_i . k_j of the loaded query block (nq rows) against the key block (nk).
+  // p~, dz and x_i . k_j of the loaded query block (nq rows) against the key
+  // block (nk): the warp takes queries r0..r0+3, lane j takes key j; each
+  // 16-byte load of a key (and its value) row serves four queries.
   auto pairs = [&](int nq, int nk) {
-    constexpr int QW = kBwdB / kBwdWarps;
-#pragma unroll 1
-    for (int a = 0; a < QW; ++a) {
-      const int i = warp * QW + a;
-      const int j = lane;
+    const int j = lane;
+    float dot[4] = {0.f, 0.f, 0.f, 0.f}, dpv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (j < nk) {
+      for (int d = 0; d < D; d += 4) {
+        const float4 kk = *reinterpret_cast<const float4*>(ks + j * DS + d);
+        const float4 vv = *reinterpret_cast<const float4*>(vs + j * DS + d);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const float4 q = *reinterpret_cast<const float4*>(qs + (r0 + a) * DS + d);
+          const float4 g = *reinterpret_cast<const float4*>(gs + (r0 + a) * DS + d);
+          dot[a] = fmaf(q.x, kk.x, fmaf(q.y, kk.y, fmaf(q.z, kk.z, fmaf(q.w, kk.w, dot[a]))));
+          dpv[a] = fmaf(g.x, vv.x, fmaf(g.y, vv.y, fmaf(g.z, vv.z, fmaf(g.w, vv.w, dpv[a]))));
+        }
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int i = r0 + a;
       float p = 0.f, g = 0.f, x = 0.f;
       if (i < nq && j < nk) {
-        float dot = 0.f, dpv = 0.f;
-        for (int d = 0; d < D; ++d) {
-          dot = fmaf(qs[i * DP + d], ks[j * DP + d], dot);
-          dpv = fmaf(gs[i * DP + d], vs[j * DP + d], dpv);
-        }
-        x = dot * kinv[j];
+        x = dot[a] * kinv[j];
         const bool masked = (causal && k_pos[j] > q_pos[i]) || (bucket_mask && k_bk[j] != q_bk[i]) ||
                             (self_mask && k_slot[j] == q_slot[i] && !q_alone[i]);
         if (!masked) {
@@ -213,7 +228,7 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
             z -= logf((float)n_shared);
           }
           p = expf(z - q_lse[i]);
-          g = p * (dpv - q_delta[i]);
+          g = p * (dpv[a] - q_delta[i]);
         }
       }
       pm[i * (kBwdB + 1) + j] = p;
@@ -223,11 +238,18 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
   };
 
   const int n_own = s1 - s0;
+  const int DL = (D + 31) / 32;
 
   // ---------------------------------------------------------- query role
-  load_queries(s0, n_own);
-  for (int i = tid; i < kBwdB * D; i += kThreads) acc1[i] = 0.f;
+  // dx_i = scale sum_j dz_ij x_j / ||x_j||, kept in registers: warp rows r0..r0+3,
+  // lane columns lane + 32 e
   {
+    float aq[4][MDL];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int e = 0; e < MDL; ++e) aq[a][e] = 0.f;
+    load_queries(s0, n_own);
     const int w0 = max(k - 1, 0) * chunk, w1 = (k + 1) * chunk;
     for (int kb = w0; kb < w1; kb += kBwdB) {
       __syncthreads();  // previous block's readers done
@@ -236,29 +258,49 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
       __syncthreads();
       pairs(n_own, nk);
       __syncthreads();
-      for (int e = tid; e < kBwdB * D; e += kThreads) {  // dx_i += scale sum_j dz_ij x_j / ||x_j||
-        const int i = e / D, d = e - i * D;
-        float a = 0.f;
-        for (int j = 0; j < nk; ++j) a = fmaf(dz[i * (kBwdB + 1) + j], ks[j * DP + d] * kinv[j], a);
-        acc1[e] = fmaf(scale, a, acc1[e]);
+      for (int j = 0; j < nk; ++j) {
+        const float kj = scale * kinv[j];
+        float w[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) w[a] = dz[(r0 + a) * (kBwdB + 1) + j] * kj;
+#pragma unroll
+        for (int e = 0; e < MDL; ++e) {
+          const int d = lane + 32 * e;
+          if (e < DL && d < D) {
+            const float kd = ks[j * DS + d];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) aq[a][e] = fmaf(w[a], kd, aq[a][e]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      if (r0 + a >= n_own) continue;
+      float* dst = dqk_bh + (long long)q_pos[r0 + a] * D;
+#pragma unroll
+      for (int e = 0; e < MDL; ++e) {
+        const int d = lane + 32 * e;
+        if (e < DL && d < D) dst[d] += aq[a][e];
       }
     }
   }
-  __syncthreads();
-  for (int e = tid; e < n_own * D; e += kThreads) {
-    const int i = e / D, d = e - i * D;
-    dqk_bh[(long long)q_pos[i] * D + d] += acc1[e];
-  }
-  __syncthreads();
+  __syncthreads();  // the query role's adds land before the key role adds to the same rows
 
   // ---------------------------------------------------------- key role
-  load_keys(s0, n_own);  // ends with the key lengths; a barrier follows below
-  for (int i = tid; i < kBwdB * D; i += kThreads) {
-    acc1[i] = 0.f;
-    acc2[i] = 0.f;
-  }
-  for (int i = tid; i < kBwdB; i += kThreads) ck[i] = 0.f;
+  // dk_j = scale sum_i dz_ij x_i and dv_j = sum_i p~_ij dout_i in registers: warp keys
+  // r0..r0+3, lane columns lane + 32 e
   {
+    float ak[4][MDL], av[4][MDL];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int e = 0; e < MDL; ++e) {
+        ak[a][e] = 0.f;
+        av[a][e] = 0.f;
+      }
+    load_keys(s0, n_own);
+    for (int i = tid; i < kBwdB; i += kThreads) ck[i] = 0.f;
     const int q0 = k * chunk, q1 = min(k + 2, n_chunks) * chunk;  // queries of chunks k and k+1
     for (int qb = q0; qb < q1; qb += kBwdB) {
       __syncthreads();
@@ -268,30 +310,48 @@ attend_bwd_simt_kernel(const T* __restrict__ qk, const T* __restrict__ v, const 
       pairs(nq, n_own);
       __syncthreads();
       for (int j = warp; j < kBwdB; j += kBwdWarps) {  // dk_j . k_j += scale sum_i dz_ij (x_i . k_j)
-        float a = lane < nq ? dz[lane * (kBwdB + 1) + j] * zq[lane * (kBwdB + 1) + j] : 0.f;
+        float c = lane < nq ? dz[lane * (kBwdB + 1) + j] * zq[lane * (kBwdB + 1) + j] : 0.f;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-        if (lane == 0) ck[j] = fmaf(scale, a, ck[j]);
+        for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+        if (lane == 0) ck[j] = fmaf(scale, c, ck[j]);
       }
-      for (int e = tid; e < kBwdB * D; e += kThreads) {
-        const int j = e / D, d = e - j * D;
-        float a = 0.f, b = 0.f;
-        for (int i = 0; i < nq; ++i) {
-          a = fmaf(dz[i * (kBwdB + 1) + j], qs[i * DP + d], a);
-          b = fmaf(pm[i * (kBwdB + 1) + j], gs[i * DP + d], b);
+      for (int i = 0; i < nq; ++i) {
+        float wz[4], wp[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          wz[a] = dz[i * (kBwdB + 1) + r0 + a];
+          wp[a] = pm[i * (kBwdB + 1) + r0 + a];
         }
-        acc1[e] = fmaf(scale, a, acc1[e]);
-        acc2[e] += b;
+#pragma unroll
+        for (int e = 0; e < MDL; ++e) {
+          const int d = lane + 32 * e;
+          if (e < DL && d < D) {
+            const float xd = qs[i * DS + d], gd = gs[i * DS + d];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              ak[a][e] = fmaf(wz[a], xd, ak[a][e]);
+              av[a][e] = fmaf(wp[a], gd, av[a][e]);
+            }
+          }
+        }
       }
     }
-  }
-  __syncthreads();
-  for (int e = tid; e < n_own * D; e += kThreads) {
-    const int j = e / D, d = e - j * D;
-    const float khat = ks[j * DP + d] * kinv[j];
-    const long long o = (long long)k_pos[j] * D + d;
-    dqk_bh[o] += (acc1[e] - kproj[j] * ck[j] * khat) * kinv[j];
-    dv_bh[o] += acc2[e];
+    __syncthreads();  // ck complete
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int j = r0 + a;
+      if (j >= n_own) continue;
+      const long long row = (long long)k_pos[j] * D;
+#pragma unroll
+      for (int e = 0; e < MDL; ++e) {
+        const int d = lane + 32 * e;
+        if (e < DL && d < D) {
+          const float khat = ks[j * DS + d] * kinv[j];
+          dqk_bh[row + d] += (scale * ak[a][e] - kproj[j] * ck[j] * khat) * kinv[j];
+          dv_bh[row + d] += av[a][e];
+        }
+      }
+    }
   }
 }
 

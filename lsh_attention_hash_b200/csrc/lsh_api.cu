@@ -490,7 +490,7 @@ lsh_status lsh_chunk_attend_backward(const void* qk, const void* v, int dtype, i
   const int threads = lsh::kBwdWarps * 32;
 #define LSH_BWD(T, TO)                                                                                   \
   do {                                                                                                    \
-    auto kfn = lsh::attend_bwd_simt_kernel<T, TO>;                                                        \
+    auto kfn = D <= 128 ? lsh::attend_bwd_simt_kernel<T, TO, 4> : lsh::attend_bwd_simt_kernel<T, TO, 8>;  \
     if (smem > 48 * 1024 &&                                                                               \
         cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)  \
       return LSH_ERR_CUDA;                                                                                \

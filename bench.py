@@ -69,6 +69,29 @@ def algorithmic(w):
     }
 
 
+def backward_flops(w):
+    """Algorithmic FLOPs of one backward over the workload: per admissible-window pair
+    (query, key) of a round, five length-D dot products or rank-1 updates (the logit, dout . v,
+    and the dq, dk, dv contributions), 2 D flops each.  A query of chunk 0 sees c keys, every
+    other query 2 c, so a (b, h, round) segment has L 2c - c^2 pairs."""
+    pairs = w.B * w.H * w.n_rounds * (w.L * 2 * w.chunk - w.chunk * w.chunk)
+    return 10.0 * w.D * pairs
+
+
+def measured_sm_max_mhz(default=1965.0):
+    """Maximum SM clock recorded with the measured peaks (the nominal 1965 MHz otherwise)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(path):
+        return default
+    with open(path) as f:
+        return float(json.load(f).get("sm_max_mhz", default))
+
+
+def alu_peak_tflops(sms, sm_mhz):
+    """FP32 FMA peak of the CUDA cores: 128 FP32 lanes per SM, 2 flops per FMA."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def kernel_bound(stage):
     return "tensor" if stage == "hash" else "hbm"
 
@@ -408,9 +431,16 @@ def run_ours(args, w, rank, world, local_rank):
                                    f"{w.n_rounds} rounds), float64 NumPy oracle, {c_secs:.1f} s"},
     }
     if args.backward:
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        sm_mhz = measured_sm_max_mhz()
+        b_ach = backward_flops(w) / (bwd_ms / bwd_steps / 1e3) / 1e12
+        b_peak = alu_peak_tflops(sms, sm_mhz)
         line["backward"] = {
             "ms": bwd_ms / bwd_steps, "value": world * w.tokens / (bwd_ms / bwd_steps / 1e3), "unit": UNIT,
             "steps": bwd_steps, "gpu_launches": w.n_rounds * bwd_steps,
+            "roofline": {"bound": "alu", "achieved": b_ach, "peak": b_peak, "unit": "TFLOP/s",
+                         "frac": b_ach / b_peak, "traffic": None,
+                         "peak_source": f"FP32 FMA on the CUDA cores: {sms} SMs x 128 lanes x 2 x {sm_mhz:.0f} MHz"},
             "note": "lsh_chunk_attend_backward alone (CUDA-core kernels, one launch per round), inputs resident"}
     print(json.dumps(line), flush=True)
 

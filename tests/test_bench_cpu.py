@@ -76,3 +76,11 @@ def test_peaks_come_from_the_measured_file_when_present():
         assert src.startswith("measured")
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             assert peaks["hbm_gbs"] == float(json.load(f)["hbm_gbs"])
+
+
+def test_backward_flop_count_and_alu_peak():
+    w = synth.small_workload("bwd_count", 1, 1, 256, 64, "f32", 8, 64, 2)
+    # chunk 0: 64 queries x 64 keys; chunks 1..3: 64 queries x 128 keys; per round
+    pairs = 2 * (64 * 64 + 3 * 64 * 128)
+    assert bench.backward_flops(w) == 10 * 64 * pairs
+    assert abs(bench.alu_peak_tflops(148, 1965.0) - 74.45) < 0.01

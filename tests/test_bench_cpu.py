@@ -84,3 +84,15 @@ def test_backward_flop_count_and_alu_peak():
     pairs = 2 * (64 * 64 + 3 * 64 * 128)
     assert bench.backward_flops(w) == 10 * 64 * pairs
     assert abs(bench.alu_peak_tflops(148, 1965.0) - 74.45) < 0.01
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Launched as two ranks (as the driver launches N > 1), rank 0 alone prints the line."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr=127.0.0.1", "--master-port=29533", os.path.join(ROOT, "bench.py"), "--impl",
+           "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3", "--gpus", "2"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300, check=True).stdout
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2

@@ -16,7 +16,7 @@ HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROO
            if f.endswith(".h")]
 
 # codes from include/lsh_attention_hash.h
-OK, INVALID, SHAPE, DTYPE, ALIGN, WORKSPACE = 0, 1, 2, 3, 4, 5
+OK, INVALID, SHAPE, DTYPE, ALIGN, WORKSPACE, UNSUPPORTED = 0, 1, 2, 3, 4, 5, 8
 F32, BF16 = 0, 1
 A = 0x10000  # a 16-byte aligned non-null address that is never dereferenced (rejected before launch)
 
@@ -103,6 +103,8 @@ def test_attend_rejects_bad_arguments_before_launch(lib):
     assert call(mask=1 | 8, bk=A) == INVALID  # union without the bucket mask
     assert call(mask=1 | 4, bk=A + 4) == ALIGN
     assert call(mask=1 | 4 | 8, bk=A, L=0) == OK
+    # the union's per-round bucket tables no longer fit in shared memory
+    assert call(mask=1 | 4 | 8, bk=A, dtype=F32, out_dtype=F32, D=256, nr=600, chunk=32) == UNSUPPORTED
     assert call(out_dtype=5) == DTYPE
     assert call(qs=A) == INVALID          # sorted qk without sorted v
     assert call(lse=None) == INVALID
@@ -134,6 +136,7 @@ def test_backward_rejects_bad_arguments_before_launch(lib):
     assert call(dqk=None) == INVALID
     assert call(lse=A + 4) == ALIGN
     assert call(dv=A + 8) == ALIGN
+    assert call(mask=1 | 4 | 8, bk=A, D=256, nr=400) == UNSUPPORTED  # union tables beyond shared memory
     assert call(B=0) == OK                    # empty: no launch
     assert call(L=0) == OK
 

@@ -42,6 +42,38 @@ def test_library_exports_every_declared_symbol(lib):
     assert lib.lsh_abi_version() == 2
 
 
+def _declared_param_counts():
+    """Number of parameters of every LSH_API declaration (void counts as none)."""
+    out = {}
+    for h in HEADERS:
+        src = open(h).read()
+        for name, params in re.findall(r"LSH_API\s+[\w\s\*]+?\b(lsh_\w+)\s*\(([^)]*)\)", src):
+            params = params.strip()
+            out[name] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """The ctypes argument lists have as many entries as the C declarations have parameters, and
+    every declared entry point has a binding signature."""
+    from lsh_attention_hash_b200 import binding
+
+    counts = _declared_param_counts()
+    assert set(counts) == set(declared_symbols())
+    for name, n in counts.items():
+        assert name in binding._SIGS, name
+        assert len(binding._SIGS[name][1]) == n, (name, len(binding._SIGS[name][1]), n)
+
+
+def test_library_exports_nothing_undeclared(lib):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", lsh.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.split() and line.split()[-1].startswith("lsh_")}
+    assert exported == set(declared_symbols()), exported ^ set(declared_symbols())
+
+
 def test_status_strings(lib):
     assert lib.lsh_status_string(0) == b"LSH_OK"
     assert lib.lsh_status_string(7) == b"LSH_ERR_TIMEOUT"

@@ -192,11 +192,14 @@ def mask_config(args):
     return {"mask": "+".join(names)} if names else {}
 
 
-def oracle_sample(w, slices=1, seed=0, masks=None):
+def oracle_sample(w, slices=1, seed=0, masks=None, threads=None):
     """Runs the float64 oracle on `slices` (b, h) slices of the workload, all rounds.
 
+    `threads` caps the BLAS thread pools (None: as many as the library starts).
     Returns (seconds, tokens, threads).
     """
+    import contextlib
+
     import numpy as np
     import threadpoolctl
 
@@ -205,18 +208,20 @@ def oracle_sample(w, slices=1, seed=0, masks=None):
 
     R = synth.projections(w, seed)
     tokens, secs = 0, 0.0
-    for n in range(slices):
-        b, h = divmod(n % (w.B * w.H), w.H)
-        qk_s, v_s = synth.slice_inputs(w, b, h, seed)
-        qk = qk_s[None, None]
-        v = v_s[None, None]
-        t0 = time.perf_counter()
-        oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, **(masks or {}))
-        secs += time.perf_counter() - t0
-        tokens += w.L
-    info = threadpoolctl.threadpool_info()
-    threads = max([i.get("num_threads", 1) for i in info] + [1])
-    return secs, tokens, threads
+    limit = threadpoolctl.threadpool_limits(threads) if threads else contextlib.nullcontext()
+    with limit:
+        for n in range(slices):
+            b, h = divmod(n % (w.B * w.H), w.H)
+            qk_s, v_s = synth.slice_inputs(w, b, h, seed)
+            qk = qk_s[None, None]
+            v = v_s[None, None]
+            t0 = time.perf_counter()
+            oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, **(masks or {}))
+            secs += time.perf_counter() - t0
+            tokens += w.L
+        info = threadpoolctl.threadpool_info()
+        used = max([i.get("num_threads", 1) for i in info] + [1])
+    return secs, tokens, used
 
 
 def run_reference(args, w, rank, world):
@@ -272,25 +277,26 @@ def run_ours(args, w, rank, world, local_rank):
     R = R_h.to(dev)
     bufs = binding.alloc_buffers(w.B, w.H, w.L, w.D, w.n_rounds, w.n_buckets, w.torch_dtype, dev)
     stream = torch.cuda.current_stream(dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    # stage boundaries of every timed step (read after the timed region: no host sync inside it)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
 
-    def step(record):
-        if record:
+    def step(ev):
+        if ev:
             ev[0].record(stream)
         lsh.lsh_hash(qk, R, w.n_buckets, buckets=bufs["buckets"], with_near_tie=False, stream=stream)
-        if record:
+        if ev:
             ev[1].record(stream)
         lsh.lsh_sort_permute(bufs["buckets"], w.n_buckets, perm=bufs["perm"], workspace=bufs["workspace"],
                              stream=stream)
-        if record:
+        if ev:
             ev[2].record(stream)
         lsh.lsh_chunk_attend(qk, v, bufs["perm"], w.chunk, out_rounds=bufs["out_rounds"],
                              lse=bufs["lse_rounds"], buckets=bufs["buckets"], stream=stream, **masks)
-        if record:
+        if ev:
             ev[3].record(stream)
         lsh.lsh_combine_rounds(bufs["out_rounds"], bufs["lse_rounds"], out=bufs["out"], want_lse=False,
                                stream=stream)
-        if record:
+        if ev:
             ev[4].record(stream)
 
     def barrier():
@@ -298,7 +304,7 @@ def run_ours(args, w, rank, world, local_rank):
             dist.barrier(device_ids=[local_rank])
 
     for _ in range(args.warmup):
-        step(False)
+        step(None)
     torch.cuda.synchronize()
     assert lsh.lsh_get_device_status(stream) == 0
 
@@ -309,15 +315,15 @@ def run_ours(args, w, rank, world, local_rank):
         barrier()
         torch.cuda.synchronize()
         t_start.record(stream)
-        for _ in range(args.steps):
-            step(True)
-            ev[4].synchronize()
-            for i, s in enumerate(STAGES):
-                stage_ms[s] += ev[i].elapsed_time(ev[i + 1])
+        for k in range(args.steps):
+            step(evs[k])
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
+    for ev in evs:
+        for i, s in enumerate(STAGES):
+            stage_ms[s] += ev[i].elapsed_time(ev[i + 1])
     assert lsh.lsh_get_device_status(stream) == 0
 
     # end to end through the public API with host buffers: H2D of the step's
@@ -407,6 +413,7 @@ def run_ours(args, w, rank, world, local_rank):
     launches_per_step = 3 + sort_launches                  # hash, sort, attend, combine
     sample_slices = 2  # about 10 s of float64 CPU work at the 64K workload
     c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices, masks=masks)
+    o_secs, o_tokens, _ = oracle_sample(w, 1, masks=masks, threads=1)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -427,8 +434,12 @@ def run_ours(args, w, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": {"value": c_tokens / c_secs, "unit": UNIT, "cores": c_threads, "kind": "oracle",
+                         "affinity_cores": len(os.sched_getaffinity(0)),
                          "sample": f"{sample_slices} (b,h) slice(s) of the workload ({c_tokens} tokens, all "
-                                   f"{w.n_rounds} rounds), float64 NumPy oracle, {c_secs:.1f} s"},
+                                   f"{w.n_rounds} rounds), float64 NumPy oracle, {c_secs:.1f} s",
+                         "one_core": {"value": o_tokens / o_secs, "unit": UNIT, "cores": 1,
+                                      "sample": f"1 (b,h) slice ({o_tokens} tokens, all {w.n_rounds} rounds), "
+                                                f"BLAS pools capped at one thread, {o_secs:.1f} s"}},
     }
     if args.backward:
         sms = torch.cuda.get_device_properties(dev).multi_processor_count

@@ -153,17 +153,21 @@ LSH_API lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L,
  *
  *   buckets, perm, inv: as for lsh_sort_permute (inv nullable).
  *
- * This call always runs the count-scan-scatter sort, whose counters take
- * B*H*n_rounds * n_buckets * ceil(L / max(4096, n_buckets)) uint32 words; it
- * returns LSH_ERR_WORKSPACE, before any launch, when that exceeds the array's
- * 4 Mi words (16 MiB).  All other argument rules and errors are those of
- * lsh_sort_permute.
+ * Shapes with L <= 65536 and n_buckets <= 1024 (the 64K workload among them)
+ * are sorted by one CTA per segment entirely in shared memory and touch the
+ * array not at all.  Larger shapes run the count-scan-scatter sort, whose
+ * counters take B*H*n_rounds * n_buckets * ceil(L / max(4096, n_buckets))
+ * uint32 words of the array; the call returns LSH_ERR_WORKSPACE, before any
+ * launch, when that exceeds the array's 4 Mi words (16 MiB).  All other
+ * argument rules and errors are those of lsh_sort_permute.
  *
- * The first call on a device looks up the array's device address (with that
- * device current), so make that first call before any stream capture.  Every
+ * The first call on a device that needs the array looks up its device
+ * address (with that device current) and keeps it for the life of the
+ * process, so make that first call before any stream capture, and do not use
+ * this call after cudaDeviceReset (the kept address would be stale).  Every
  * call on a device shares the one array and leaves its contents behind; the
- * call clears what must start at zero itself.  Calls whose work overlaps on the
- * GPU (different streams, or graphs running at the same time) race on the
+ * call clears what must start at zero itself.  Calls whose work overlaps on
+ * the GPU (different streams, or graphs running at the same time) race on the
  * array: order them, for example on one stream.
  */
 LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H, int L,

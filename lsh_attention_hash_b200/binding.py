@@ -10,7 +10,6 @@ happens in the library's CUDA kernels; there is no CPU fallback.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 import torch
@@ -300,11 +299,17 @@ def lsh_get_device_status(stream=None) -> int:
 
 
 def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, causal=False, bucket_mask=False, union=False,
-                  scale=None, stream=None, return_all=False, bufs=None):
+                  scale=None, stream=None, return_all=False, bufs=None, check=False):
     """The whole forward pass: hash, sort, chunk attention, round merge (four C-ABI calls).
 
     ``bufs`` may hold preallocated outputs (keys: buckets, near_tie, perm, workspace,
     out_rounds, lse_rounds, out, lse) so that repeated calls allocate nothing.
+
+    The calls are asynchronous.  Errors that the kernels detect while they run (an
+    exhausted bounded wait, a bucket id out of range) are recorded in the device
+    status word, not returned: with ``check=True`` the stream is synchronised and a
+    non-zero status raises ``LSHError``; otherwise the caller reads it with
+    ``lsh_get_device_status`` before trusting the outputs.
     """
     b = bufs or {}
     buckets, near = lsh_hash(qk, R, n_buckets, buckets=b.get("buckets"), near_tie=b.get("near_tie"),
@@ -316,6 +321,8 @@ def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, causal=False, b
                               out_rounds=b.get("out_rounds"), lse=b.get("lse_rounds"), stream=stream)
     out, lse_out = lsh_combine_rounds(o, lse, out=b.get("out"), lse_out=b.get("lse"),
                                       want_lse=return_all or "lse" in b, stream=stream)
+    if check:
+        _check(lsh_get_device_status(stream), "lsh_attention (device status)")
     if return_all:
         return {"buckets": buckets, "near_tie": near, "perm": perm, "o_rounds": o, "lse_rounds": lse,
                 "out": out, "lse": lse_out}
@@ -337,6 +344,3 @@ def alloc_buffers(B, H, L, D, n_rounds, n_buckets, dtype, device, with_near_tie=
         bufs["near_tie"] = torch.empty((B, H, n_rounds, L), dtype=torch.uint8, device=device)
     return bufs
 
-
-def default_scale(D):
-    return 1.0 / math.sqrt(D)

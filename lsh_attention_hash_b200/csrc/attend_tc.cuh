@@ -330,77 +330,87 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
   return colscale / fmaxf(sqrtf(ss), 1e-12f);
 }
 
-// One pass of the softmax over a row's 128 keys (four groups of 32 S columns,
-// the next group's TMEM load in flight while the current one is processed):
-// w = 2^(S * colmul - m) in fp32 (self masked, a missing previous chunk dead,
-// with CAUSAL a key after the query's original position masked, with BUCKET a
-// key outside the query's bucket masked), l += w, and
-// the weights go to P as bf16 pairs right away: P's group g lands on S columns
-// whose values this row has already consumed.  With MASK bits, `others`
-// counts the admissible keys (CAUSAL: the earlier ones; BUCKET alone: those of
-// the query's bucket, self included) and `self_w` keeps the P words of the
-// self group (for the self-only fix-up).
+template <int D, int MASK>
+__device__ __forceinline__ void softmax_group(uint32_t sbuf, uint32_t pcol, int g, const uint32_t (&cur)[32],
+                                              const float* cm, const int32_t* kp, const int32_t* kb, bool dead,
+                                              bool self_grp, int lane, float m, float& l, int qpos, int qb,
+                                              int& others) {
+  constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
+  // key multipliers (and positions, buckets) as 16-byte loads: each group's 32 values start on a
+  // 16-byte boundary
+  const float4* cm4 = reinterpret_cast<const float4*>(cm);
+  const int4* kp4 = reinterpret_cast<const int4*>(kp);
+  const int4* kb4 = reinterpret_cast<const int4*>(kb);
+  uint32_t w16[16];
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float4 c4 = cm4[e >> 2];
+    // shifted logits in the log2 domain, S * colmul - m as one FMA
+    float v0 = fmaf(__uint_as_float(cur[e]), (e & 2) ? c4.z : c4.x, -m);
+    float v1 = fmaf(__uint_as_float(cur[e + 1]), (e & 2) ? c4.w : c4.y, -m);
+    if (CAUSAL || BUCKET) {  // keys are distinct tokens: position == qpos only for self
+      bool c0 = true, c1 = true;  // counted: admissible and (CAUSAL) not self
+      if (CAUSAL) {
+        const int4 k4 = kp4[e >> 2];
+        const int p0 = (e & 2) ? k4.z : k4.x, p1 = (e & 2) ? k4.w : k4.y;
+        if (p0 > qpos) v0 = -INFINITY;
+        if (p1 > qpos) v1 = -INFINITY;
+        c0 = p0 < qpos;
+        c1 = p1 < qpos;
+      }
+      if (BUCKET) {
+        const int4 b4 = kb4[e >> 2];
+        const int b0 = (e & 2) ? b4.z : b4.x, b1 = (e & 2) ? b4.w : b4.y;
+        if (b0 != qb) v0 = -INFINITY;
+        if (b1 != qb) v1 = -INFINITY;
+        c0 = c0 && b0 == qb;
+        c1 = c1 && b1 == qb;
+      }
+      if (!dead) others += (int)c0 + (int)c1;
+    }
+    if (self_grp) {
+      if (e == lane) v0 = -INFINITY;
+      if (e + 1 == lane) v1 = -INFINITY;
+    }
+    const float a = dead ? 0.f : tc::ex2_approx(v0);
+    const float c = dead ? 0.f : tc::ex2_approx(v1);
+    l += a + c;
+    w16[e >> 1] = tc::pack_bf16x2(a, c);
+  }
+  tc::tmem_st16(sbuf + pcol + 16 * g, w16);
+}
+
+// One pass of the softmax over a row's 128 keys, four groups of 32 S columns
+// (the next group's TMEM load in flight while the current one is processed): w = 2^(S * colmul - m) in fp32 (self masked, a missing previous chunk
+// dead, with CAUSAL a key after the query's original position masked, with
+// BUCKET a key outside the query's bucket masked), l += w, and the weights go
+// to P as bf16 pairs right away: P's group g lands on S columns whose values
+// this row has already consumed.  With MASK bits, `others` counts the
+// admissible keys (CAUSAL: the earlier ones; BUCKET alone: those of the
+// query's bucket, self included).
 template <int D, int MASK>
 __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint32_t pcol, const float* cm_lo,
                                              const float* cm_hi, int g_first, int g_self, int lane, int self_mask,
-                                             float m, float& l, const uint32_t (&g0)[32], const int32_t* kp_lo,
-                                             const int32_t* kp_hi, int qpos, const int32_t* kb_lo,
-                                             const int32_t* kb_hi, int qb, int& others, uint32_t (&self_w)[16]) {
-  constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
+                                             float m, float& l, const int32_t* kp_lo, const int32_t* kp_hi,
+                                             int qpos, const int32_t* kb_lo, const int32_t* kb_hi, int qb,
+                                             int& others) {
   uint32_t ra[32], rb[32];
+  tc::tmem_ld32(sbuf + scol, ra);
+  tc::tmem_wait_ld_regs(ra);
 #pragma unroll
-  for (int e = 0; e < 32; ++e) ra[e] = g0[e];  // group 0, loaded by the caller
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    uint32_t(&cur)[32] = (g & 1) ? rb : ra;
-    uint32_t(&nxt)[32] = (g & 1) ? ra : rb;
-    if (g < 3) tc::tmem_ld32(sbuf + scol + 32 * (g + 1), nxt);
-    // key multipliers as 16-byte loads (each group's 32 floats start on a 16-byte boundary)
-    const float4* cm4 = reinterpret_cast<const float4*>(g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2));
-    const int4* kp4 = reinterpret_cast<const int4*>(g < 2 ? kp_lo + 32 * g : kp_hi + 32 * (g - 2));
-    const int4* kb4 = reinterpret_cast<const int4*>(g < 2 ? kb_lo + 32 * g : kb_hi + 32 * (g - 2));
-    const bool dead = g < g_first;
-    uint32_t w16[16];
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      const float4 c4 = cm4[e >> 2];
-      float v0 = __uint_as_float(cur[e]) * ((e & 2) ? c4.z : c4.x);
-      float v1 = __uint_as_float(cur[e + 1]) * ((e & 2) ? c4.w : c4.y);
-      if (CAUSAL || BUCKET) {  // keys are distinct tokens: position == qpos only for self
-        bool c0 = true, c1 = true;  // counted: admissible and (CAUSAL) not self
-        if (CAUSAL) {
-          const int4 k4 = kp4[e >> 2];
-          const int p0 = (e & 2) ? k4.z : k4.x, p1 = (e & 2) ? k4.w : k4.y;
-          if (p0 > qpos) v0 = -INFINITY;
-          if (p1 > qpos) v1 = -INFINITY;
-          c0 = p0 < qpos;
-          c1 = p1 < qpos;
-        }
-        if (BUCKET) {
-          const int4 b4 = kb4[e >> 2];
-          const int b0 = (e & 2) ? b4.z : b4.x, b1 = (e & 2) ? b4.w : b4.y;
-          if (b0 != qb) v0 = -INFINITY;
-          if (b1 != qb) v1 = -INFINITY;
-          c0 = c0 && b0 == qb;
-          c1 = c1 && b1 == qb;
-        }
-        if (!dead) others += (int)c0 + (int)c1;
-      }
-      if (g == g_self && self_mask) {
-        if (e == lane) v0 = -INFINITY;
-        if (e + 1 == lane) v1 = -INFINITY;
-      }
-      const float a = dead ? 0.f : tc::ex2_approx(v0 - m);
-      const float c = dead ? 0.f : tc::ex2_approx(v1 - m);
-      l += a + c;
-      w16[e >> 1] = tc::pack_bf16x2(a, c);
-    }
-    tc::tmem_st16(sbuf + pcol + 16 * g, w16);
-    if ((CAUSAL || BUCKET) && g >= 2 && g == g_self) {
-#pragma unroll
-      for (int k = 0; k < 16; ++k) self_w[k] = w16[k];
-    }
-    if (g < 3) tc::tmem_wait_ld_regs(nxt);
+  for (int h = 0; h < 2; ++h) {  // keys [64 h, 64 h + 64): groups 2h (in ra) and 2h + 1
+    const float* cm = h ? cm_hi : cm_lo;
+    const int32_t* kp = h ? kp_hi : kp_lo;
+    const int32_t* kb = h ? kb_hi : kb_lo;
+    const bool dead = 2 * h < g_first;  // g_first is 0 or 2: both groups of the first half
+    tc::tmem_ld32(sbuf + scol + 64 * h + 32, rb);
+    softmax_group<D, MASK>(sbuf, pcol, 2 * h, ra, cm, kp, kb, dead, self_mask && 2 * h == g_self, lane, m, l,
+                           qpos, qb, others);
+    tc::tmem_wait_ld_regs(rb);
+    if (h == 0) tc::tmem_ld32(sbuf + scol + 64, ra);
+    softmax_group<D, MASK>(sbuf, pcol, 2 * h + 1, rb, cm + 32, kp + 32, kb + 32, dead,
+                           self_mask && 2 * h + 1 == g_self, lane, m, l, qpos, qb, others);
+    if (h == 0) tc::tmem_wait_ld_regs(ra);
   }
 }
 
@@ -408,17 +418,19 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
 // alone in their bucket inside the window) see only themselves: their P becomes
 // one-hot at the own key (bf16 1.0 at element `lane` of the self group) and
 // their weight sum 1 (the shift m is their own logit).  The whole warp rewrites
-// the self group, the other rows with the words they already had.  `others`
-// counts self too when only the bucket mask is on.
+// the self group, the other rows with the words they already had (read back
+// from TMEM).  `others` counts self too when only the bucket mask is on.
 template <int MASK>
 __device__ __forceinline__ void self_only_fixup(uint32_t sbuf, uint32_t pcol, int g_self, int lane, int others,
-                                                const uint32_t (&self_w)[16], float& l) {
+                                                float& l) {
   const bool only = (MASK & kMaskCausal) ? others == 0 : others <= 1;
   if (!__any_sync(0xffffffffu, only)) return;
   uint32_t w16[16];
+  tc::tmem_wait_st();
+  tc::tmem_ld16_wait(sbuf + pcol + 16 * g_self, w16);
 #pragma unroll
   for (int k = 0; k < 16; ++k)
-    w16[k] = !only ? self_w[k] : (k == (lane >> 1) ? ((lane & 1) ? 0x3F800000u : 0x00003F80u) : 0u);
+    if (only) w16[k] = k == (lane >> 1) ? ((lane & 1) ? 0x3F800000u : 0x00003F80u) : 0u;
   tc::tmem_st16(sbuf + pcol + 16 * g_self, w16);
   if (only) l = 1.f;
 }
@@ -426,7 +438,7 @@ __device__ __forceinline__ void self_only_fixup(uint32_t sbuf, uint32_t pcol, in
 // Exact maximum of a row's scaled logits (self excluded while it has other keys;
 // with MASK bits, keys after the query's position / outside its bucket excluded).
 template <int MASK>
-__device__ __forceinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const float* cm_lo, const float* cm_hi,
+__device__ __noinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const float* cm_lo, const float* cm_hi,
                                                int g_first, int g_self, int lane, int self_mask,
                                                const int32_t* kp_lo, const int32_t* kp_hi, int qpos,
                                                const int32_t* kb_lo, const int32_t* kb_hi, int qb) {
@@ -491,12 +503,61 @@ __device__ __noinline__ void restore_s(const uint8_t* smem, uint32_t sbuf, uint3
   tc::tmem_wait_st();
 }
 
+// 32 output values of a row (O columns times 1 / sum of the weights) with 32-byte
+// stores (the row is 32-byte aligned) under the L2 policy `pol`.
+__device__ __forceinline__ void store_o32(__nv_bfloat16* dst, const uint32_t (&raw)[32], float inv_l, uint64_t pol) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 16) {  // 32 bf16 = two 32-byte stores
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      w[k] = tc::pack_bf16x2(__uint_as_float(raw[e + 2 * k]) * inv_l, __uint_as_float(raw[e + 2 * k + 1]) * inv_l);
+    tc::st_global_v8_hint(dst + e, w, pol);
+  }
+}
+__device__ __forceinline__ void store_o32(float* dst, const uint32_t (&raw)[32], float inv_l, uint64_t pol) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 8) {  // 32 floats = four 32-byte stores
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) w[k] = __float_as_uint(__uint_as_float(raw[e + k]) * inv_l);
+    tc::st_global_v8_hint(dst + e, w, pol);
+  }
+}
+
+// The epilogue for output rows that are only 16-byte aligned (16-byte stores),
+// kept out of line: the aligned case is the one the warps run.
+template <int D, typename TO>
+__device__ __noinline__ void epilogue_plain(uint32_t sbuf, TO* dst, float inv_l, bool valid, uint64_t* buf_empty) {
+#pragma unroll 1
+  for (int g = 0; g < D / 32; ++g) {
+    uint32_t raw[32];
+    tc::tmem_ld32(sbuf + kOOff + 32 * g, raw);
+    tc::tmem_wait_ld_regs(raw);
+    if (g == D / 32 - 1) {
+      tc::tc_fence_before();
+      tc::mbar_arrive(buf_empty);
+    }
+    if (valid) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        float y[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y[k] = __uint_as_float(raw[e + k]) * inv_l;
+        store8(dst + 32 * g + e, y);
+      }
+    }
+  }
+}
+
 template <int D, typename TO, int MASK>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) {
   using Lay = Layout<D>;
   constexpr bool MASKED = MASK != 0;  // a self-only fix-up may be needed
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte-aligned base as an offset from the shared array itself (not an integer
+  // cast), so that every access through it stays a shared-memory access
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* full = bars;            // [3] slot filled (64 producer lanes' copies landed)
   uint64_t* empty = bars + 3;       // [3] slot released by the UMMAs
@@ -669,6 +730,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const bool low = q < 2;              // rows 0..63: keys [0, 128); rows 64..127: keys [64, 192)
     const int g_self = 2 + (q & 1);      // 32-key group of the row's own key; in it, element `lane`
+    // per-round outputs are written once and read once by the merge: stored
+    // evict-first, so that the rows the slice's rounds gather again stay in L2
+    const uint64_t pol_out = tc::l2_evict_first();
     StepIter it;
     it.init(p);
     if (wg == 1) it.advance(p);
@@ -689,29 +753,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
         if (!low) colmul[sp * kRows + r] = row_colmul<D>(smem + Lay::kQK + sp * Lay::kSlotBytes, r, p.colscale);
         tc::mbar_arrive(&cm_full[sp]);
       }
-      // own key multiplier from the diagonal of S (||k_r||^2 at key 64 + r % 64); the
-      // pass's first S group is loaded at the same time, so its latency hides
-      // behind the key-multiplier exchange
-      float diag;
-      uint32_t sg0[32];
+      // own key multiplier from the diagonal of S (||k_r||^2 at key 64 + r % 64)
+      float diag = 0.f;
       {
         uint32_t raw[32];
         tc::tmem_ld32(sbuf + scol + 32 * g_self, raw);
-        tc::tmem_ld32(sbuf + scol, sg0);
         tc::tmem_wait_ld_regs(raw);
-        tc::tmem_wait_ld_regs(sg0);
-        diag = 0.f;
 #pragma unroll
         for (int e = 0; e < 32; ++e) diag = (e == lane) ? __uint_as_float(raw[e]) : diag;
       }
       const float cm_own = p.colscale / fmaxf(sqrtf(fmaxf(diag, 0.f)), 1e-12f);
       colmul[sc * kRows + r] = cm_own;
       tc::mbar_arrive(&cm_full[sc]);
+      ok = warp_wait(&cm_full[sp], (fp / kSlots) & 1, abort_flag) &&
+           warp_wait(&cm_full[sc], (fc / kSlots) & 1, abort_flag);
+      if (!ok) break;
       const int chunk = 2 * it.j + (low ? 0 : 1);
       const bool valid = chunk < p.n_chunks;
       const int pos = perm_s[sc * kRows + r];
-      ok = warp_wait(&cm_full[sp], (fp / kSlots) & 1, abort_flag) && warp_wait(&cm_full[sc], (fc / kSlots) & 1, abort_flag);
-      if (!ok) break;
       const float* cm_lo = low ? colmul + sp * kRows + 64 : colmul + sc * kRows;  // keys 0..63 of the row
       const float* cm_hi = low ? colmul + sc * kRows : colmul + sc * kRows + 64;  // keys 64..127
       const int32_t* kp_lo = low ? perm_s + sp * kRows + 64 : perm_s + sc * kRows;  // their positions
@@ -720,31 +779,27 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       const int32_t* kb_hi = low ? bk_s + sc * kRows : bk_s + sc * kRows + 64;
       const int qb = (MASK & kMaskBucket) ? bk_s[sc * kRows + r] : 0;
       int others = 0;
-      uint32_t self_w[16];
       const int g_first = (low && it.j == 0) ? 2 : 0;  // chunk 0 has no previous chunk
       // shift: ||q|| * scale * log2(e) bounds every logit of the row (log2 domain)
-      float m = diag * cm_own;
+      const float m_cs = diag * cm_own;
+      float m = m_cs;
       float l = 0.f;  // sum of the weights (log-sum-exp); O is normalised by the rounded weights' sum
       const uint32_t pcol = low ? 0 : 32;  // P column of the row's first key
-      softmax_pass<D, MASK>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0, kp_lo,
-                            kp_hi, pos, kb_lo, kb_hi, qb, others, self_w);
-      if (MASKED) self_only_fixup<MASK>(sbuf, pcol, g_self, lane, others, self_w, l);
-      if (__any_sync(0xffffffffu, !(l > 1e-30f))) {
+#pragma unroll 1
+      for (int attempt = 0;; ++attempt) {
+        l = 0.f;
+        others = 0;
+        softmax_pass<D, MASK>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, kp_lo,
+                              kp_hi, pos, kb_lo, kb_hi, qb, others);
+        if (MASKED) self_only_fixup<MASK>(sbuf, pcol, g_self, lane, others, l);
+        if (attempt > 0 || !__any_sync(0xffffffffu, !(l > 1e-30f))) break;
         // the bound was too loose for some row of the warp (long query rows): S is
         // rebuilt in TMEM from the rows in shared memory (P has overwritten part of
         // it) and the warp's rows are redone with their exact maxima
         restore_s<D>(smem, sbuf, scol, sp, sc, r, low);
-        const float m_cs = m;
         m = exact_row_max<MASK>(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, kp_lo, kp_hi, pos,
                                 kb_lo, kb_hi, qb);
         if (MASKED && m == -INFINITY) m = m_cs;  // self-only row: its own logit is the shift
-        l = 0.f;
-        others = 0;
-        tc::tmem_ld32(sbuf + scol, sg0);
-        tc::tmem_wait_ld_regs(sg0);
-        softmax_pass<D, MASK>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, sg0,
-                              kp_lo, kp_hi, pos, kb_lo, kb_hi, qb, others, self_w);
-        if (MASKED) self_only_fixup<MASK>(sbuf, pcol, g_self, lane, others, self_w, l);
       }
       {
         uint32_t z[32];
@@ -762,43 +817,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       // O = sum p~ v / sum p~ (p~ the bf16 weights in P): a convex combination of the values
       const float inv_l = 1.f / __uint_as_float(tc::tmem_ld1(sbuf + lr_col<D>()));
       TO* dst = reinterpret_cast<TO*>(p.out) + (it.seg * p.L + pos) * (long long)D;
+      if (p.out_v8) {
 #pragma unroll
-      for (int g = 0; g < D / 32; ++g) {
-        uint32_t raw[32];
-        tc::tmem_ld32(sbuf + kOOff + 32 * g, raw);
-        tc::tmem_wait_ld();
-        if (g == D / 32 - 1) {
-          tc::tc_fence_before();
-          tc::mbar_arrive(&buf_empty[b]);
-        }
-        if (valid) {
-          if (sizeof(TO) == 2 && p.out_v8) {  // 32 bf16 = two 32-byte stores
-#pragma unroll
-            for (int e = 0; e < 32; e += 16) {
-              uint32_t w[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k)
-                w[k] = tc::pack_bf16x2(__uint_as_float(raw[e + 2 * k]) * inv_l, __uint_as_float(raw[e + 2 * k + 1]) * inv_l);
-              tc::st_global_v8(dst + 32 * g + e, w);
-            }
-          } else if (sizeof(TO) == 4 && p.out_v8) {  // 32 floats = four 32-byte stores
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint32_t w[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k) w[k] = __float_as_uint(__uint_as_float(raw[e + k]) * inv_l);
-              tc::st_global_v8(dst + 32 * g + e, w);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              float y[8];
-#pragma unroll
-              for (int k = 0; k < 8; ++k) y[k] = __uint_as_float(raw[e + k]) * inv_l;
-              store8(dst + 32 * g + e, y);
-            }
+        for (int g = 0; g < D / 32; ++g) {
+          uint32_t raw[32];
+          tc::tmem_ld32(sbuf + kOOff + 32 * g, raw);
+          tc::tmem_wait_ld_regs(raw);
+          if (g == D / 32 - 1) {
+            tc::tc_fence_before();
+            tc::mbar_arrive(&buf_empty[b]);
           }
+          if (valid) store_o32(dst + 32 * g, raw, inv_l, pol_out);
         }
+      } else {
+        epilogue_plain<D, TO>(sbuf, dst, inv_l, valid, &buf_empty[b]);
       }
       if (valid) p.lse[it.seg * p.L + pos] = (m + __log2f(l)) * 0.6931471805599453f;
       it.advance(p);

@@ -116,7 +116,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                const Params p) {
   using Lay = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte-aligned base as an offset from the shared array itself (not an integer
+  // cast), so that every access through it stays a shared-memory access
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off(p.half));
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 2;

@@ -282,7 +282,6 @@ lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L, int n_r
     lsh::sort_segment_kernel<<<(unsigned)segs, lsh::kSegWarps * 32, smem, s>>>(buckets, L, n_buckets, perm, inv);
     if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
   } else {
-    if (segs > 65535) return LSH_ERR_UNSUPPORTED;  // grid.y limit of the multi-launch sort
     const int T = lsh::sort_tile(n_buckets);
     const int nt = (L + T - 1) / T;
     uint32_t* cnt = (uint32_t*)workspace;
@@ -293,7 +292,7 @@ lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L, int n_r
       cudaFuncSetAttribute(lsh::sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
       cudaFuncSetAttribute(lsh::sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
   }
-    dim3 grid(nt, (unsigned)segs);
+    dim3 grid((unsigned)segs, nt);
     lsh::sort_count_kernel<<<grid, 256, hist_smem, s>>>(buckets, L, n_buckets, T, cnt);
     if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
     lsh::sort_scan_kernel<<<(unsigned)segs, 1024, 0, s>>>(cnt, (long long)n_buckets * nt);
@@ -352,13 +351,22 @@ lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H, int L,
   if (!aligned16(buckets) || !aligned16(perm) || (inv && !aligned16(inv))) return LSH_ERR_ALIGN;
   const long long segs = (long long)B * H * n_rounds;
   if (segs == 0 || L == 0) return LSH_OK;
+  cudaStream_t s = as_stream(stream);
+  if (sort_by_segment(L, n_buckets)) {
+    // one CTA per segment, all state in shared memory: no scratch at all
+    const size_t smem = lsh::sort_segment_smem(L, n_buckets);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(lsh::sort_segment_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+      return LSH_ERR_CUDA;
+    lsh::sort_segment_kernel<<<(unsigned)segs, lsh::kSegWarps * 32, smem, s>>>(buckets, L, n_buckets, perm, inv);
+    return launch_status();
+  }
   const size_t words = lsh::sort_ws_elems(segs, L, n_buckets);
   if (words > kNoallocScratchWords) return LSH_ERR_WORKSPACE;
-  if (segs > 65535) return LSH_ERR_UNSUPPORTED;
   uint32_t* cnt = noalloc_scratch_ptr();
   if (!cnt) return LSH_ERR_CUDA;
 
-  cudaStream_t s = as_stream(stream);
   const int T = lsh::sort_tile(n_buckets);
   const int nt = (L + T - 1) / T;
   const bool in_smem = n_buckets <= kSortSmemBuckets;
@@ -369,7 +377,7 @@ lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H, int L,
     cudaFuncSetAttribute(lsh::sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
     cudaFuncSetAttribute(lsh::sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
   }
-  dim3 grid(nt, (unsigned)segs);
+  dim3 grid((unsigned)segs, nt);
   lsh::sort_count_kernel<<<grid, 256, hist_smem, s>>>(buckets, L, n_buckets, T, cnt);
   if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
   lsh::sort_scan_kernel<<<(unsigned)segs, 1024, 0, s>>>(cnt, (long long)n_buckets * nt);

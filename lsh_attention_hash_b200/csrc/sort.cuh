@@ -37,8 +37,9 @@ __global__ void __launch_bounds__(256)
 sort_count_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, int T,
                   uint32_t* __restrict__ cnt) {
   extern __shared__ uint32_t hist[];
-  const int tile = blockIdx.x, nt = gridDim.x;
-  const long long seg = blockIdx.y;
+  // segments on grid.x (up to 2^31 - 1 of them), tiles on grid.y (at most L / 4096 <= 4096)
+  const int tile = blockIdx.y, nt = gridDim.y;
+  const long long seg = blockIdx.x;
   const bool in_smem = n_buckets <= kSortSmemBuckets;
   uint32_t* gcnt = cnt + (size_t)seg * n_buckets * nt;
   if (in_smem) {
@@ -114,8 +115,8 @@ __global__ void __launch_bounds__(32)
 sort_scatter_kernel(const int32_t* __restrict__ buckets, int L, int n_buckets, int T,
                     uint32_t* __restrict__ cnt, int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   extern __shared__ uint32_t run[];
-  const int tile = blockIdx.x, nt = gridDim.x;
-  const long long seg = blockIdx.y;
+  const int tile = blockIdx.y, nt = gridDim.y;
+  const long long seg = blockIdx.x;
   const int lane = threadIdx.x;
   const bool in_smem = n_buckets <= kSortSmemBuckets;
   uint32_t* gcnt = cnt + (size_t)seg * n_buckets * nt;

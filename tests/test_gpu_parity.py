@@ -364,3 +364,4 @@ def test_64k_workload_bucket_mask_sampled_slices():
     """The full-size launch with the bucket mask alone (tensor-core path), sampled slots of two slices."""
     w = synth.WORKLOADS["64k"]
     _sampled_slices(w, [(0, 0), (7, 7)], slot_sample=2048, bucket_mask=True)
+

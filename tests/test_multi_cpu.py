@@ -6,12 +6,14 @@ their own timings."""
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from lsh_attention_hash_b200 import multi, synth
+from oracle import oracle_lsh_attention
 
 
 def _free_port():
@@ -49,6 +51,53 @@ def test_two_gloo_ranks_agree_on_max_timing_and_draw_distinct_batches():
         assert got == [11.0, 5.0]                # max over ranks of (10 + r, 5 - r)
         assert digests[0] != digests[1]          # the ranks' inputs differ
     assert out[0][1] == out[1][1]
+
+
+def _shard_main(rank, world, port, out):
+    """Strong scaling by slices: the rank computes the (b, h) slices of its shard of one batch
+    (the float64 oracle stands in for a GPU's four calls), then the ranks all-gather the outputs."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = synth.small_workload("shard", 2, 3, 128, 16, "f32", 8, 32, 2)
+        qk, v, R = synth.make_inputs(w, seed=7)
+        mine = multi.shard_slices(w.B, w.H, rank, world)
+        local = np.zeros((len(mine), w.L, w.D))
+        local_lse = np.zeros((len(mine), w.L))
+        for n, (b, h) in enumerate(mine):
+            res = oracle_lsh_attention(qk[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], R, w.n_buckets, w.chunk)
+            local[n] = res["out"][0, 0]
+            local_lse[n] = res["lse"][0, 0]
+        # equal-size buffers for all_gather: pad to the largest shard
+        n_max = max(len(multi.shard_slices(w.B, w.H, r, world)) for r in range(world))
+        send = torch.zeros((n_max, w.L, w.D + 1), dtype=torch.float64)
+        send[:len(mine), :, :w.D] = torch.from_numpy(local)
+        send[:len(mine), :, w.D] = torch.from_numpy(local_lse)
+        recv = [torch.zeros_like(send) for _ in range(world)]
+        dist.all_gather(recv, send)
+        full = np.zeros((w.B * w.H, w.L, w.D + 1))
+        for r in range(world):
+            lo, hi = multi.slice_shard(w.B, w.H, r, world)
+            full[lo:hi] = recv[r][:hi - lo].numpy()
+        out[rank] = full
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_slice_shards_gathered_equal_one_process_run(world):
+    manager = mp.get_context("spawn").Manager()
+    out = manager.dict()
+    mp.start_processes(_shard_main, args=(world, _free_port(), out), nprocs=world, start_method="spawn",
+                       join=True)
+    w = synth.small_workload("shard", 2, 3, 128, 16, "f32", 8, 32, 2)
+    qk, v, R = synth.make_inputs(w, seed=7)
+    ref = oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk)
+    want = np.concatenate([ref["out"].reshape(w.B * w.H, w.L, w.D),
+                           ref["lse"].reshape(w.B * w.H, w.L, 1)], axis=2)
+    for rank in range(world):
+        assert np.array_equal(out[rank], want), f"rank {rank}"
 
 
 def test_max_over_ranks_without_process_group_is_identity():

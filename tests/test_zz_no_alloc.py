@@ -7,9 +7,10 @@ synchronisation).  Instead of a caller workspace it uses a 16 MiB static
 device array inside the library, which keeps the previous call's contents.
 
 The test calls it through the C ABI twice in a row, on different inputs, for
-both counter paths of the sort (shared-memory histograms, and global-memory
-counters that the call must clear itself), and checks that every result is
-identical to the workspace-based lsh_sort_permute.  Sizes beyond the static
+every path of the sort (one CTA per segment with no scratch at all, as at the
+64K workload; shared-memory histograms; global-memory counters that the call
+must clear itself), and checks that every result is identical to the
+workspace-based lsh_sort_permute.  Sizes beyond the static
 array are rejected with LSH_ERR_WORKSPACE before any launch.  This file runs
 last (pytest collects it after the others) and also passes on its own.
 """
@@ -44,7 +45,9 @@ def _noalloc(buckets, n_buckets, perm, inv):
 
 
 @pytest.mark.parametrize("shape,n_buckets", [
-    ((2, 3, 2, 5000), 64),        # counters in shared memory, ragged last tile
+    ((1, 2, 4, 65536), 1024),     # the 64K workload's segments: one CTA per segment, no scratch
+    ((1, 1, 70000, 16), 16),      # more than 65535 segments (one CTA per segment)
+    ((2, 3, 2, 70000), 64),       # counters in shared memory, ragged last tile
     ((1, 2, 1, 70000), 32768),    # counters in global memory: cleared by the call
 ])
 def test_noalloc_sort_matches_workspace_sort_on_consecutive_calls(shape, n_buckets):

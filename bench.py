@@ -192,10 +192,13 @@ def mask_config(args):
     return {"mask": "+".join(names)} if names else {}
 
 
-def oracle_sample(w, slices=1, seed=0, masks=None, threads=None):
+def oracle_sample(w, slices=1, seed=0, masks=None, threads=None, max_tokens=None):
     """Runs the float64 oracle on `slices` (b, h) slices of the workload, all rounds.
 
     `threads` caps the BLAS thread pools (None: as many as the library starts).
+    `max_tokens` (a multiple of the chunk) bounds the sample on very long
+    sequences: the oracle then runs on the first `max_tokens` positions of each
+    slice with the workload's own D, buckets, chunk and rounds.
     Returns (seconds, tokens, threads).
     """
     import contextlib
@@ -213,29 +216,45 @@ def oracle_sample(w, slices=1, seed=0, masks=None, threads=None):
         for n in range(slices):
             b, h = divmod(n % (w.B * w.H), w.H)
             qk_s, v_s = synth.slice_inputs(w, b, h, seed)
+            if max_tokens is not None and max_tokens < w.L:
+                qk_s, v_s = qk_s[:max_tokens], v_s[:max_tokens]
             qk = qk_s[None, None]
             v = v_s[None, None]
             t0 = time.perf_counter()
             oracle_lsh_attention(qk, v, R, w.n_buckets, w.chunk, **(masks or {}))
             secs += time.perf_counter() - t0
-            tokens += w.L
+            tokens += qk_s.shape[0]
         info = threadpoolctl.threadpool_info()
         used = max([i.get("num_threads", 1) for i in info] + [1])
     return secs, tokens, used
 
 
+def cpu_sample_plan(w, seconds=10.0):
+    """(slices, max_tokens) of a bounded oracle sample of about `seconds` of float64 CPU work: the
+    oracle runs at about 1.5e10 operations/s here, and a token costs its hash (D * n_buckets per
+    round) and its attention (8 * chunk * D per round).  Long sequences are cut to a prefix of a
+    slice (a multiple of the chunk); short ones repeat slices (at most 256)."""
+    per_token = w.n_rounds * (w.D * w.n_buckets + 8 * w.chunk * w.D) + 2000
+    tokens = max(w.chunk, int(1.5e10 * seconds / per_token))
+    if tokens >= w.L:
+        return min(256, max(1, tokens // w.L)), None
+    return 1, max(w.chunk, (tokens // w.chunk) * w.chunk)
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return
+    slices, cap = cpu_sample_plan(w, seconds=4.0)
     for _ in range(args.warmup):
-        oracle_sample(w, 1, masks=mask_options(args))
+        oracle_sample(w, 1, masks=mask_options(args), max_tokens=cap)
     secs, tokens, threads = 0.0, 0, 1
     for _ in range(args.steps):
-        s, t, threads = oracle_sample(w, 1, masks=mask_options(args))
+        s, t, threads = oracle_sample(w, slices, masks=mask_options(args), max_tokens=cap)
         secs += s
         tokens += t
     value = tokens / secs
-    sample = f"one (b,h) slice of the workload per step ({w.L} tokens, all {w.n_rounds} rounds), float64 NumPy oracle"
+    what = f"the first {cap} tokens of a (b,h) slice" if cap else f"{slices} (b,h) slice(s) ({slices * w.L} tokens)"
+    sample = f"per step {what} of the workload, all {w.n_rounds} rounds, float64 NumPy oracle"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
@@ -411,9 +430,15 @@ def run_ours(args, w, rank, world, local_rank):
     else:
         sort_launches = 3 + (1 if w.n_buckets > 16384 else 0)  # count, scan, scatter (+ counter clear)
     launches_per_step = 3 + sort_launches                  # hash, sort, attend, combine
-    sample_slices = 2  # about 10 s of float64 CPU work at the 64K workload
-    c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices, masks=masks)
-    o_secs, o_tokens, _ = oracle_sample(w, 1, masks=masks, threads=1)
+    sample_slices, sample_cap = cpu_sample_plan(w, 10.0)  # about 10 s of float64 CPU work
+    c_secs, c_tokens, c_threads = oracle_sample(w, sample_slices, masks=masks, max_tokens=sample_cap)
+    one_slices, one_cap = cpu_sample_plan(w, 6.0)
+    o_secs, o_tokens, _ = oracle_sample(w, one_slices, masks=masks, threads=1, max_tokens=one_cap)
+
+    def sample_text(slices, cap, tokens):
+        if cap:
+            return f"the first {cap} tokens of a (b,h) slice"
+        return f"{slices} (b,h) slice(s) of the workload ({tokens} tokens)"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -435,11 +460,11 @@ def run_ours(args, w, rank, world, local_rank):
         "clocks": clk.summary(),
         "cpu_baseline": {"value": c_tokens / c_secs, "unit": UNIT, "cores": c_threads, "kind": "oracle",
                          "affinity_cores": len(os.sched_getaffinity(0)),
-                         "sample": f"{sample_slices} (b,h) slice(s) of the workload ({c_tokens} tokens, all "
-                                   f"{w.n_rounds} rounds), float64 NumPy oracle, {c_secs:.1f} s",
+                         "sample": f"{sample_text(sample_slices, sample_cap, c_tokens)}, all {w.n_rounds} rounds, "
+                                   f"float64 NumPy oracle, {c_secs:.1f} s",
                          "one_core": {"value": o_tokens / o_secs, "unit": UNIT, "cores": 1,
-                                      "sample": f"1 (b,h) slice ({o_tokens} tokens, all {w.n_rounds} rounds), "
-                                                f"BLAS pools capped at one thread, {o_secs:.1f} s"}},
+                                      "sample": f"{sample_text(one_slices, one_cap, o_tokens)}, all {w.n_rounds} "
+                                                f"rounds, BLAS pools capped at one thread, {o_secs:.1f} s"}},
     }
     if args.backward:
         sms = torch.cuda.get_device_properties(dev).multi_processor_count

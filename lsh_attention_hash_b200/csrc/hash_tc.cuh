@@ -3,13 +3,16 @@
 // Ultralytics glossary "Reformer", section "Atencao LSH": bucket = position of
 // the largest value of [xR, -xR] for a random projection R per round.
 //
-// Served case: bf16 rows, D in {64, 128}, n_buckets/2 = `half` a multiple of
-// 64 with half <= 256 or half % 256 == 0, and R[round] small enough to stay in
-// shared memory (D * half * 2 <= 128 KB).  Each persistent CTA owns one round:
-// R[round] is loaded once by TMA (MN-major, 128-byte swizzle) and 128-row tiles
-// of QK stream through a two-stage TMA ring.  p = x R accumulates in fp32 in
-// TMEM (two buffers of NC <= 256 columns, so the next tile's UMMA overlaps the
-// current epilogue).
+// Served case: bf16 rows, D in {64, 128}, n_buckets/2 = `half` 32, or a
+// multiple of 64 with half <= 256 or half % 256 == 0 (half = 32: R[round] is
+// copied into a 64-column tile whose upper 32 columns are zero, by plain loads).  Each persistent CTA owns one round
+// and 128-row tiles of QK stream through a two-stage TMA ring.  R[round] (MN-
+// major, 128-byte swizzle) either stays in shared memory, loaded once by TMA
+// (D * half * 2 <= 128 KB), or, for larger bucket counts (RS > 0), streams
+// through an RS-stage TMA ring in chunks of NC columns for every tile (it is
+// re-read from L2, where the rounds' projections stay).  p = x R accumulates in
+// fp32 in TMEM (two buffers of NC <= 256 columns, so the next chunk's UMMA
+// overlaps the current epilogue).
 //
 // Epilogue (one row per thread): the bucket is argmax over [p, -p], i.e. the
 // largest |p_k| and its sign.  Values are handled in groups of 16: the key of
@@ -36,21 +39,33 @@ constexpr int kRows = 128;
 __host__ __device__ constexpr int threads_for(int split) { return 64 + 128 * split; }
 constexpr int kStages = 2;
 
+constexpr int kMaxRS = 4;  // stages of the streamed projection ring
+
 template <int D>
 struct Layout {
   static constexpr uint32_t kHalfBytes = kRows * 128;           // 128 rows x 64 bf16
   static constexpr uint32_t kStageBytes = (D / 64) * kHalfBytes;
   static constexpr uint32_t kA = 0;
-  static constexpr uint32_t kR = kStages * kStageBytes;          // R[round]: (half/64) boxes of D x 128 B
-  __host__ __device__ static constexpr uint32_t bar_off(int half) { return kR + (uint32_t)D * half * 2; }
+  static constexpr uint32_t kR = kStages * kStageBytes;          // R: (columns / 64) boxes of D x 128 B
+  // resident: all of R[round] (at least one 64-column box); streamed: RS chunks of nc columns
+  __host__ __device__ static constexpr uint32_t r_bytes(int half, int nc, int rs) {
+    return rs ? (uint32_t)rs * D * nc * 2 : (uint32_t)D * (half < 64 ? 64 : half) * 2;
+  }
+  __host__ __device__ static constexpr uint32_t bar_off(int half, int nc, int rs) { return kR + r_bytes(half, nc, rs); }
   // a_full[2] a_empty[2] acc_full[2] acc_empty[2] r_full done part_done[2] merged[2]
-  static constexpr int kNumBars = 14;
+  // then the streamed ring's rs_full[kMaxRS] rs_empty[kMaxRS]
+  static constexpr int kNumBars = 14 + 2 * kMaxRS;
   // row states of parts 1..3: [2 tile parities][3 parts][5 fields][128 rows] x 4 B
-  __host__ __device__ static constexpr uint32_t xchg_off(int half) { return bar_off(half) + kNumBars * 8 + 16; }
-  __host__ __device__ static constexpr uint32_t smem_bytes(int half) { return xchg_off(half) + 2 * 3 * 5 * kRows * 4 + 1024; }
+  __host__ __device__ static constexpr uint32_t xchg_off(int half, int nc, int rs) {
+    return bar_off(half, nc, rs) + kNumBars * 8 + 16;
+  }
+  __host__ __device__ static constexpr uint32_t smem_bytes(int half, int nc, int rs) {
+    return xchg_off(half, nc, rs) + 2 * 3 * 5 * kRows * 4 + 1024;
+  }
 };
 
 struct Params {
+  const __nv_bfloat16* r;  // [n_rounds][D][half] (the 32-column case copies it by plain loads)
   int32_t* buckets;    // [B*H][n_rounds][L]
   uint8_t* near_tie;   // same, nullable
   long long nrows;     // B*H*L
@@ -110,7 +125,7 @@ __device__ __forceinline__ void process16(RowState& st, const uint32_t* raw, int
   }
 }
 
-template <int D, int NC, bool FLAG, int SPLIT>
+template <int D, int NC, bool FLAG, int SPLIT, int RS>
 __global__ void __launch_bounds__(threads_for(SPLIT), 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_r,
                const Params p) {
@@ -119,7 +134,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   // 1024-byte-aligned base as an offset from the shared array itself (not an integer
   // cast), so that every access through it stays a shared-memory access
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off(p.half));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bar_off(p.half, NC, RS));
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 2;
   uint64_t* acc_full = bars + 4;
@@ -128,7 +143,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   uint64_t* done_bar = bars + 9;
   uint64_t* part_done = bars + 10;  // [2] parts 1.. states written ((SPLIT-1) * 128 arrivals)
   uint64_t* merged = bars + 12;     // [2] those states consumed (128 arrivals)
-  float* xchg = reinterpret_cast<float*>(smem + Lay::xchg_off(p.half));
+  uint64_t* rs_full = bars + 14;    // [RS] streamed R chunk landed
+  uint64_t* rs_empty = rs_full + kMaxRS;  // [RS] its UMMAs retired
+  float* xchg = reinterpret_cast<float*>(smem + Lay::xchg_off(p.half, NC, RS));
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + Lay::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + Lay::kNumBars) + 1;
 
@@ -141,11 +158,15 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       tc::mbar_init(&a_empty[i], 1);
       tc::mbar_init(&acc_full[i], 1);
       tc::mbar_init(&acc_empty[i], 128 * SPLIT);
-      tc::mbar_init(&part_done[i], 128 * (SPLIT - 1));
+      tc::mbar_init(&part_done[i], SPLIT > 1 ? 128 * (SPLIT - 1) : 1);  // unused with one part
       tc::mbar_init(&merged[i], 128);
     }
     tc::mbar_init(r_full, 1);
     tc::mbar_init(done_bar, 1);
+    for (int i = 0; i < RS; ++i) {
+      tc::mbar_init(&rs_full[i], 1);
+      tc::mbar_init(&rs_empty[i], 1);
+    }
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -156,13 +177,30 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
+    if (RS == 0 && p.half < 64) {
+      // R[round] (D x 32) into one 64-column MN-major tile with the 128-byte
+      // swizzle: row k holds columns 0..31 in its 16-byte pieces 0..3, pieces
+      // 4..7 are zero (the UMMA reads only N = 32 columns of it)
+      const __nv_bfloat16* rsrc = p.r + (size_t)round * D * p.half;
+      for (int idx = lane; idx < D * 8; idx += 32) {
+        const int k = idx >> 3, c = idx & 7;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (c < 4) val = *reinterpret_cast<const uint4*>(rsrc + (size_t)k * p.half + c * 8);
+        *reinterpret_cast<uint4*>(smem + Lay::kR + k * 128 + ((c ^ (k & 7)) << 4)) = val;
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(r_full);
+    }
     if (lane == 0) {
       tc::prefetch_tensormap(&map_x);
       tc::prefetch_tensormap(&map_r);
-      tc::mbar_arrive_expect_tx(r_full, (uint32_t)D * p.half * 2);
-      for (int b = 0; b < p.half / 64; ++b)
-        tc::tma_load_2d(smem + Lay::kR + b * D * 128, &map_r, r_full, b * 64, round * D);
-      uint32_t it = 0;
+      if (RS == 0 && p.half >= 64) {  // R[round] resident: loaded once
+        tc::mbar_arrive_expect_tx(r_full, (uint32_t)D * p.half * 2);
+        for (int b = 0; b < p.half / 64; ++b)
+          tc::tma_load_2d(smem + Lay::kR + b * D * 128, &map_r, r_full, b * 64, round * D);
+      }
+      uint32_t it = 0, rq = 0;
       bool ok = true;
       for (long long tile = first_tile; tile < p.n_tiles; tile += p.per_round, ++it) {
         const int s = it % kStages;
@@ -173,6 +211,19 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         for (int h = 0; h < D / 64; ++h)
           tc::tma_load_2d(smem + Lay::kA + s * Lay::kStageBytes + h * Lay::kHalfBytes, &map_x, &a_full[s], h * 64,
                           (int)(tile * kRows));
+        if (RS > 0) {  // the tile's pass over R[round], chunk by chunk
+          for (int c = 0; ok && c < p.nchunks; ++c, ++rq) {
+            const int sr = rq % RS;
+            ok = tc::mbar_wait(&rs_empty[sr], ((rq / RS) & 1) ^ 1, abort_flag);
+            if (!ok) break;
+            tc::mbar_arrive_expect_tx(&rs_full[sr], (uint32_t)D * NC * 2);
+#pragma unroll
+            for (int b = 0; b < NC / 64; ++b)
+              tc::tma_load_2d(smem + Lay::kR + sr * (D * NC * 2) + b * D * 128, &map_r, &rs_full[sr],
+                              c * NC + b * 64, round * D);
+          }
+          if (!ok) break;
+        }
       }
       // never leave with copies in flight
       for (uint32_t k = (it > kStages ? it - kStages : 0); k < it; ++k) {
@@ -180,9 +231,14 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         while (!tc::mbar_try_wait(&a_full[k % kStages], (k / kStages) & 1))
           if (tc::globaltimer() - t0 > tc::kWaitNs / 16) break;
       }
-      {
+      if (RS == 0 && p.half >= 64) {
         const unsigned long long t0 = tc::globaltimer();
         while (!tc::mbar_try_wait(r_full, 0))
+          if (tc::globaltimer() - t0 > tc::kWaitNs / 16) break;
+      }
+      for (uint32_t k = (rq > (uint32_t)RS ? rq - RS : 0); k < rq; ++k) {
+        const unsigned long long t0 = tc::globaltimer();
+        while (!tc::mbar_try_wait(&rs_full[k % RS], (k / RS) & 1))
           if (tc::globaltimer() - t0 > tc::kWaitNs / 16) break;
       }
     }
@@ -192,24 +248,35 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       const uint32_t idesc = tc::idesc_bf16_f32(128, NC, 0, 1);
       const uint32_t a0 = tc::smem_u32(smem + Lay::kA);
       const uint32_t r0 = tc::smem_u32(smem + Lay::kR);
-      bool ok = tc::mbar_wait(r_full, 0, abort_flag);
-      uint32_t it = 0, seq = 0;
+      bool ok = RS > 0 || tc::mbar_wait(r_full, 0, abort_flag);
+      uint32_t it = 0, seq = 0, rq = 0;
       for (long long tile = first_tile; ok && tile < p.n_tiles; tile += p.per_round, ++it) {
         const int s = it % kStages;
         ok = tc::mbar_wait(&a_full[s], (it / kStages) & 1, abort_flag);
         if (!ok) break;
         for (int c = 0; c < p.nchunks; ++c, ++seq) {
           const int b = seq & 1;
+          const int sr = RS > 0 ? (int)(rq % RS) : 0;
+          if (RS > 0) {
+            ok = tc::mbar_wait(&rs_full[sr], (rq / RS) & 1, abort_flag);
+            if (!ok) break;
+          }
           ok = tc::mbar_wait(&acc_empty[b], ((seq >> 1) & 1) ^ 1, abort_flag);
           if (!ok) break;
           tc::tc_fence_after();
+          // chunk c of R[round]: resident at its offset, or the ring stage it streamed into
+          const uint32_t rbase = RS > 0 ? r0 + sr * (D * NC * 2) : r0 + (c * (NC / 64)) * D * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t ad = tc::sdesc_sw128(a0 + s * Lay::kStageBytes + (kk >> 2) * Lay::kHalfBytes + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = tc::sdesc_sw128(r0 + (c * (NC / 64)) * D * 128 + kk * 2048, D * 128, 1024);
+            const uint64_t bd = tc::sdesc_sw128(rbase + kk * 2048, D * 128, 1024);
             tc::umma_ss(tmem + b * NC, ad, bd, idesc, kk > 0);
           }
           tc::umma_commit(&acc_full[b]);
+          if (RS > 0) {
+            tc::umma_commit(&rs_empty[sr]);
+            ++rq;
+          }
         }
         if (!ok) break;
         tc::umma_commit(&a_empty[s]);
@@ -250,7 +317,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       }
       if (!ok) break;
       const int tp = it & 1;
-      if (ch > 0) {
+      if (SPLIT > 1 && ch > 0) {
         float* xs = xchg + (tp * 3 + (ch - 1)) * 5 * kRows;
         ok = att_tc::warp_wait(&merged[tp], ((it >> 1) & 1) ^ 1, abort_flag);
         if (!ok) break;
@@ -262,8 +329,10 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         tc::mbar_arrive(&part_done[tp]);
         continue;
       }
-      ok = att_tc::warp_wait(&part_done[tp], (it >> 1) & 1, abort_flag);
-      if (!ok) break;
+      if (SPLIT > 1) {
+        ok = att_tc::warp_wait(&part_done[tp], (it >> 1) & 1, abort_flag);
+        if (!ok) break;
+      }
 #pragma unroll
       for (int o = 0; o < SPLIT - 1; ++o) {
         const float* xs = xchg + (tp * 3 + o) * 5 * kRows;
@@ -281,7 +350,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
           st.v1 = fmaxf(st.v1, o_v1);
         }
       }
-      tc::mbar_arrive(&merged[tp]);
+      if (SPLIT > 1) tc::mbar_arrive(&merged[tp]);
       const long long row = tile * kRows + r;
       if (row < p.nrows) {
         const uint32_t kb = __float_as_uint(st.best_key);

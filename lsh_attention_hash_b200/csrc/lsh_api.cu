@@ -98,23 +98,31 @@ inline bool make_tile_map(CUtensorMap* map, const void* base, long long rows, lo
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Whether the tensor-core hash serves this shape (see hash_tc.cuh).
+// Whether the tensor-core hash serves this shape (see hash_tc.cuh): R[round]
+// resident in shared memory (D * half * 2 <= 128 KB) or streamed in chunks of
+// 256 columns (half a multiple of 256).
 inline bool hash_tc_eligible(int dtype, int D, int half, int n_rounds, const DevInfo& di) {
   if (dtype != LSH_BF16 || di.major != 10 || (D != 64 && D != 128)) return false;
-  if (half % 64 != 0 || !(half <= 256 ? (half == 64 || half == 128 || half == 256) : half % 256 == 0)) return false;
-  if ((long long)D * half * 2 > 128 * 1024) return false;
+  if (half != 32 && (half % 64 != 0 || !(half <= 256 ? (half == 64 || half == 128 || half == 256) : half % 256 == 0)))
+    return false;
   return n_rounds <= di.sms;
 }
+inline bool hash_tc_streams_r(int D, int half) { return (long long)D * half * 2 > 128 * 1024; }
 
-template <int D, int NC, bool FLAG, int SPLIT>
+template <int D, int NC, bool FLAG, int SPLIT, int RS>
 lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, int n_rounds, int half,
                           int32_t* buckets, uint8_t* near_tie, cudaStream_t s, int sms) {
   using namespace lsh::hash_tc;
   const long long rows = (long long)B * H * L;
   CUtensorMap mx, mr;
-  if (!make_tile_map(&mx, qk, rows, D, 64, kRows) || !make_tile_map(&mr, R, (long long)n_rounds * D, half, 64, D))
-    return LSH_ERR_CUDA;
+  if (!make_tile_map(&mx, qk, rows, D, 64, kRows)) return LSH_ERR_CUDA;
+  if (half >= 64) {
+    if (!make_tile_map(&mr, R, (long long)n_rounds * D, half, 64, D)) return LSH_ERR_CUDA;
+  } else {
+    mr = mx;  // 32 columns: the kernel copies R[round] by plain loads and never reads this map
+  }
   Params p;
+  p.r = static_cast<const __nv_bfloat16*>(R);
   p.buckets = buckets;
   p.near_tie = near_tie;
   p.nrows = rows;
@@ -126,8 +134,8 @@ lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, in
   p.per_round = (int)std::max<long long>(1, std::min<long long>(sms / n_rounds, p.n_tiles));
   p.key_mask = 0x7FFFFFF0u;
   const unsigned grid = (unsigned)(p.per_round * n_rounds);
-  auto kfn = hash_tc_kernel<D, NC, FLAG, SPLIT>;
-  const int smem = (int)Layout<D>::smem_bytes(half);
+  auto kfn = hash_tc_kernel<D, NC, FLAG, SPLIT, RS>;
+  const int smem = (int)Layout<D>::smem_bytes(half, NC, RS);
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LSH_ERR_CUDA;
   kfn<<<grid, threads_for(SPLIT), smem, s>>>(mx, mr, p);
@@ -137,15 +145,21 @@ lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, in
 template <int D>
 lsh_status dispatch_hash_tc(const void* qk, const void* R, int B, int H, int L, int n_rounds, int half,
                             int32_t* buckets, uint8_t* near_tie, cudaStream_t s, int sms) {
-#define LSH_HTC(NC)                                                                                    \
-  return near_tie                                                                                      \
-             ? launch_hash_tc<D, NC, true, (NC >= 128 ? 4 : 2)>(qk, R, B, H, L, n_rounds, half, buckets, \
-                                                                 near_tie, s, sms)                     \
-             : launch_hash_tc<D, NC, false, (NC >= 128 ? 4 : 2)>(qk, R, B, H, L, n_rounds, half, buckets, \
-                                                                  near_tie, s, sms)
-  if (half == 64) LSH_HTC(64);
-  if (half == 128) LSH_HTC(128);
-  LSH_HTC(256);
+#define LSH_HTC(NC, RS)                                                                                  \
+  return near_tie                                                                                        \
+             ? launch_hash_tc<D, NC, true, (NC >= 128 ? 4 : 2), RS>(qk, R, B, H, L, n_rounds, half, buckets, \
+                                                                     near_tie, s, sms)                     \
+             : launch_hash_tc<D, NC, false, (NC >= 128 ? 4 : 2), RS>(qk, R, B, H, L, n_rounds, half, buckets, \
+                                                                      near_tie, s, sms)
+  // streamed projection ring: 3 chunks of 32 KB at D 64, 2 of 64 KB at D 128
+  if (hash_tc_streams_r(D, half)) LSH_HTC(256, D == 64 ? 3 : 2);
+  if (half == 32) {  // one epilogue part (32 columns)
+    return near_tie ? launch_hash_tc<D, 32, true, 1, 0>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, sms)
+                    : launch_hash_tc<D, 32, false, 1, 0>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, sms);
+  }
+  if (half == 64) LSH_HTC(64, 0);
+  if (half == 128) LSH_HTC(128, 0);
+  LSH_HTC(256, 0);
 #undef LSH_HTC
 }
 

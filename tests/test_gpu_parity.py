@@ -365,3 +365,22 @@ def test_64k_workload_bucket_mask_sampled_slices():
     w = synth.WORKLOADS["64k"]
     _sampled_slices(w, [(0, 0), (7, 7)], slot_sample=2048, bucket_mask=True)
 
+
+
+@pytest.mark.parametrize("D,n_buckets,L", [(64, 4096, 1000), (128, 1536, 777), (64, 16384, 300),
+                                           (128, 64, 1000), (64, 64, 777)])
+def test_hash_streamed_and_narrow_projection(D, n_buckets, L):
+    """The tensor-core hash's edge layouts of R[round]: bucket counts whose projection does not fit
+    in shared memory (D * n_buckets > 128 K elements; R streams in 256-column chunks through a ring
+    for every 128-row tile) and 64 buckets (32 columns, copied into a zero-padded 64-column tile,
+    one epilogue part).  Buckets bit-exact against the float64 oracle except flagged rows, ragged
+    row counts, several rounds; the flag-free instantiation (the one the bench times) agrees with
+    the flagged one on every row."""
+    w = synth.small_workload("stream", 1, 2, L, D, "bf16", n_buckets, 64 if L % 64 == 0 else 1, 3)
+    qk, v, R = synth.make_inputs(w, seed=21)
+    qk_d, R_d = qk.to(DEV), R.to(DEV)
+    b, nt = lsh.lsh_hash(qk_d, R_d, w.n_buckets)
+    b_nf, _ = lsh.lsh_hash(qk_d, R_d, w.n_buckets, with_near_tie=False)
+    assert lsh.lsh_get_device_status() == 0
+    parity.check_hash(qk, R, w.n_buckets, b, nt, 1e-2)
+    assert torch.equal(b, b_nf)

@@ -60,12 +60,19 @@ constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBufCols = 256;  // one step buffer
 constexpr uint32_t kOOff = 96;      // O columns inside a step buffer
+// registers per thread after the launch's 168: warpgroup 0 (producers, issuers)
+// gives up 64, the two softmax warpgroups take 24 each (128 x 64 >= 256 x 24)
+constexpr uint32_t kLowRegs = 104, kSoftRegs = 192;
 template <int D>
 __host__ __device__ constexpr uint32_t lr_col() { return kOOff + D; }
 
 // Compile-time masks of an instantiation (besides the self mask, a runtime flag).
 constexpr int kMaskCausal = 1;  // a key after the query's original position is not admissible
 constexpr int kMaskBucket = 2;  // a key in another bucket than the query's is not admissible
+// (with kMaskBucket) each admissible logit is lowered by log N, N = the number of
+// rounds (at most kUnionRounds) whose hash puts query and key in one bucket
+constexpr int kMaskUnion = 4;
+constexpr int kUnionRounds = 8;
 
 template <int D>
 struct Layout {
@@ -78,7 +85,10 @@ struct Layout {
   static constexpr uint32_t kPerm = kOnes + 16 * 128;               // int32 [kSlots][128]
   static constexpr uint32_t kColMul = kPerm + kSlots * kRows * 4;   // float [kSlots][128]
   static constexpr uint32_t kBk = kColMul + kSlots * kRows * 4;     // int32 [kSlots][128] (bucket mask)
-  static constexpr uint32_t kBar = kBk + kSlots * kRows * 4;
+  // int32 [kSlots][128][8]: every round's bucket of each row (union correction)
+  static constexpr uint32_t kBkAll = kBk + kSlots * kRows * 4;
+  static constexpr uint32_t kLog2 = kBkAll + kSlots * kRows * kUnionRounds * 4;  // float [16]: log2(n)
+  static constexpr uint32_t kBar = kLog2 + 16 * 4;
   // full[3] empty[3] cm_full[3] s_full[2] p_ready[2] o_full[2] buf_empty[2] done
   static constexpr int kNumBars = 18;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;   // tmem base, abort flag
@@ -105,6 +115,15 @@ struct Params {
   const uint8_t* v;
   int out_v8;            // output rows 32-byte aligned: 32-byte stores
 };
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 // Warp-uniform bounded wait: every lane acquires the phase itself, lane 0
 // decides on abort / timeout so that the warp leaves together.
@@ -273,7 +292,7 @@ __device__ __forceinline__ void fill_positions(const Params& p, const Fill& f, i
 // and its 16-byte piece c at ((c ^ (r % 8)) * 16), the 128-byte swizzle the
 // UMMA descriptors expect.  Every producer lane then arrives on `full_bar`
 // when its copies have landed.
-template <int D, bool BUCKET>
+template <int D, bool BUCKET, bool UNION>
 __device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, uint64_t* full_bar, int slot,
                                               const Fill& f, int pw, const int (&pos)[2]) {
   using Lay = Layout<D>;
@@ -292,6 +311,17 @@ __device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, ui
       perm_s[i] = pos[k];
       if (BUCKET)  // the row's bucket lands with the row (same cp.async group, same barrier)
         tc::cp_async4(tc::smem_u32(smem + Lay::kBk) + (slot * kRows + i) * 4, p.buckets + f.seg * p.L + pos[k]);
+      if (UNION) {  // the row's bucket in every round of its (b, h) slice (-2: no such round)
+        const long long seg0 = (f.seg / p.n_rounds) * p.n_rounds;
+        const uint32_t dst = tc::smem_u32(smem + Lay::kBkAll) + ((slot * kRows + i) * kUnionRounds) * 4;
+#pragma unroll
+        for (int rr = 0; rr < kUnionRounds; ++rr) {
+          if (rr < p.n_rounds)
+            tc::cp_async4(dst + rr * 4, p.buckets + (seg0 + rr) * p.L + pos[k]);
+          else
+            reinterpret_cast<int32_t*>(smem + Lay::kBkAll)[(slot * kRows + i) * kUnionRounds + rr] = -2;
+        }
+      }
       grow[k] = p.sorted_input ? f.seg * p.L + chunk * kC + (i & 63) : (f.seg / p.n_rounds) * p.L + pos[k];
     }
     const uint32_t qk_dst = tc::smem_u32(smem + Lay::kQK + slot * Lay::kSlotBytes);
@@ -330,12 +360,24 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
   return colscale / fmaxf(sqrtf(ss), 1e-12f);
 }
 
+// The union correction of one key: log2 of the number of rounds whose buckets
+// of query and key agree (`ku`: the key's kUnionRounds buckets, `qu`: the
+// query's, -1 for rounds that do not exist; `lg2`: log2 of 0..8, 0 at 0).
+__device__ __forceinline__ float union_log2(const int32_t* ku, const int (&qu)[kUnionRounds], const float* lg2) {
+  const int4 a = reinterpret_cast<const int4*>(ku)[0], b = reinterpret_cast<const int4*>(ku)[1];
+  const int n = (a.x == qu[0]) + (a.y == qu[1]) + (a.z == qu[2]) + (a.w == qu[3]) + (b.x == qu[4]) +
+                (b.y == qu[5]) + (b.z == qu[6]) + (b.w == qu[7]);
+  return lg2[n];
+}
+
 template <int D, int MASK>
 __device__ __forceinline__ void softmax_group(uint32_t sbuf, uint32_t pcol, int g, const uint32_t (&cur)[32],
                                               const float* cm, const int32_t* kp, const int32_t* kb, bool dead,
                                               bool self_grp, int lane, float m, float& l, int qpos, int qb,
-                                              int& others) {
+                                              int& others, const int32_t* ku, const int (&qu)[kUnionRounds],
+                                              const float* lg2) {
   constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
+  constexpr bool UNION = (MASK & kMaskUnion) != 0;
   // key multipliers (and positions, buckets) as 16-byte loads: each group's 32 values start on a
   // 16-byte boundary
   const float4* cm4 = reinterpret_cast<const float4*>(cm);
@@ -368,6 +410,10 @@ __device__ __forceinline__ void softmax_group(uint32_t sbuf, uint32_t pcol, int 
       }
       if (!dead) others += (int)c0 + (int)c1;
     }
+    if (UNION) {  // lower each logit by log2 of the rounds the pair shares
+      v0 -= union_log2(ku + e * kUnionRounds, qu, lg2);
+      v1 -= union_log2(ku + (e + 1) * kUnionRounds, qu, lg2);
+    }
     if (self_grp) {
       if (e == lane) v0 = -INFINITY;
       if (e + 1 == lane) v1 = -INFINITY;
@@ -393,7 +439,8 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
                                              const float* cm_hi, int g_first, int g_self, int lane, int self_mask,
                                              float m, float& l, const int32_t* kp_lo, const int32_t* kp_hi,
                                              int qpos, const int32_t* kb_lo, const int32_t* kb_hi, int qb,
-                                             int& others) {
+                                             int& others, const int32_t* ku_lo, const int32_t* ku_hi,
+                                             const int (&qu)[kUnionRounds], const float* lg2) {
   uint32_t ra[32], rb[32];
   tc::tmem_ld32(sbuf + scol, ra);
   tc::tmem_wait_ld_regs(ra);
@@ -402,14 +449,16 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
     const float* cm = h ? cm_hi : cm_lo;
     const int32_t* kp = h ? kp_hi : kp_lo;
     const int32_t* kb = h ? kb_hi : kb_lo;
+    const int32_t* ku = h ? ku_hi : ku_lo;
     const bool dead = 2 * h < g_first;  // g_first is 0 or 2: both groups of the first half
     tc::tmem_ld32(sbuf + scol + 64 * h + 32, rb);
     softmax_group<D, MASK>(sbuf, pcol, 2 * h, ra, cm, kp, kb, dead, self_mask && 2 * h == g_self, lane, m, l,
-                           qpos, qb, others);
+                           qpos, qb, others, ku, qu, lg2);
     tc::tmem_wait_ld_regs(rb);
     if (h == 0) tc::tmem_ld32(sbuf + scol + 64, ra);
     softmax_group<D, MASK>(sbuf, pcol, 2 * h + 1, rb, cm + 32, kp + 32, kb + 32, dead,
-                           self_mask && 2 * h + 1 == g_self, lane, m, l, qpos, qb, others);
+                           self_mask && 2 * h + 1 == g_self, lane, m, l, qpos, qb, others,
+                           ku + 32 * kUnionRounds, qu, lg2);
     if (h == 0) tc::tmem_wait_ld_regs(ra);
   }
 }
@@ -417,12 +466,14 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
 // Rows with no admissible key but themselves (causal: no earlier key; bucket:
 // alone in their bucket inside the window) see only themselves: their P becomes
 // one-hot at the own key (bf16 1.0 at element `lane` of the self group) and
-// their weight sum 1 (the shift m is their own logit).  The whole warp rewrites
-// the self group, the other rows with the words they already had (read back
-// from TMEM).  `others` counts self too when only the bucket mask is on.
+// their weight sum 1 (the shift m is their own logit; under the union
+// correction the self pair shares every round, so its weight is 1 / n_rounds).
+// The whole warp rewrites the self group, the other rows with the words they
+// already had (read back from TMEM).  `others` counts self too when only the
+// bucket mask is on.
 template <int MASK>
 __device__ __forceinline__ void self_only_fixup(uint32_t sbuf, uint32_t pcol, int g_self, int lane, int others,
-                                                float& l) {
+                                                float& l, float self_weight) {
   const bool only = (MASK & kMaskCausal) ? others == 0 : others <= 1;
   if (!__any_sync(0xffffffffu, only)) return;
   uint32_t w16[16];
@@ -432,7 +483,7 @@ __device__ __forceinline__ void self_only_fixup(uint32_t sbuf, uint32_t pcol, in
   for (int k = 0; k < 16; ++k)
     if (only) w16[k] = k == (lane >> 1) ? ((lane & 1) ? 0x3F800000u : 0x00003F80u) : 0u;
   tc::tmem_st16(sbuf + pcol + 16 * g_self, w16);
-  if (only) l = 1.f;
+  if (only) l = self_weight;
 }
 
 // Exact maximum of a row's scaled logits (self excluded while it has other keys;
@@ -441,8 +492,11 @@ template <int MASK>
 __device__ __noinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const float* cm_lo, const float* cm_hi,
                                                int g_first, int g_self, int lane, int self_mask,
                                                const int32_t* kp_lo, const int32_t* kp_hi, int qpos,
-                                               const int32_t* kb_lo, const int32_t* kb_hi, int qb) {
+                                               const int32_t* kb_lo, const int32_t* kb_hi, int qb,
+                                               const int32_t* ku_lo, const int32_t* ku_hi,
+                                               const int (&qu)[kUnionRounds], const float* lg2) {
   constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
+  constexpr bool UNION = (MASK & kMaskUnion) != 0;
   float m = -INFINITY;
 #pragma unroll 1
   for (int g = 0; g < 4; ++g) {
@@ -453,9 +507,11 @@ __device__ __noinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const 
     const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
     const int32_t* kp = g < 2 ? kp_lo + 32 * g : kp_hi + 32 * (g - 2);
     const int32_t* kb = g < 2 ? kb_lo + 32 * g : kb_hi + 32 * (g - 2);
+    const int32_t* ku = g < 2 ? ku_lo + 32 * g * kUnionRounds : ku_hi + 32 * (g - 2) * kUnionRounds;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       float v = __uint_as_float(raw[e]) * cm[e];
+      if (UNION) v -= union_log2(ku + e * kUnionRounds, qu, lg2);
       if (CAUSAL && kp[e] > qpos) v = -INFINITY;
       if (BUCKET && kb[e] != qb) v = -INFINITY;
       if (g == g_self && self_mask && e == lane) v = -INFINITY;
@@ -593,6 +649,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
   {
     uint32_t* ones = reinterpret_cast<uint32_t*>(smem + Lay::kOnes);
     for (int i = threadIdx.x; i < 16 * 128 / 4; i += kThreads) ones[i] = 0x3F803F80u;  // two bf16 1.0
+    if (threadIdx.x < 16)  // log2 of a shared-round count (0: unused, the key is masked)
+      reinterpret_cast<float*>(smem + Lay::kLog2)[threadIdx.x] = threadIdx.x > 1 ? log2f((float)threadIdx.x) : 0.f;
     tc::fence_proxy_async_smem();
   }
   if (warp == 2) tc::tmem_alloc(tmem_holder, kTmemCols);
@@ -601,128 +659,135 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp < 2) {
-    // ------------------------------------------------------------ producers
-    // Fills F (gathered now), F+1 (positions loaded), F+2 (rows warmed in L2 with
-    // per-line prefetches now; positions loaded one iteration earlier), F+3
-    // (positions loading).  The gathers are latency-bound and shared memory holds
-    // one fill in flight, so rows that reach L2 early shorten the next gathers.
-    const int pw = warp;
-    uint32_t f = 0;
-    FillIter it0, it1, it2, it3;
-    it0.init(p);
-    it1 = it0;
-    if (it1.valid) it1.advance(p);
-    it2 = it1;
-    if (it2.valid) it2.advance(p);
-    it3 = it2;
-    if (it3.valid) it3.advance(p);
-    int pos0[2] = {0, 0}, pos1[2] = {0, 0}, pos2[2] = {0, 0};
-    if (it0.valid) fill_positions(p, it0.get(p), pw, pos0);
-    if (it1.valid) fill_positions(p, it1.get(p), pw, pos1);
-    if (it2.valid) fill_positions(p, it2.get(p), pw, pos2);
-    while (it0.valid) {
-      int pos3[2] = {0, 0};
-      if (it3.valid) fill_positions(p, it3.get(p), pw, pos3);
-      if (it2.valid) {
-        const Fill pf = it2.get(p);
+  if (warp < 4) {
+    // warpgroup 0 (producers and UMMA issuers) hands registers to the softmax
+    // warpgroups; every warp of a warpgroup executes the same setmaxnreg
+    setmaxnreg_dec<kLowRegs>();
+    if (warp < 2) {
+      // ------------------------------------------------------------ producers
+      // Fills F (gathered now), F+1 (positions loaded), F+2 (rows warmed in L2 with
+      // per-line prefetches now; positions loaded one iteration earlier), F+3
+      // (positions loading).  The gathers are latency-bound and shared memory holds
+      // one fill in flight, so rows that reach L2 early shorten the next gathers.
+      const int pw = warp;
+      uint32_t f = 0;
+      FillIter it0, it1, it2, it3;
+      it0.init(p);
+      it1 = it0;
+      if (it1.valid) it1.advance(p);
+      it2 = it1;
+      if (it2.valid) it2.advance(p);
+      it3 = it2;
+      if (it3.valid) it3.advance(p);
+      int pos0[2] = {0, 0}, pos1[2] = {0, 0}, pos2[2] = {0, 0};
+      if (it0.valid) fill_positions(p, it0.get(p), pw, pos0);
+      if (it1.valid) fill_positions(p, it1.get(p), pw, pos1);
+      if (it2.valid) fill_positions(p, it2.get(p), pw, pos2);
+      while (it0.valid) {
+        int pos3[2] = {0, 0};
+        if (it3.valid) fill_positions(p, it3.get(p), pw, pos3);
+        if (it2.valid) {
+          const Fill pf = it2.get(p);
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int i = 64 * pw + 32 * k + lane;
-          if (i >= pf.row0 && i < pf.row0 + pf.nrows) {
-            const int chunk = (i - pf.row0) < 64 ? pf.cA : pf.cB;
-            const long long g = p.sorted_input ? pf.seg * p.L + chunk * kC + (i & 63)
-                                               : (pf.seg / p.n_rounds) * p.L + pos2[k];
+          for (int k = 0; k < 2; ++k) {
+            const int i = 64 * pw + 32 * k + lane;
+            if (i >= pf.row0 && i < pf.row0 + pf.nrows) {
+              const int chunk = (i - pf.row0) < 64 ? pf.cA : pf.cB;
+              const long long g = p.sorted_input ? pf.seg * p.L + chunk * kC + (i & 63)
+                                                 : (pf.seg / p.n_rounds) * p.L + pos2[k];
 #pragma unroll
-            for (int ln = 0; ln < D * 2; ln += 128) {
-              tc::prefetch_l2_line(p.qk + g * D * 2 + ln);
-              tc::prefetch_l2_line(p.v + g * D * 2 + ln);
+              for (int ln = 0; ln < D * 2; ln += 128) {
+                tc::prefetch_l2_line(p.qk + g * D * 2 + ln);
+                tc::prefetch_l2_line(p.v + g * D * 2 + ln);
+              }
             }
           }
         }
-      }
-      const Fill cur = it0.get(p);
-      const int slot = f % kSlots;
-      if (!warp_wait(&empty[slot], ((f / kSlots) & 1) ^ 1, abort_flag)) break;
-      producer_fill<D, (MASK & kMaskBucket) != 0>(p, smem, &full[slot], slot, cur, pw, pos0);
-      ++f;
-      it0 = it1;
-      it1 = it2;
-      it2 = it3;
-      if (it3.valid) it3.advance(p);
+        const Fill cur = it0.get(p);
+        const int slot = f % kSlots;
+        if (!warp_wait(&empty[slot], ((f / kSlots) & 1) ^ 1, abort_flag)) break;
+        producer_fill<D, (MASK & kMaskBucket) != 0, (MASK & kMaskUnion) != 0>(p, smem, &full[slot], slot, cur, pw,
+                                                                                 pos0);
+        ++f;
+        it0 = it1;
+        it1 = it2;
+        it2 = it3;
+        if (it3.valid) it3.advance(p);
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        pos0[k] = pos1[k];
-        pos1[k] = pos2[k];
-        pos2[k] = pos3[k];
-      }
-    }
-    // never leave with copies in flight
-    asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ UMMA issuers
-    // warp 2 lane 0 issues the S UMMAs, warp 3 lane 0 the PV UMMAs; each waits
-    // on one barrier at a time.  tcgen05.commit tracks the issuing thread's own
-    // UMMAs.
-    if (lane == 0) {
-      const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK);
-      const uint32_t v0 = tc::smem_u32(smem + Lay::kV);
-      StepIter it;
-      it.init(p);
-      if (warp == 2) {
-        const uint32_t id_prev = tc::idesc_bf16_f32(128, 64, 0, 0);
-        const uint32_t id_pair = tc::idesc_bf16_f32(128, 128, 0, 0);
-        while (it.valid) {
-          const uint32_t fp = it.f - 1, fc = it.f;
-          if (!issuer_wait(&full[fp % kSlots], (fp / kSlots) & 1, abort_flag) ||
-              !issuer_wait(&full[fc % kSlots], (fc / kSlots) & 1, abort_flag) ||
-              !issuer_wait(&buf_empty[it.t & 1], ((it.t >> 1) & 1) ^ 1, abort_flag))
-            break;
-          tc::tc_fence_after();
-          const uint32_t sbuf = tmem + (it.t & 1) * kBufCols;
-          const uint32_t qk_c = qk0 + (fc % kSlots) * Lay::kSlotBytes;
-          const uint32_t qk_p = qk0 + (fp % kSlots) * Lay::kSlotBytes + 64 * 128;  // rows 64..127
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * Lay::kHalfBytes + (kk & 3) * 32;
-            const uint64_t a = tc::sdesc_sw128(qk_c + koff, 16, 1024);
-            const uint64_t bp = tc::sdesc_sw128(qk_p + koff, 16, 1024);
-            tc::umma_ss(sbuf, a, bp, id_prev, kk > 0);
-            tc::umma_ss(sbuf + 64, a, a, id_pair, kk > 0);
-          }
-          tc::umma_commit(&s_full[it.t & 1]);
-          it.advance(p);
-        }
-      } else {
-        const uint32_t id_pv = tc::idesc_bf16_f32(128, D, 0, 1);
-        const uint32_t id_lr = tc::idesc_bf16_f32(128, 16, 0, 1);
-        const uint64_t ones_desc = tc::sdesc_sw128(tc::smem_u32(smem + Lay::kOnes), Lay::kHalfBytes, 1024);
-        while (it.valid) {
-          if (!issuer_wait(&p_ready[it.t & 1], (it.t >> 1) & 1, abort_flag)) break;
-          tc::tc_fence_after();
-          const uint32_t sbuf = tmem + (it.t & 1) * kBufCols;
-          const uint32_t sp = (it.f - 1) % kSlots, sc = it.f % kSlots;
-#pragma unroll
-          for (int kk = 0; kk < 12; ++kk) {
-            const uint32_t vrow = kk < 4 ? v0 + sp * Lay::kSlotBytes + (64 + 16 * kk) * 128
-                                         : v0 + sc * Lay::kSlotBytes + (16 * (kk - 4)) * 128;
-            const uint64_t b = tc::sdesc_sw128(vrow, Lay::kHalfBytes, 1024);
-            tc::umma_ts(sbuf + kOOff, sbuf + kk * 8, b, id_pv, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < 12; ++kk)  // every 16-key step reads the same 16 rows of ones
-            tc::umma_ts(sbuf + lr_col<D>(), sbuf + kk * 8, ones_desc, id_lr, kk > 0);
-          tc::umma_commit(&o_full[it.t & 1]);
-          tc::umma_commit(&empty[sp]);
-          if (it.last_of_unit()) tc::umma_commit(&empty[sc]);
-          it.advance(p);
+        for (int k = 0; k < 2; ++k) {
+          pos0[k] = pos1[k];
+          pos1[k] = pos2[k];
+          pos2[k] = pos3[k];
         }
       }
-      tc::umma_commit(done_bar);
-      drain_wait(done_bar, 0);
+      // never leave with copies in flight
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else {
+      // ------------------------------------------------------------ UMMA issuers
+      // warp 2 lane 0 issues the S UMMAs, warp 3 lane 0 the PV UMMAs; each waits
+      // on one barrier at a time.  tcgen05.commit tracks the issuing thread's own
+      // UMMAs.
+      if (lane == 0) {
+        const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK);
+        const uint32_t v0 = tc::smem_u32(smem + Lay::kV);
+        StepIter it;
+        it.init(p);
+        if (warp == 2) {
+          const uint32_t id_prev = tc::idesc_bf16_f32(128, 64, 0, 0);
+          const uint32_t id_pair = tc::idesc_bf16_f32(128, 128, 0, 0);
+          while (it.valid) {
+            const uint32_t fp = it.f - 1, fc = it.f;
+            if (!issuer_wait(&full[fp % kSlots], (fp / kSlots) & 1, abort_flag) ||
+                !issuer_wait(&full[fc % kSlots], (fc / kSlots) & 1, abort_flag) ||
+                !issuer_wait(&buf_empty[it.t & 1], ((it.t >> 1) & 1) ^ 1, abort_flag))
+              break;
+            tc::tc_fence_after();
+            const uint32_t sbuf = tmem + (it.t & 1) * kBufCols;
+            const uint32_t qk_c = qk0 + (fc % kSlots) * Lay::kSlotBytes;
+            const uint32_t qk_p = qk0 + (fp % kSlots) * Lay::kSlotBytes + 64 * 128;  // rows 64..127
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t koff = (kk >> 2) * Lay::kHalfBytes + (kk & 3) * 32;
+              const uint64_t a = tc::sdesc_sw128(qk_c + koff, 16, 1024);
+              const uint64_t bp = tc::sdesc_sw128(qk_p + koff, 16, 1024);
+              tc::umma_ss(sbuf, a, bp, id_prev, kk > 0);
+              tc::umma_ss(sbuf + 64, a, a, id_pair, kk > 0);
+            }
+            tc::umma_commit(&s_full[it.t & 1]);
+            it.advance(p);
+          }
+        } else {
+          const uint32_t id_pv = tc::idesc_bf16_f32(128, D, 0, 1);
+          const uint32_t id_lr = tc::idesc_bf16_f32(128, 16, 0, 1);
+          const uint64_t ones_desc = tc::sdesc_sw128(tc::smem_u32(smem + Lay::kOnes), Lay::kHalfBytes, 1024);
+          while (it.valid) {
+            if (!issuer_wait(&p_ready[it.t & 1], (it.t >> 1) & 1, abort_flag)) break;
+            tc::tc_fence_after();
+            const uint32_t sbuf = tmem + (it.t & 1) * kBufCols;
+            const uint32_t sp = (it.f - 1) % kSlots, sc = it.f % kSlots;
+#pragma unroll
+            for (int kk = 0; kk < 12; ++kk) {
+              const uint32_t vrow = kk < 4 ? v0 + sp * Lay::kSlotBytes + (64 + 16 * kk) * 128
+                                           : v0 + sc * Lay::kSlotBytes + (16 * (kk - 4)) * 128;
+              const uint64_t b = tc::sdesc_sw128(vrow, Lay::kHalfBytes, 1024);
+              tc::umma_ts(sbuf + kOOff, sbuf + kk * 8, b, id_pv, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 12; ++kk)  // every 16-key step reads the same 16 rows of ones
+              tc::umma_ts(sbuf + lr_col<D>(), sbuf + kk * 8, ones_desc, id_lr, kk > 0);
+            tc::umma_commit(&o_full[it.t & 1]);
+            tc::umma_commit(&empty[sp]);
+            if (it.last_of_unit()) tc::umma_commit(&empty[sc]);
+            it.advance(p);
+          }
+        }
+        tc::umma_commit(done_bar);
+        drain_wait(done_bar, 0);
+      }
+      __syncwarp();
     }
-    __syncwarp();
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc<kSoftRegs>();
     // ------------------------------------------------------------ softmax + epilogue
     const int wg = (warp - 4) >> 2;      // 0: even steps, 1: odd steps
     const int q = warp & 3;              // TMEM lane quarter of this warp
@@ -778,6 +843,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       const int32_t* kb_lo = low ? bk_s + sp * kRows + 64 : bk_s + sc * kRows;      // their buckets
       const int32_t* kb_hi = low ? bk_s + sc * kRows : bk_s + sc * kRows + 64;
       const int qb = (MASK & kMaskBucket) ? bk_s[sc * kRows + r] : 0;
+      // union correction: every round's bucket of the keys (per fill row) and of the query
+      const int32_t* bku = reinterpret_cast<const int32_t*>(smem + Lay::kBkAll);
+      const int32_t* ku_lo = low ? bku + (sp * kRows + 64) * kUnionRounds : bku + (sc * kRows) * kUnionRounds;
+      const int32_t* ku_hi = low ? bku + (sc * kRows) * kUnionRounds : bku + (sc * kRows + 64) * kUnionRounds;
+      const float* lg2 = reinterpret_cast<const float*>(smem + Lay::kLog2);
+      int qu[kUnionRounds];
+#pragma unroll
+      for (int rr = 0; rr < kUnionRounds; ++rr)
+        qu[rr] = ((MASK & kMaskUnion) && rr < p.n_rounds) ? bku[(sc * kRows + r) * kUnionRounds + rr] : -1;
+      const float self_weight = (MASK & kMaskUnion) ? 1.f / (float)p.n_rounds : 1.f;
       int others = 0;
       const int g_first = (low && it.j == 0) ? 2 : 0;  // chunk 0 has no previous chunk
       // shift: ||q|| * scale * log2(e) bounds every logit of the row (log2 domain)
@@ -790,15 +865,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
         l = 0.f;
         others = 0;
         softmax_pass<D, MASK>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, kp_lo,
-                              kp_hi, pos, kb_lo, kb_hi, qb, others);
-        if (MASKED) self_only_fixup<MASK>(sbuf, pcol, g_self, lane, others, l);
+                              kp_hi, pos, kb_lo, kb_hi, qb, others, ku_lo, ku_hi, qu, lg2);
+        if (MASKED) self_only_fixup<MASK>(sbuf, pcol, g_self, lane, others, l, self_weight);
         if (attempt > 0 || !__any_sync(0xffffffffu, !(l > 1e-30f))) break;
         // the bound was too loose for some row of the warp (long query rows): S is
         // rebuilt in TMEM from the rows in shared memory (P has overwritten part of
         // it) and the warp's rows are redone with their exact maxima
         restore_s<D>(smem, sbuf, scol, sp, sc, r, low);
         m = exact_row_max<MASK>(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, kp_lo, kp_hi, pos,
-                                kb_lo, kb_hi, qb);
+                                kb_lo, kb_hi, qb, ku_lo, ku_hi, qu, lg2);
         if (MASKED && m == -INFINITY) m = m_cs;  // self-only row: its own logit is the shift
       }
       {

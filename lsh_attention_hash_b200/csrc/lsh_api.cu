@@ -431,14 +431,17 @@ lsh_status lsh_chunk_attend(const void* qk, const void* v, int dtype, int B, int
 
   const DevInfo di = dev_info();
   if (dtype == LSH_BF16 && chunk == lsh::att_tc::kC && (D == 64 || D == 128) && di.major == 10 &&
-      !union_count) {
+      (!union_count || n_rounds <= lsh::att_tc::kUnionRounds)) {
     using lsh::att_tc::kMaskBucket;
     using lsh::att_tc::kMaskCausal;
+    using lsh::att_tc::kMaskUnion;
 #define LSH_ATT_TC_M(DD, TO, MM)                                                                            \
   return launch_attend_tc<DD, TO, MM>(qk, v, qk_sorted, v_sorted, perm, buckets, B, H, L, n_rounds, self_mask, \
                                       scale, out_rounds, lse, s, di.sms)
 #define LSH_ATT_TC(DD, TO)                                                              \
   do {                                                                                  \
+    if (union_count && causal) LSH_ATT_TC_M(DD, TO, kMaskCausal | kMaskBucket | kMaskUnion); \
+    if (union_count) LSH_ATT_TC_M(DD, TO, kMaskBucket | kMaskUnion);                    \
     if (causal && bucket_mask) LSH_ATT_TC_M(DD, TO, kMaskCausal | kMaskBucket);         \
     if (causal) LSH_ATT_TC_M(DD, TO, kMaskCausal);                                      \
     if (bucket_mask) LSH_ATT_TC_M(DD, TO, kMaskBucket);                                 \

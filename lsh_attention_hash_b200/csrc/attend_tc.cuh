@@ -1,4 +1,4 @@
-// Chunk attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+// Chunk attention on the 5th-generation tensor cores (tcgen05 + TMEM).
 //
 // twgreatdaily ICLR 2020 Reformer article, section "1 LSH Attention": after
 // the (bucket, position) sort the sequence is cut into chunks; a chunk's
@@ -20,8 +20,9 @@
 //                                accumulated behind P in the same TMEM buffer
 // and the rows go back to their original positions perm[s].
 //
-// Warp roles (384 threads, persistent CTAs, one per SM; 12 warps leave 168
-// registers per thread):
+// Warp roles (384 threads, persistent CTAs, one per SM, launched at 168
+// registers per thread; warpgroup 0 gives registers to the softmax warpgroups
+// with setmaxnreg, 104 / 192):
 //   warps 0-1  producers: read perm and gather the QK and V rows of each chunk
 //              with 16-byte cp.async copies (32 lanes generate addresses in
 //              parallel; many small TMA row gathers were issue-bound) straight
@@ -42,7 +43,14 @@
 // goes); a row whose sum would underflow under that shift has its S rebuilt
 // from shared memory and is redone with its exact maximum.  O is normalised by
 // the sum of the bf16 weights P holds, which 12 more UMMAs of P against a
-// tile of ones leave beside O.
+// tile of ones leave beside O.  The per-round outputs are stored with an L2
+// evict-first policy (written once, read once by the merge), so that the rows
+// the slice's other rounds gather again stay in L2.
+// Masks are compile-time bits: causal (key positions against the query's),
+// bucket (each row's bucket lands with the row), and with the bucket mask the
+// multi-round union correction (each row's bucket in every round, up to 8,
+// lands with the row; each admissible logit is lowered by log2 of the number of
+// rounds the pair shares).
 // TMEM: two step buffers of 256 columns (S: 192 fp32, P: first 96, O: 96..96+D,
 // row sums: 16 columns after O).
 // Every wait is bounded; a timeout unwinds the CTA cleanly.

@@ -9,9 +9,11 @@ chunk 64, 8 rounds).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-N > 1 runs under torchrun, one rank per GPU: every rank processes its own full
-workload (the (b, h) slices are independent, so there is no collective on the
-data path) -> weak scaling; the step time is the max over ranks.
+N > 1 runs under torchrun, one rank per GPU.  The (b, h) slices are
+independent, so there is no collective on the data path; the step time is the
+max over ranks.  --split replicas (default): every rank processes its own full
+workload -> weak scaling.  --split slices: the ranks split the B*H slices of one
+batch -> strong scaling (the 1M workload's 8 heads over up to 8 GPUs).
 
 --impl reference times the float64 CPU oracle (the only other implementation
 of the method here) on rank 0, one bounded sample of the same workload per
@@ -258,8 +260,9 @@ def run_reference(args, w, rank, world):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": dict(workload_config(w), **mask_config(args)),
+        "higher_is_better": True, "scaling": "strong" if args.split == "slices" else "weak",
+        "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": dict(workload_config(w, args.split, world), **mask_config(args)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -267,12 +270,14 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w):
+def workload_config(w, split="replicas", world=1):
+    parallelism = ("replicas (independent (b,h) slices per GPU)" if split == "replicas" else
+                   f"slices ({w.B * w.H} (b,h) slices of one batch split over {world} GPU(s))")
     return {
         "workload": f"{w.name}: B={w.B} H={w.H} L={w.L} D={w.D} {w.dtype} n_buckets={w.n_buckets} "
                     f"chunk={w.chunk} n_rounds={w.n_rounds}",
         "global_batch": w.B, "seq_len": w.L, "heads": w.H, "head_dim": w.D,
-        "parallelism": "replicas (independent (b,h) slices per GPU)",
+        "parallelism": parallelism,
         "l2": "inputs larger than L2 (QK+V = %.1f GiB per GPU), no flush" % (2 * w.tokens * w.D * (2 if w.dtype == 'bf16' else 4) / 2**30),
     }
 
@@ -281,6 +286,8 @@ def workload_config(w):
 # GPU arm
 # ---------------------------------------------------------------------------
 def run_ours(args, w, rank, world, local_rank):
+    import dataclasses
+
     import torch
     import torch.distributed as dist
 
@@ -290,7 +297,16 @@ def run_ours(args, w, rank, world, local_rank):
     masks = mask_options(args)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    qk_h, v_h, R_h = synth.make_inputs(w, seed=multi.rank_seed(0, rank), pin=True)
+    w_job = w  # the whole job's workload (tokens counted for the metric)
+    if args.split == "slices":
+        # this rank's contiguous share of the batch's (b, h) slices, run as one B = 1 batch
+        mine = multi.shard_slices(w.B, w.H, rank, world)
+        if not mine:
+            raise SystemExit(f"--split slices: {world} ranks for {w.B * w.H} slices")
+        qk_h, v_h, R_h = synth.make_shard_inputs(w, mine, seed=0, pin=True)
+        w = dataclasses.replace(w, B=1, H=len(mine))
+    else:
+        qk_h, v_h, R_h = synth.make_inputs(w, seed=multi.rank_seed(0, rank), pin=True)
     qk = qk_h.to(dev)
     v = v_h.to(dev)
     R = R_h.to(dev)
@@ -402,8 +418,9 @@ def run_ours(args, w, rank, world, local_rank):
     if rank != 0:
         return
     ms_step = elapsed_ms / args.steps
-    value = world * w.tokens / (ms_step / 1e3)
-    e2e_value = world * w.tokens / (e2e_ms / e2e_steps / 1e3)
+    job_tokens = w_job.tokens if args.split == "slices" else world * w.tokens
+    value = job_tokens / (ms_step / 1e3)
+    e2e_value = job_tokens / (e2e_ms / e2e_steps / 1e3)
     h2d = qk_h.numel() * qk_h.element_size() + v_h.numel() * v_h.element_size() + R_h.numel() * R_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
 
@@ -441,9 +458,10 @@ def run_ours(args, w, rank, world, local_rank):
         return f"{slices} (b,h) slice(s) of the workload ({tokens} tokens)"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if args.split == "slices" else "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": dict(workload_config(w), **mask_config(args)),
+        "config": dict(workload_config(w_job, args.split, world), **mask_config(args)),
         "roofline": {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": recorded_traffic(dominant, args.workload),
                      "peak_source": peak_src + (", sustained tensor peak" if bound == "tensor" else "")},
@@ -488,6 +506,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="64k")
+    ap.add_argument("--split", choices=["replicas", "slices"], default="replicas",
+                    help="N > 1: replicas (each rank its own batch) or slices (the ranks split one batch)")
     ap.add_argument("--causal", action="store_true",
                     help="causal window: keys after the query's position are masked")
     ap.add_argument("--bucket-mask", action="store_true",

@@ -128,3 +128,22 @@ def small_workload(name: str, B: int, H: int, L: int, D: int, dtype: str, n_buck
                    chunk: int, n_rounds: int, **kw) -> Workload:
     """A workload of arbitrary size for tests (same generator, any shape)."""
     return Workload(name, B, H, L, D, dtype, n_buckets, chunk, n_rounds, **kw)
+
+
+def make_shard_inputs(w: Workload, slices, seed: int = 0, threads: int = 8, pin: bool = False):
+    """(qk [1,n,L,D], v [1,n,L,D], R) of the given (b, h) slices of one batch (the strong-scaling
+    split of a batch over ranks: every slice is generated from its own (b, h) stream, so the shards
+    of all ranks together are exactly the batch of ``make_inputs``)."""
+    n = len(slices)
+    qk = torch.empty((1, n, w.L, w.D), dtype=w.torch_dtype, pin_memory=pin)
+    v = torch.empty_like(qk, pin_memory=pin)
+
+    def fill(i):
+        b, h = slices[i]
+        q_s, v_s = slice_inputs(w, b, h, seed)
+        qk[0, i].copy_(q_s)
+        v[0, i].copy_(v_s)
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(fill, range(n)))
+    return qk, v, projections(w, seed)

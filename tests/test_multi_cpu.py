@@ -100,6 +100,25 @@ def test_slice_shards_gathered_equal_one_process_run(world):
         assert np.array_equal(out[rank], want), f"rank {rank}"
 
 
+@pytest.mark.parametrize("world", [2, 3, 8])
+def test_shard_inputs_are_the_batch_slices(world):
+    """bench.py --split slices: the ranks' shard inputs, concatenated in rank order, are exactly the
+    batch that one process generates (same slices, same values), and R is the same on every rank."""
+    w = synth.small_workload("shard_inputs", 2, 4, 64, 16, "bf16", 8, 32, 2)
+    qk, v, R = synth.make_inputs(w, seed=0)
+    parts_qk, parts_v = [], []
+    for rank in range(world):
+        sl = multi.shard_slices(w.B, w.H, rank, world)
+        if not sl:
+            continue
+        q_r, v_r, R_r = synth.make_shard_inputs(w, sl, seed=0)
+        assert torch.equal(R_r, R)
+        parts_qk.append(q_r[0])
+        parts_v.append(v_r[0])
+    assert torch.equal(torch.cat(parts_qk), qk.reshape(w.B * w.H, w.L, w.D))
+    assert torch.equal(torch.cat(parts_v), v.reshape(w.B * w.H, w.L, w.D))
+
+
 def test_max_over_ranks_without_process_group_is_identity():
     assert multi.max_over_ranks([1.5, 2.0]) == [1.5, 2.0]
 

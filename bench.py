@@ -80,6 +80,13 @@ def backward_flops(w):
     return 10.0 * w.D * pairs
 
 
+def backward_on_tensor_cores(w, args):
+    """The library's tensor-core backward serves bf16, D 128, chunk 64, L % 128 == 0 and the plain
+    window (with or without the self mask); everything else runs on the CUDA cores."""
+    return (w.dtype == "bf16" and w.D == 128 and w.chunk == 64 and w.L % 128 == 0
+            and not args.causal and not args.bucket_mask and not args.union)
+
+
 def measured_sm_max_mhz(default=1965.0):
     """Maximum SM clock recorded with the measured peaks (the nominal 1965 MHz otherwise)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -485,17 +492,26 @@ def run_ours(args, w, rank, world, local_rank):
                                                 f"rounds, BLAS pools capped at one thread, {o_secs:.1f} s"}},
     }
     if args.backward:
-        sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        sm_mhz = measured_sm_max_mhz()
         b_ach = backward_flops(w) / (bwd_ms / bwd_steps / 1e3) / 1e12
-        b_peak = alu_peak_tflops(sms, sm_mhz)
+        if backward_on_tensor_cores(w, args):
+            b_peak, b_bound, b_unit = peaks["bf16_tflops"], "tensor", "TFLOP/s"
+            b_src = peak_src + ", bf16 tensor peak (the five products run as UMMAs)"
+            b_launches = (w.n_rounds + 1) * bwd_steps  # per-token terms, then one launch per round
+            b_note = ("lsh_chunk_attend_backward alone (tensor cores: one per-token pass, then one launch per "
+                      "round), inputs resident")
+        else:
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            sm_mhz = measured_sm_max_mhz()
+            b_peak, b_bound, b_unit = alu_peak_tflops(sms, sm_mhz), "alu", "TFLOP/s"
+            b_src = f"FP32 FMA on the CUDA cores: {sms} SMs x 128 lanes x 2 x {sm_mhz:.0f} MHz"
+            b_launches = w.n_rounds * bwd_steps
+            b_note = "lsh_chunk_attend_backward alone (CUDA-core kernels, one launch per round), inputs resident"
         line["backward"] = {
             "ms": bwd_ms / bwd_steps, "value": world * w.tokens / (bwd_ms / bwd_steps / 1e3), "unit": UNIT,
-            "steps": bwd_steps, "gpu_launches": w.n_rounds * bwd_steps,
-            "roofline": {"bound": "alu", "achieved": b_ach, "peak": b_peak, "unit": "TFLOP/s",
-                         "frac": b_ach / b_peak, "traffic": None,
-                         "peak_source": f"FP32 FMA on the CUDA cores: {sms} SMs x 128 lanes x 2 x {sm_mhz:.0f} MHz"},
-            "note": "lsh_chunk_attend_backward alone (CUDA-core kernels, one launch per round), inputs resident"}
+            "steps": bwd_steps, "gpu_launches": b_launches,
+            "roofline": {"bound": b_bound, "achieved": b_ach, "peak": b_peak, "unit": b_unit,
+                         "frac": b_ach / b_peak, "traffic": None, "peak_source": b_src},
+            "note": b_note}
     print(json.dumps(line), flush=True)
 
 

@@ -1,0 +1,754 @@
+// Backward of the chunk attention and the round merge on the 5th-generation
+// tensor cores (tcgen05 + TMEM).
+//
+// Training through LSH attention recomputes from the stored hash (twgreatdaily
+// ICLR 2020 Reformer article, section "1 LSH Attention"; Ultralytics glossary
+// "Reformer", "Atencao LSH"): perm stays fixed.  With the rounds merged by their
+// log-sum-exp, an admissible pair (i, j) of a round has the merged weight
+// p~_ij = exp(z_ij - LSE_i), z_ij = scale (x_i . x_j) / ||x_j||, and the
+// gradient of sum(dout * out) is
+//     dz_ij = p~_ij (dout_i . v_j - dout_i . out_i)
+//     dv_j += p~_ij dout_i
+//     dx_i += scale dz_ij x_j / ||x_j||                        (query role)
+//     dx_j += G_j - (x_j . G_j) x_j / ||x_j||^2,
+//             G_j = scale sum_i dz_ij x_i / ||x_j||            (key role through the
+//                                                              key normalisation)
+// With Z_ij = scale dz_ij / ||x_j|| both roles are plain products:
+// dQ = Z X (over the keys) and G = Z^T X (over the queries).
+//
+// Served case: bf16 rows and bf16 out / dout, D = 128, chunk 64, L a multiple
+// of 128, the plain window with or without the self mask.  One launch per round
+// (rounds in order: each adds into the fp32 gradients the previous ones left;
+// the first one stores).  A fill is two consecutive sorted chunks (2t, 2t+1),
+// 128 query rows; its key window is the three chunks 2t-1, 2t, 2t+1, taken one
+// 64-key block at a time.  Per block b:
+//   S_b  [128 x 64] = X_fill X_b^T      (TMEM, fp32)
+//   dP_b [128 x 64] = dO_fill V_b^T
+//   P~ = exp2(S s_j - LSE_i log2 e), Z = P~ (dP - Delta_i) scale / ||x_j||  (bf16,
+//        shared memory, written by the softmax warps; rows outside the block's
+//        window are never read)
+//   dK^T, dV^T of the block's 64 keys  [128 (D) x 64] += X_fill^T Z, dO_fill^T P~
+//   dQ^T of each query chunk that sees the block [128 x 64] += X_b^T Z^T
+// All gradients are kept transposed (TMEM lane = feature d, column = token), so
+// that a chunk's query-role and key-role sums land in the same columns: one
+// TMEM region per chunk holds H = dQ + G and the dv sums, in a ring of three
+// regions (chunk 2t+1 is finished by the next fill's first block).  The
+// epilogue warps take a finished region: x_j . H_j (a reduction over the 128
+// lanes) minus x_j . dQ_j (= sum_k Z_jk S_jk, summed by the softmax warps as
+// they go) gives x_j . G_j for the key-normalisation term; the rows are added
+// into dqk / dv at the tokens' original positions (32 lanes write 128
+// consecutive bytes of one row).
+//
+// Work units are runs of fills of one (b, h) segment.  A unit's first fill
+// takes the chunk before it from a leading fill, whose key-role sums belong to
+// the previous unit; a unit that ends before its segment does runs one more
+// half fill (the next unit's first query chunk against its last chunk, key
+// role only), so every token's rows have one writer per launch: no atomics,
+// and reruns are bit-identical.
+//
+// Warp roles (512 threads, one CTA per SM; launched at 128 registers, warpgroup
+// 0 gives 56 to the others with setmaxnreg: 72 / 144 / 144 / 152):
+//   warps 0-1   producers: 16-byte cp.async row gathers (X, V, dO) through perm
+//               into 128-byte-swizzled tiles, two fill slots for X and V, one
+//               dO tile, plus each row's LSE, Delta and length terms;
+//   warp 2      TMEM owner; its lane 0 issues every UMMA;
+//   warps 4-11  softmax: both warpgroups take every row (TMEM lane), keys
+//               0-31 / 32-63 of each block;
+//   warps 12-15 epilogue.
+// TMEM (512 columns): S (64) and dP (64) of the current block, then three
+// chunk regions of H (64) and dv (64).  Every wait is bounded; a timeout
+// unwinds the CTA cleanly.
+#pragma once
+
+#include "attend_tc.cuh"
+
+namespace lsh {
+namespace bwd_tc {
+
+constexpr int kC = 64;
+constexpr int kRows = 128;
+constexpr int kD = 128;
+constexpr int kThreads = 512;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSCol = 0, kPCol = 64, kRegCol0 = 128, kRegCols = 128;
+// registers per thread after the launch's 128: 72 (producers, issuer), 144 (softmax), 152 (epilogue);
+// 128 x (72 + 2 x 144 + 152) = 65536
+constexpr uint32_t kLowRegs = 72, kSoftRegs = 144, kEpiRegs = 152;
+
+struct Layout {
+  static constexpr uint32_t kHalf = kRows * 128;       // 128 rows x 64 bf16
+  static constexpr uint32_t kTile = 2 * kHalf;         // 128 rows x 128 bf16
+  static constexpr uint32_t kQK = 0;                   // [2] X rows of a fill slot
+  static constexpr uint32_t kV = 2 * kTile;            // [2] V rows
+  static constexpr uint32_t kDO = 4 * kTile;           // dO rows of the current fill
+  static constexpr uint32_t kP = 5 * kTile;            // P~ of one key block [128 x 64] bf16
+  static constexpr uint32_t kZ = kP + kHalf;           // Z of one key block
+  static constexpr uint32_t kAux = kZ + kHalf;         // float4 [2][128]: LSE log2 e, Delta, 1/||x||, kcorr
+  static constexpr uint32_t kKinv = kAux + 2 * kRows * 16;  // float [2][128]: 1/||x|| (vector loads)
+  static constexpr uint32_t kPerm = kKinv + 2 * kRows * 4;  // int32 [2][128]: original positions
+  static constexpr uint32_t kR = kPerm + 2 * kRows * 4;     // float [2][2][128]: x_i . dQ_i partials
+  static constexpr uint32_t kXH = kR + 2 * 2 * kRows * 4;   // float [4][32]: epilogue partial sums
+  static constexpr uint32_t kBar = kXH + 4 * 32 * 4;
+  // slot_full[2] slot_free[2] do_full do_free sp_full sp_free pz_full pz_free
+  // hv_done[3] hv_free[3] r_full[2] done
+  static constexpr int kNumBars = 19;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem base, abort flag
+  static constexpr uint32_t kBytes = kMisc + 16;
+  static constexpr uint32_t kSmem = kBytes + 1024;        // slack for 1024-byte alignment
+};
+
+struct Params {
+  const uint8_t* qk;      // bf16 [bh][L][128]
+  const uint8_t* v;
+  const uint8_t* dout;
+  const int32_t* perm;    // [bh][n_rounds][L]
+  const float4* aux;      // [bh][L]: LSE log2 e, dout . out, 1/max(||x||, 1e-12), (||x|| >= 1e-12) / ||x||^2
+  float* dqk;             // fp32 [bh][L][128]
+  float* dv;
+  int L;
+  int n_rounds;
+  int round;
+  int n_fills;            // L / 128
+  int run;                // fills per work unit
+  int units_per_seg;
+  long long n_units;
+  int self_mask;
+  float scale;
+  int accumulate;         // 0: the first round stores, 1: later rounds add
+};
+
+enum : int { kLead = 0, kFull = 1, kHalo = 2 };
+
+// Walks this CTA's fills: per unit a leading fill (chunk 2 t0 - 1 in rows
+// 64..127; nothing to copy at a segment start), the unit's fills t0 .. t1-1,
+// and, when the segment goes on, the half fill t1 (chunk 2 t1 in rows 0..63).
+struct FillIt {
+  long long u, bh;
+  int t, t0, t1, kind;
+  bool valid;
+  __device__ __forceinline__ void load_unit(const Params& p) {
+    valid = u < p.n_units;
+    if (!valid) return;
+    bh = u / p.units_per_seg;
+    t0 = (int)(u - bh * p.units_per_seg) * p.run;
+    t1 = min(t0 + p.run, p.n_fills);
+    t = t0;
+    kind = kLead;
+  }
+  __device__ __forceinline__ void init(const Params& p) {
+    u = blockIdx.x;
+    load_unit(p);
+  }
+  __device__ __forceinline__ void advance(const Params& p) {
+    if (kind == kLead) {
+      kind = kFull;
+    } else if (kind == kFull && t + 1 < t1) {
+      ++t;
+    } else if (kind == kFull && t1 < p.n_fills) {
+      kind = kHalo;
+      t = t1;
+    } else {
+      u += gridDim.x;
+      load_unit(p);
+    }
+  }
+  __device__ __forceinline__ bool has_prev() const { return t > 0; }
+  // the key-role sums of chunk 2t-1 belong to this unit (not to the previous one)
+  __device__ __forceinline__ bool owns_prev() const { return t > 0 && (kind == kHalo || t > t0); }
+};
+
+// Original positions of this producer lane's two rows of a fill (rows 64 pw + lane, +32).
+__device__ __forceinline__ bool fill_rows(const Params& p, const FillIt& f, int pw, int (&pos)[2]) {
+  const int lane = threadIdx.x & 31;
+  // rows present: lead -> 64..127 (if t0 > 0); full -> 0..127; halo -> 0..63
+  bool mine;
+  int chunk;
+  if (f.kind == kLead) {
+    mine = pw == 1 && f.t0 > 0;
+    chunk = 2 * f.t0 - 1;
+  } else if (f.kind == kHalo) {
+    mine = pw == 0;
+    chunk = 2 * f.t;
+  } else {
+    mine = true;
+    chunk = 2 * f.t + pw;
+  }
+  pos[0] = pos[1] = 0;
+  if (mine) {
+    const int32_t* pr = p.perm + (f.bh * p.n_rounds + p.round) * (long long)p.L + chunk * kC;
+    pos[0] = pr[lane];
+    pos[1] = pr[32 + lane];
+  }
+  return mine;
+}
+
+// Gathers 64 rows (local rows 64 pw ..) of each listed tensor into a 128-row
+// swizzled tile: 16-byte piece c of row r at (c / 8) * kHalf + r * 128 +
+// ((c % 8) ^ (r % 8)) * 16, the layout the UMMA descriptors expect.
+__device__ __forceinline__ void gather64(uint32_t dst, const uint8_t* src, long long rowbase, int pw,
+                                         const int (&pos)[2]) {
+  const int lane = threadIdx.x & 31;
+  const int c = lane & 15;
+#pragma unroll 4
+  for (int it = 0; it < 32; ++it) {
+    const int rl = 2 * it + (lane >> 4);  // row within the warp's 64
+    const int pr = __shfl_sync(0xffffffffu, rl < 32 ? pos[0] : pos[1], rl & 31);
+    const int r = 64 * pw + rl;
+    const uint32_t off = (c >> 3) * Layout::kHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+    tc::cp_async16(dst + off, src + ((rowbase + pr) * kD + c * 8) * 2);
+  }
+}
+
+// Barrier among `n` threads that also ANDs their predicates: a group decides together whether to go on.
+__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.b32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((int)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float (&o)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+  o[0] = __low2float(a);
+  o[1] = __high2float(a);
+  o[2] = __low2float(b);
+  o[3] = __high2float(b);
+}
+
+__device__ __forceinline__ uint32_t swz(int r, int c) {  // 16-byte piece c (0..7) of row r of a 64-wide tile
+  return (uint32_t)(r * 128 + (((c ^ r) & 7) << 4));
+}
+
+// lane l of the result holds the sum over the warp's lanes of v[l]
+__device__ __forceinline__ float transpose_reduce(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool hi = (lane & o) != 0;
+#pragma unroll
+    for (int e = 0; e < o; ++e) {
+      const float send = hi ? v[e] : v[e + o];
+      const float keep = hi ? v[e + o] : v[e];
+      v[e] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+// 16-feature step kk of a K-major operand (rows along M/N, 128 features, two 64-wide halves)
+__device__ __forceinline__ uint64_t kdesc(uint32_t row0, int kk) {
+  return tc::sdesc_sw128(row0 + (kk >> 2) * Layout::kHalf + (kk & 3) * 32, 16, 1024);
+}
+// MN-major operand whose K index is the tile row, starting at row r0 (a multiple of 16)
+__device__ __forceinline__ uint64_t mdesc(uint32_t tile, int r0) {
+  return tc::sdesc_sw128(tile + r0 * 128, Layout::kHalf, 1024);
+}
+// D (+)= A B^T over `steps` 16-wide K steps; A and B advance by a_step / b_step bytes per step
+__device__ __forceinline__ void mma_run(uint32_t d, uint64_t a, uint32_t a_step, uint64_t b, uint32_t b_step,
+                                        uint32_t idesc, int steps, bool acc) {
+#pragma unroll 1
+  for (int kk = 0; kk < steps; ++kk) {
+    tc::umma_ss(d, a + (uint64_t)((kk * a_step) >> 4), b + (uint64_t)((kk * b_step) >> 4), idesc, acc || kk > 0);
+  }
+}
+
+// S = X_fill X_b^T and dP = dO_fill V_b^T of one 64-key block (rows kx / kv of the X / V tiles)
+__device__ __forceinline__ void issue_sdp(uint32_t tmem, uint32_t xs, uint32_t do0, uint32_t kx, uint32_t kv,
+                                          uint64_t* sp_full) {
+  const uint32_t id_s = tc::idesc_bf16_f32(128, 64, 0, 0);  // both K-major
+#pragma unroll 1
+  for (int kk = 0; kk < kD / 16; ++kk) {
+    tc::umma_ss(tmem + kSCol, kdesc(xs, kk), kdesc(kx, kk), id_s, kk > 0);
+    tc::umma_ss(tmem + kPCol, kdesc(do0, kk), kdesc(kv, kk), id_s, kk > 0);
+  }
+  tc::umma_commit(sp_full);
+}
+
+// Lane 0 of warp 2: every UMMA of the CTA, in fill order (see the kernel's comment).
+__device__ __noinline__ void issuer(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag) {
+  using Lay = Layout;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+  uint64_t* slot_full = bars;
+  uint64_t* slot_free = bars + 2;
+  uint64_t* do_full = bars + 4;
+  uint64_t* do_free = bars + 5;
+  uint64_t* sp_full = bars + 6;
+  uint64_t* sp_free = bars + 7;
+  uint64_t* pz_full = bars + 8;
+  uint64_t* pz_free = bars + 9;
+  uint64_t* hv_done = bars + 10;
+  uint64_t* hv_free = bars + 13;
+  const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK), v0 = tc::smem_u32(smem + Lay::kV);
+  const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
+  const uint32_t pt = tc::smem_u32(smem + Lay::kP), zt = tc::smem_u32(smem + Lay::kZ);
+  const uint32_t id_kv = tc::idesc_bf16_f32(128, 64, 1, 1);  // dK^T, dV^T: both MN-major
+  const uint32_t id_q = tc::idesc_bf16_f32(128, 64, 1, 0);   // dQ^T: A MN-major, B K-major
+  constexpr uint32_t kRowStep = 16 * 128;                    // 16 tile rows
+  FillIt f;
+  f.init(p);
+  uint32_t F = 0, nd = 0, kb = 0, n = 0;  // fills, dO fills, blocks, owned chunks
+  bool ok = true;
+  while (ok && f.valid) {
+    const uint32_t s = F & 1, sp = (F + 1) & 1;
+    if (f.kind == kLead) {
+      ++F;
+      f.advance(p);
+      continue;
+    }
+    const bool full = f.kind == kFull, has_prev = f.has_prev(), owns_prev = f.owns_prev();
+    const bool first = full && f.t == f.t0, seg_end = full && f.t == p.n_fills - 1;
+    ok = att_tc::issuer_wait(&slot_full[s], (F >> 1) & 1, abort_flag) &&
+         (!has_prev || att_tc::issuer_wait(&slot_full[sp], ((F - 1) >> 1) & 1, abort_flag)) &&
+         att_tc::issuer_wait(do_full, nd & 1, abort_flag);
+    if (!ok) break;
+    tc::tc_fence_after();
+    const uint32_t xs = qk0 + s * Lay::kTile, vs = v0 + s * Lay::kTile;
+    const uint32_t xp = qk0 + sp * Lay::kTile, vp = v0 + sp * Lay::kTile;
+    if (first && !has_prev) tc::umma_commit(&slot_free[sp]);  // nothing of the leading fill is read
+    // blocks: 0 = chunk 2t-1 (rows 64.. of the previous slot), 1 = chunk 2t, 2 = chunk 2t+1
+    const int b_first = has_prev ? 0 : 1, b_last = full ? 2 : 0;
+    // regions: chunk 2t-1 -> owned chunk n-1, 2t -> n, 2t+1 -> n+1
+    const uint32_t rp = tmem + kRegCol0 + ((n + 2) % 3) * kRegCols;
+    const uint32_t r0 = tmem + kRegCol0 + (n % 3) * kRegCols;
+    const uint32_t r1 = tmem + kRegCol0 + ((n + 1) % 3) * kRegCols;
+    for (int b = b_first; b <= b_last; ++b) {
+      if (b == b_first) {
+        ok = att_tc::issuer_wait(sp_free, (kb & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        tc::tc_fence_after();
+      }
+      if (b == b_first)  // S and dP of the first block
+        issue_sdp(tmem, xs, do0, b == 0 ? xp + 64 * 128 : xs, b == 0 ? vp + 64 * 128 : vs, sp_full);
+      if (b < b_last) {  // the next block's S and dP while the softmax works on this one
+        ok = att_tc::issuer_wait(sp_free, kb & 1, abort_flag);
+        if (!ok) break;
+        tc::tc_fence_after();
+        const uint32_t ro = b + 1 == 2 ? 64 * 128 : 0;
+        issue_sdp(tmem, xs, do0, xs + ro, vs + ro, sp_full);
+      }
+      ok = att_tc::issuer_wait(pz_full, kb & 1, abort_flag);
+      if (!ok) break;
+      tc::tc_fence_after();
+      // first write into a chunk region waits until the epilogue has read the chunk three before it
+      if (b == 0) {
+        if (owns_prev) {  // key role of chunk 2t-1: queries of chunk 2t (rows 0..63)
+          mma_run(rp, mdesc(xs, 0), kRowStep, mdesc(zt, 0), kRowStep, id_kv, 4, true);
+          mma_run(rp + 64, mdesc(do0, 0), kRowStep, mdesc(pt, 0), kRowStep, id_kv, 4, true);
+        }
+        if (full) {
+          ok = att_tc::issuer_wait(&hv_free[n % 3], ((n / 3) & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          tc::tc_fence_after();
+          // dQ^T of chunk 2t from the keys of chunk 2t-1
+          mma_run(r0, mdesc(xp + 64 * 128, 0), kRowStep, kdesc(zt, 0), 32, id_q, 4, false);
+        }
+        tc::umma_commit(pz_free);
+        if (owns_prev) tc::umma_commit(&hv_done[(n + 2) % 3]);
+        if (first) tc::umma_commit(&slot_free[sp]);  // the leading fill's slot
+      } else if (b == 1) {
+        if (!has_prev) {
+          ok = att_tc::issuer_wait(&hv_free[n % 3], ((n / 3) & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          tc::tc_fence_after();
+        }
+        // key role of chunk 2t: all 128 queries
+        mma_run(r0, mdesc(xs, 0), kRowStep, mdesc(zt, 0), kRowStep, id_kv, 8, has_prev);
+        mma_run(r0 + 64, mdesc(do0, 0), kRowStep, mdesc(pt, 0), kRowStep, id_kv, 8, false);
+        // dQ^T of chunk 2t from the keys of chunk 2t
+        mma_run(r0, mdesc(xs, 0), kRowStep, kdesc(zt, 0), 32, id_q, 4, true);
+        ok = att_tc::issuer_wait(&hv_free[(n + 1) % 3], (((n + 1) / 3) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        tc::tc_fence_after();
+        // dQ^T of chunk 2t+1 from the keys of chunk 2t
+        mma_run(r1, mdesc(xs, 0), kRowStep, kdesc(zt + 64 * 128, 0), 32, id_q, 4, false);
+        tc::umma_commit(pz_free);
+        tc::umma_commit(&hv_done[n % 3]);
+      } else {
+        // key role of chunk 2t+1: queries of chunk 2t+1 (rows 64..127)
+        mma_run(r1, mdesc(xs, 64), kRowStep, mdesc(zt, 64), kRowStep, id_kv, 4, true);
+        mma_run(r1 + 64, mdesc(do0, 64), kRowStep, mdesc(pt, 64), kRowStep, id_kv, 4, false);
+        // dQ^T of chunk 2t+1 from the keys of chunk 2t+1
+        mma_run(r1, mdesc(xs, 64), kRowStep, kdesc(zt + 64 * 128, 0), 32, id_q, 4, true);
+        tc::umma_commit(pz_free);
+        if (seg_end) tc::umma_commit(&hv_done[(n + 1) % 3]);
+      }
+      ++kb;
+    }
+    if (!ok) break;
+    tc::umma_commit(do_free);
+    if (!full) tc::umma_commit(&slot_free[s]);  // the half fill's slot
+    if (full) n += 2;
+    ++nd;
+    ++F;
+    f.advance(p);
+  }
+  uint64_t* done_bar = bars + 18;
+  tc::umma_commit(done_bar);
+  att_tc::drain_wait(done_bar, 0);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params p) {
+  using Lay = Layout;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte-aligned base as an offset from the shared array itself (stays a shared-memory pointer)
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+  uint64_t* slot_full = bars;      // [2] a fill's rows and tables landed (64 producer lanes)
+  uint64_t* slot_free = bars + 2;  // [2] a fill slot may be refilled
+  uint64_t* do_full = bars + 4;    // dO rows landed (64)
+  uint64_t* do_free = bars + 5;    // dO tile read by the fill's last UMMA
+  uint64_t* sp_full = bars + 6;    // S and dP of a block computed
+  uint64_t* sp_free = bars + 7;    // S and dP loaded by the softmax (256)
+  uint64_t* pz_full = bars + 8;    // P~ and Z of a block written (256)
+  uint64_t* pz_free = bars + 9;    // P~ and Z read by the block's UMMAs
+  uint64_t* hv_done = bars + 10;   // [3] a chunk region finished
+  uint64_t* hv_free = bars + 13;   // [3] a chunk region read by the epilogue (128)
+  uint64_t* r_full = bars + 16;    // [2] x . dQ partials of a fill written (256)
+  uint64_t* done_bar = bars + 18;  // every UMMA retired
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
+  const float4* aux_s = reinterpret_cast<const float4*>(smem + Lay::kAux);
+  const float* kinv_s = reinterpret_cast<const float*>(smem + Lay::kKinv);
+  const int32_t* perm_s = reinterpret_cast<const int32_t*>(smem + Lay::kPerm);
+  float* r_s = reinterpret_cast<float*>(smem + Lay::kR);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&slot_full[i], 64);
+      tc::mbar_init(&slot_free[i], 1);
+      tc::mbar_init(&r_full[i], 256);
+    }
+    tc::mbar_init(do_full, 64);
+    tc::mbar_init(do_free, 1);
+    tc::mbar_init(sp_full, 1);
+    tc::mbar_init(sp_free, 256);
+    tc::mbar_init(pz_full, 256);
+    tc::mbar_init(pz_free, 1);
+    for (int i = 0; i < 3; ++i) {
+      tc::mbar_init(&hv_done[i], 1);
+      tc::mbar_init(&hv_free[i], 128);
+    }
+    tc::mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 2) tc::tmem_alloc(tmem_holder, kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const long long L = p.L;
+
+  if (warp < 4) {
+    att_tc::setmaxnreg_dec<kLowRegs>();
+    if (warp < 2) {
+      // ------------------------------------------------------------ producers
+      const int pw = warp;
+      const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK), v0 = tc::smem_u32(smem + Lay::kV);
+      const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
+      FillIt f;
+      f.init(p);
+      uint32_t F = 0, nd = 0;
+      while (f.valid) {
+        const int s = F & 1;
+        int pos[2];
+        const bool mine = fill_rows(p, f, pw, pos);
+        if (!att_tc::warp_wait(&slot_free[s], ((F >> 1) & 1) ^ 1, abort_flag)) break;
+        if (mine) {
+          const long long rb = f.bh * L;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int i = 64 * pw + 32 * k + lane;
+            const long long g = rb + pos[k];
+            tc::cp_async16(tc::smem_u32(smem + Lay::kAux) + (s * kRows + i) * 16, p.aux + g);
+            tc::cp_async4(tc::smem_u32(smem + Lay::kKinv) + (s * kRows + i) * 4,
+                          reinterpret_cast<const float*>(p.aux + g) + 2);
+            tc::cp_async4(tc::smem_u32(smem + Lay::kPerm) + (s * kRows + i) * 4,
+                          p.perm + (f.bh * p.n_rounds + p.round) * L +
+                              (f.kind == kLead ? 2 * f.t0 - 1 : 2 * f.t + (f.kind == kFull ? pw : 0)) * kC +
+                              32 * k + lane);
+          }
+          gather64(qk0 + s * Lay::kTile, p.qk, rb, pw, pos);
+          if (f.kind != kHalo) gather64(v0 + s * Lay::kTile, p.v, rb, pw, pos);
+        }
+        tc::cp_async_arrive(&slot_full[s]);
+        if (f.kind != kLead) {
+          if (!att_tc::warp_wait(do_free, (nd & 1) ^ 1, abort_flag)) break;
+          if (mine) gather64(do0, p.dout, f.bh * L, pw, pos);
+          tc::cp_async_arrive(do_full);
+          ++nd;
+        }
+        ++F;
+        f.advance(p);
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");  // never leave with copies in flight
+    } else if (warp == 2) {
+      // ------------------------------------------------------------ UMMA issuer
+      if (lane == 0) issuer(p, smem, tmem, abort_flag);
+      __syncwarp();
+    }
+  } else if (warp < 12) {
+    att_tc::setmaxnreg_inc<kSoftRegs>();
+    // ------------------------------------------------------------ softmax
+    const int wg = (warp - 4) >> 2;  // keys 32 wg .. 32 wg + 31 of each block
+    const int q = warp & 3;
+    const int i = 32 * q + lane;     // query row of the fill
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const float c2 = p.scale * 1.4426950408889634f;
+    uint8_t* pz_p = smem + Lay::kP;
+    uint8_t* pz_z = smem + Lay::kZ;
+    FillIt f;
+    f.init(p);
+    uint32_t F = 0, kb = 0, ff = 0;
+    bool ok = true;
+    while (f.valid) {
+      const uint32_t s = F & 1, sp = (F + 1) & 1;
+      if (f.kind == kLead) {
+        ++F;
+        f.advance(p);
+        continue;
+      }
+      const bool full = f.kind == kFull, has_prev = f.has_prev();
+      ok = att_tc::warp_wait(&slot_full[s], (F >> 1) & 1, abort_flag) &&
+           (!has_prev || att_tc::warp_wait(&slot_full[sp], ((F - 1) >> 1) & 1, abort_flag));
+      if (!ok) break;
+      // LSE log2 e and Delta of the row (a half fill has rows 0..63 only)
+      const float4 qa = (full || q < 2) ? aux_s[s * kRows + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      float r = 0.f;                            // x_i . dQ_i over this warp group's keys
+      int blocks[3], nb = 0;
+      if (has_prev) blocks[nb++] = 0;
+      if (full) {
+        blocks[nb++] = 1;
+        blocks[nb++] = 2;
+      }
+      for (int bi = 0; bi < nb; ++bi) {
+        const int b = blocks[bi];
+        const bool active = b == 1 || (b == 0 ? q < 2 : q >= 2);  // the block is in the row's window
+        ok = att_tc::warp_wait(sp_full, kb & 1, abort_flag);
+        if (!ok) break;
+        tc::tc_fence_after();
+        uint32_t sr[32], dr[32];
+        if (active) {
+          tc::tmem_ld32(tmem + lane_base + kSCol + 32 * wg, sr);
+          tc::tmem_ld32(tmem + lane_base + kPCol + 32 * wg, dr);
+          tc::tmem_wait_ld_regs(sr);
+          tc::tmem_wait_ld_regs(dr);
+        }
+        tc::tc_fence_before();
+        tc::mbar_arrive(sp_free);
+        uint32_t pw16[16], zw16[16];
+        if (active) {
+          // keys of the block: slot and first row
+          const float* kin = kinv_s + (b == 0 ? sp * kRows + 64 : s * kRows + (b == 2 ? 64 : 0)) + 32 * wg;
+          // own key: block 1 for rows 0..63, block 2 for rows 64..127, element `lane` of group wg == q % 2
+          const bool self_grp = p.self_mask && b != 0 && (q & 1) == wg && (b == 1) == (q < 2);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(kin + e);
+            const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+            float pe[4], ze[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float sv = __uint_as_float(sr[e + u]);
+              float pv = tc::ex2_approx(fmaf(sv, kv[u] * c2, -qa.x));
+              if (self_grp && e + u == lane) pv = 0.f;
+              const float zv = pv * (__uint_as_float(dr[e + u]) - qa.y) * (kv[u] * p.scale);
+              pe[u] = pv;
+              ze[u] = zv;
+            }
+            pw16[e / 2] = tc::pack_bf16x2(pe[0], pe[1]);
+            pw16[e / 2 + 1] = tc::pack_bf16x2(pe[2], pe[3]);
+            zw16[e / 2] = tc::pack_bf16x2(ze[0], ze[1]);
+            zw16[e / 2 + 1] = tc::pack_bf16x2(ze[2], ze[3]);
+            // x_i . dQ_i with the rounded Z the UMMA sees
+            const __nv_bfloat162 z01 = *reinterpret_cast<const __nv_bfloat162*>(&zw16[e / 2]);
+            const __nv_bfloat162 z23 = *reinterpret_cast<const __nv_bfloat162*>(&zw16[e / 2 + 1]);
+            r = fmaf(__low2float(z01), __uint_as_float(sr[e]), r);
+            r = fmaf(__high2float(z01), __uint_as_float(sr[e + 1]), r);
+            r = fmaf(__low2float(z23), __uint_as_float(sr[e + 2]), r);
+            r = fmaf(__high2float(z23), __uint_as_float(sr[e + 3]), r);
+          }
+        }
+        ok = att_tc::warp_wait(pz_free, (kb & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        if (active) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t off = swz(i, 4 * wg + c);
+            *reinterpret_cast<uint4*>(pz_p + off) =
+                make_uint4(pw16[4 * c], pw16[4 * c + 1], pw16[4 * c + 2], pw16[4 * c + 3]);
+            *reinterpret_cast<uint4*>(pz_z + off) =
+                make_uint4(zw16[4 * c], zw16[4 * c + 1], zw16[4 * c + 2], zw16[4 * c + 3]);
+          }
+          tc::fence_proxy_async_smem();
+        }
+        tc::mbar_arrive(pz_full);
+        ++kb;
+      }
+      if (!ok) break;
+      if (full) {
+        r_s[((ff & 1) * 2 + wg) * kRows + i] = r;
+        tc::mbar_arrive(&r_full[ff & 1]);
+        ++ff;
+      }
+      ++F;
+      f.advance(p);
+    }
+  } else {
+    att_tc::setmaxnreg_inc<kEpiRegs>();
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int d = 32 * q + lane;  // feature of this thread (TMEM lane)
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    float* xh = reinterpret_cast<float*>(smem + Lay::kXH);
+    FillIt f;
+    f.init(p);
+    uint32_t F = 0, n = 0, ff = 0;
+    bool ok = true;
+    // one finished chunk: region of owned chunk c, rows [row0, row0 + 64) of slot s, x . dQ partials rbuf
+    // every wait of the epilogue warps ends in one joint decision, so that their named barriers stay matched
+    auto epi_wait = [&](uint64_t* bar, uint32_t parity) {
+      return bar_and(1, 128, att_tc::warp_wait(bar, parity, abort_flag));
+    };
+    auto chunk_out = [&](uint32_t c, uint32_t s, int row0, uint32_t rbuf, long long bh) -> bool {
+      if (!epi_wait(&hv_done[c % 3], (c / 3) & 1)) return false;
+      tc::tc_fence_after();
+      const uint32_t reg = tmem + lane_base + kRegCol0 + (c % 3) * kRegCols;
+      const uint8_t* xt = smem + Lay::kQK + s * Lay::kTile + (d >> 6) * Lay::kHalf;
+      const int dc = (d & 63) >> 3, de = d & 7;
+      float* dq_bh = p.dqk + bh * L * kD + d;
+      float* dv_bh = p.dv + bh * L * kD + d;
+      const int32_t* pm = perm_s + s * kRows + row0;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t hr[32], vr[32];
+        tc::tmem_ld32(reg + 32 * h, hr);
+        tc::tmem_ld32(reg + 64 + 32 * h, vr);
+        tc::tmem_wait_ld_regs(hr);
+        tc::tmem_wait_ld_regs(vr);
+        if (h == 1) {
+          tc::tc_fence_before();
+          tc::mbar_arrive(&hv_free[c % 3]);
+        }
+        auto xval = [&](int e) {  // x of token row row0 + 32 h + e, feature d
+          return __bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16*>(xt + swz(row0 + 32 * h + e, dc) + 2 * de));
+        };
+        float part;
+        {
+          float pr[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pr[e] = xval(e) * __uint_as_float(hr[e]);
+          part = transpose_reduce(pr, lane);  // token row0 + 32 h + lane, this warp's 32 features
+        }
+        xh[q * 32 + lane] = part;
+        tc::named_bar_sync(1, 128);
+        const int row_l = row0 + 32 * h + lane;
+        const float tot = xh[lane] + xh[32 + lane] + xh[64 + lane] + xh[96 + lane];
+        const float rr = r_s[(rbuf * 2) * kRows + row_l] + r_s[(rbuf * 2 + 1) * kRows + row_l];
+        const float coef = (tot - rr) * aux_s[s * kRows + row_l].w;  // (x . G) (||x|| >= 1e-12) / ||x||^2
+        tc::named_bar_sync(1, 128);  // xh is reused by the next half
+#pragma unroll
+        for (int e0 = 0; e0 < 32; e0 += 8) {
+          float oq[8], ov[8];
+          int off[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            off[e] = pm[32 * h + e0 + e] * kD;
+            oq[e] = 0.f;
+            ov[e] = 0.f;
+            if (p.accumulate) {
+              oq[e] = dq_bh[off[e]];
+              ov[e] = dv_bh[off[e]];
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float cf = __shfl_sync(0xffffffffu, coef, e0 + e);
+            dq_bh[off[e]] = oq[e] + fmaf(-cf, xval(e0 + e), __uint_as_float(hr[e0 + e]));
+            dv_bh[off[e]] = ov[e] + __uint_as_float(vr[e0 + e]);
+          }
+        }
+      }
+      return true;
+    };
+    auto release = [&](uint32_t s) {  // after the slot's last reader in this warp group
+      tc::named_bar_sync(1, 128);
+      if (threadIdx.x == 12 * 32) tc::mbar_arrive(&slot_free[s]);
+    };
+    while (f.valid) {
+      const uint32_t s = F & 1, sp = (F + 1) & 1;
+      if (f.kind == kLead) {
+        ++F;
+        f.advance(p);
+        continue;
+      }
+      if (f.owns_prev()) {  // chunk 2t-1 (rows 64.. of the previous slot) finished by this fill's first block
+        if (!chunk_out(n - 1, sp, 64, (ff + 1) & 1, f.bh)) break;
+        release(sp);
+      }
+      if (f.kind == kFull) {
+        ok = epi_wait(&slot_full[s], (F >> 1) & 1);
+        ok = ok && epi_wait(&r_full[ff & 1], (ff >> 1) & 1);
+        if (!ok) break;
+        if (!chunk_out(n, s, 0, ff & 1, f.bh)) break;
+        if (f.t == p.n_fills - 1) {  // segment end: chunk 2t+1 has no later queries
+          if (!chunk_out(n + 1, s, 64, ff & 1, f.bh)) break;
+          release(s);
+        }
+        n += 2;
+        ++ff;
+      }
+      ++F;
+      f.advance(p);
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Per-token terms of the backward: LSE log2 e, Delta = dout . out, 1/max(||x||, 1e-12)
+// and the key-normalisation coefficient (||x|| >= 1e-12) / max(||x||, 1e-12)^2.
+// One warp per token; D = 128, bf16 rows.
+__global__ void bwd_aux_kernel(const __nv_bfloat16* __restrict__ qk, const __nv_bfloat16* __restrict__ out,
+                               const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
+                               float4* __restrict__ aux, long long n_tokens) {
+  const long long tok = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (tok >= n_tokens) return;
+  const int lane = threadIdx.x & 31;
+  float x[4], o[4], g[4];
+  load4_bf16(qk + tok * kD + 4 * lane, x);
+  load4_bf16(out + tok * kD + 4 * lane, o);
+  load4_bf16(dout + tok * kD + 4 * lane, g);
+  float ss = 0.f, dl = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    ss = fmaf(x[e], x[e], ss);
+    dl = fmaf(g[e], o[e], dl);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    dl += __shfl_xor_sync(0xffffffffu, dl, off);
+  }
+  if (lane == 0) {
+    const float nrm = sqrtf(ss);
+    const float kinv = 1.f / fmaxf(nrm, 1e-12f);
+    aux[tok] = make_float4(lse[tok] * 1.4426950408889634f, dl, kinv, nrm >= 1e-12f ? kinv * kinv : 0.f);
+  }
+}
+
+}  // namespace bwd_tc
+}  // namespace lsh

@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 
 #include "attend_bwd_simt.cuh"
+#include "attend_bwd_tc.cuh"
 #include "attend_simt.cuh"
 #include "attend_tc.cuh"
 #include "combine.cuh"
@@ -196,6 +197,54 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
     return LSH_ERR_CUDA;
   kfn<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
+}
+
+// Tensor-core backward (bf16 rows and out / dout, D 128, chunk 64, L % 128 == 0,
+// plain window) on sm_100: per-token terms into a stream-ordered scratch
+// buffer, then one launch per round.
+lsh_status launch_attend_bwd_tc(const void* qk, const void* v, const int32_t* perm, int B, int H, int L,
+                                int n_rounds, int self_mask, float scale, const void* out, const float* lse,
+                                const void* dout, float* dqk, float* dv, cudaStream_t s, int sms) {
+  using namespace lsh::bwd_tc;
+  // the setmaxnreg split hands out exactly the registers the launch holds: 512 threads x 128
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, attend_bwd_tc_kernel) != cudaSuccess || fa.numRegs != 128) return LSH_ERR_UNSUPPORTED;
+  const long long bhs = (long long)B * H, n_tok = bhs * L;
+  float4* aux = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&aux), (size_t)n_tok * sizeof(float4), s) != cudaSuccess)
+    return LSH_ERR_CUDA;
+  const int warps = 8;
+  bwd_aux_kernel<<<(unsigned)((n_tok + warps - 1) / warps), warps * 32, 0, s>>>(
+      (const __nv_bfloat16*)qk, (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, aux, n_tok);
+  Params p;
+  p.qk = (const uint8_t*)qk;
+  p.v = (const uint8_t*)v;
+  p.dout = (const uint8_t*)dout;
+  p.perm = perm;
+  p.aux = aux;
+  p.dqk = dqk;
+  p.dv = dv;
+  p.L = L;
+  p.n_rounds = n_rounds;
+  p.n_fills = L / kRows;
+  p.run = 16;
+  p.units_per_seg = (p.n_fills + p.run - 1) / p.run;
+  p.n_units = bhs * p.units_per_seg;
+  p.self_mask = self_mask;
+  p.scale = scale;
+  const unsigned grid = (unsigned)std::min<long long>(p.n_units, sms);
+  const int smem = (int)Layout::kSmem;
+  lsh_status st = LSH_OK;
+  if (cudaFuncSetAttribute(attend_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    st = LSH_ERR_CUDA;
+  for (int r = 0; st == LSH_OK && r < n_rounds; ++r) {  // rounds in order: each token has one writer per launch
+    p.round = r;
+    p.accumulate = r > 0 ? 1 : 0;
+    attend_bwd_tc_kernel<<<grid, kThreads, smem, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) st = LSH_ERR_CUDA;
+  }
+  if (cudaFreeAsync(aux, s) != cudaSuccess && st == LSH_OK) st = LSH_ERR_CUDA;
+  return st;
 }
 
 }  // namespace
@@ -507,6 +556,11 @@ lsh_status lsh_chunk_attend_backward(const void* qk, const void* v, int dtype, i
   const size_t smem = lsh::bwd_smem_words(D, n_rounds, union_count) * 4;
   if (smem > (size_t)227 * 1024) return LSH_ERR_UNSUPPORTED;  // union with very many rounds
   cudaStream_t s = as_stream(stream);
+  const DevInfo di = dev_info();
+  if (di.major == 10 && dtype == LSH_BF16 && out_dtype == LSH_BF16 && D == 128 && chunk == 64 && L % 128 == 0 &&
+      !causal && !bucket_mask)
+    return launch_attend_bwd_tc(qk, v, perm, B, H, L, n_rounds, self_mask, scale, out, lse, dout, dqk, dv, s,
+                                di.sms);
   const size_t grad_bytes = (size_t)bhs * L * D * sizeof(float);
   if (cudaMemsetAsync(dqk, 0, grad_bytes, s) != cudaSuccess || cudaMemsetAsync(dv, 0, grad_bytes, s) != cudaSuccess)
     return LSH_ERR_CUDA;

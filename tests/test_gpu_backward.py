@@ -83,6 +83,36 @@ def test_backward_is_deterministic():
     assert torch.equal(dqk, dqk2) and torch.equal(dv, dv2)
 
 
+# The tensor-core backward serves bf16, D 128, chunk 64, L % 128 == 0 and the plain window: work units of
+# 16 fills (2048 tokens), so L > 2048 has leading and half fills between units.
+@pytest.mark.parametrize("name,shape,kw", [
+    ("bwd_tc_one_fill", (1, 1, 128, 128, "bf16", 16, 64, 1), dict()),
+    ("bwd_tc_units", (1, 2, 4096, 128, "bf16", 64, 64, 2), dict()),
+    ("bwd_tc_ragged_units_noself", (1, 1, 5120, 128, "bf16", 64, 64, 3), dict(self_mask=False)),
+    ("bwd_tc_scale", (2, 1, 1024, 128, "bf16", 32, 64, 2), dict(scale=0.5)),
+])
+def test_tensor_core_backward_matches_oracle(name, shape, kw):
+    w = synth.small_workload(name, *shape)
+    qk, v, dout, res, dqk, dv = _run(w, zlib.crc32(name.encode()) % 1000, **kw)
+    _check(qk, v, dout, res, dqk, dv, w.chunk, w.torch_dtype, **kw)
+
+
+def test_tensor_core_backward_more_units_than_sms():
+    """160 one-fill units: every persistent CTA walks several (b, h) slices."""
+    w = synth.small_workload("bwd_tc_many", 10, 16, 128, 128, "bf16", 16, 64, 2)
+    qk, v, dout, res, dqk, dv = _run(w, 11)
+    _check(qk, v, dout, res, dqk, dv, w.chunk, w.torch_dtype, slices=[(0, 0), (3, 7), (9, 15), (5, 0)])
+
+
+def test_tensor_core_backward_is_deterministic():
+    w = synth.small_workload("bwd_tc_det", 1, 2, 4096, 128, "bf16", 64, 64, 2)
+    qk, v, dout, res, dqk, dv = _run(w, 5)
+    dqk2, dv2 = lsh.lsh_chunk_attend_backward(qk.to(DEV), v.to(DEV), res["perm"], w.chunk, res["out"], res["lse"],
+                                              dout.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(dqk, dqk2) and torch.equal(dv, dv2)
+
+
 @pytest.mark.slow
 def test_64k_workload_backward_one_slice():
     """The full-size backward launch (B 8, H 8, L 65536, D 128, bf16, 1024 buckets, chunk 64, 8 rounds),

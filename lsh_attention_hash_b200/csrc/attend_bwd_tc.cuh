@@ -35,9 +35,11 @@
 // regions (chunk 2t+1 is finished by the next fill's first block).  The
 // epilogue warps take a finished region: x_j . H_j (a reduction over the 128
 // lanes) minus x_j . dQ_j (= sum_k Z_jk S_jk, summed by the softmax warps as
-// they go) gives x_j . G_j for the key-normalisation term; the rows are added
-// into dqk / dv at the tokens' original positions (32 lanes write 128
-// consecutive bytes of one row).
+// they go) gives x_j . G_j for the key-normalisation term; the rows go to
+// dqk / dv at the tokens' original positions (32 lanes cover 128 consecutive
+// bytes of one row), stored by the first round and added in L2 by the later
+// ones (fire-and-forget reductions: one writer per element and launch, so the
+// sums do not depend on timing).
 //
 // Work units are runs of fills of one (b, h) segment.  A unit's first fill
 // takes the chunk before it from a leading fill, whose key-role sums belong to
@@ -221,6 +223,10 @@ __device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float (&o)[4]
   o[1] = __high2float(a);
   o[2] = __low2float(b);
   o[3] = __high2float(b);
+}
+
+__device__ __forceinline__ void red_add(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ uint32_t swz(int r, int c) {  // 16-byte piece c (0..7) of row r of a 64-wide tile
@@ -655,25 +661,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         const float rr = r_s[(rbuf * 2) * kRows + row_l] + r_s[(rbuf * 2 + 1) * kRows + row_l];
         const float coef = (tot - rr) * aux_s[s * kRows + row_l].w;  // (x . G) (||x|| >= 1e-12) / ||x||^2
         tc::named_bar_sync(1, 128);  // xh is reused by the next half
+        // each element of dqk / dv has one writer per launch and the launches run in order, so a
+        // reduction in L2 (no load round trip) adds exactly what a read-modify-write would
 #pragma unroll
-        for (int e0 = 0; e0 < 32; e0 += 8) {
-          float oq[8], ov[8];
-          int off[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            off[e] = pm[32 * h + e0 + e] * kD;
-            oq[e] = 0.f;
-            ov[e] = 0.f;
-            if (p.accumulate) {
-              oq[e] = dq_bh[off[e]];
-              ov[e] = dv_bh[off[e]];
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float cf = __shfl_sync(0xffffffffu, coef, e0 + e);
-            dq_bh[off[e]] = oq[e] + fmaf(-cf, xval(e0 + e), __uint_as_float(hr[e0 + e]));
-            dv_bh[off[e]] = ov[e] + __uint_as_float(vr[e0 + e]);
+        for (int e = 0; e < 32; ++e) {
+          const int off = pm[32 * h + e] * kD;
+          const float cf = __shfl_sync(0xffffffffu, coef, e);
+          const float gq = fmaf(-cf, xval(e), __uint_as_float(hr[e]));
+          const float gv = __uint_as_float(vr[e]);
+          if (p.accumulate) {
+            red_add(dq_bh + off, gq);
+            red_add(dv_bh + off, gv);
+          } else {
+            dq_bh[off] = gq;
+            dv_bh[off] = gv;
           }
         }
       }

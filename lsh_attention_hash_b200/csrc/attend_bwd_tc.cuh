@@ -90,7 +90,8 @@ struct Layout {
   static constexpr uint32_t kPerm = kKinv + 2 * kRows * 4;  // int32 [2][128]: original positions
   static constexpr uint32_t kR = kPerm + 2 * kRows * 4;     // float [2][2][128]: x_i . dQ_i partials
   static constexpr uint32_t kXH = kR + 2 * 2 * kRows * 4;   // float [4][32]: epilogue partial sums
-  static constexpr uint32_t kBar = kXH + 4 * 32 * 4;
+  static constexpr uint32_t kStage = kXH + 4 * 32 * 4;      // float [4 warps][32 tokens][32 features]
+  static constexpr uint32_t kBar = kStage + 4 * 32 * 32 * 4;
   // slot_full[2] slot_free[2] do_full do_free sp_full sp_free pz_full pz_free
   // hv_done[3] hv_free[3] r_full[2] done
   static constexpr int kNumBars = 19;
@@ -225,8 +226,9 @@ __device__ __forceinline__ void load4_bf16(const __nv_bfloat16* p, float (&o)[4]
   o[3] = __high2float(b);
 }
 
-__device__ __forceinline__ void red_add(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+__device__ __forceinline__ void red_add_v4(float* p, float4 v) {  // 16-byte aligned
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
 }
 
 __device__ __forceinline__ uint32_t swz(int r, int c) {  // 16-byte piece c (0..7) of row r of a 64-wide tile
@@ -357,7 +359,7 @@ __device__ __noinline__ void issuer(const Params& p, uint8_t* smem, uint32_t tme
         }
         tc::umma_commit(pz_free);
         if (owns_prev) tc::umma_commit(&hv_done[(n + 2) % 3]);
-        if (first) tc::umma_commit(&slot_free[sp]);  // the leading fill's slot
+        if (first) tc::umma_commit(&slot_free[sp]);  // the leading fill's slot (full fills: the epilogue)
       } else if (b == 1) {
         if (!has_prev) {
           ok = att_tc::issuer_wait(&hv_free[n % 3], ((n / 3) & 1) ^ 1, abort_flag);
@@ -408,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* slot_full = bars;      // [2] a fill's rows and tables landed (64 producer lanes)
   uint64_t* slot_free = bars + 2;  // [2] a fill slot may be refilled
-  uint64_t* do_full = bars + 4;    // dO rows landed (64)
+  uint64_t* do_full = bars + 4;    // dO rows landed (32 lanes of warp 3)
   uint64_t* do_free = bars + 5;    // dO tile read by the fill's last UMMA
   uint64_t* sp_full = bars + 6;    // S and dP of a block computed
   uint64_t* sp_free = bars + 7;    // S and dP loaded by the softmax (256)
@@ -432,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       tc::mbar_init(&slot_free[i], 1);
       tc::mbar_init(&r_full[i], 256);
     }
-    tc::mbar_init(do_full, 64);
+    tc::mbar_init(do_full, 32);
     tc::mbar_init(do_free, 1);
     tc::mbar_init(sp_full, 1);
     tc::mbar_init(sp_free, 256);
@@ -459,10 +461,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       // ------------------------------------------------------------ producers
       const int pw = warp;
       const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK), v0 = tc::smem_u32(smem + Lay::kV);
-      const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
       FillIt f;
       f.init(p);
-      uint32_t F = 0, nd = 0;
+      uint32_t F = 0;
       while (f.valid) {
         const int s = F & 1;
         int pos[2];
@@ -486,16 +487,29 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
           if (f.kind != kHalo) gather64(v0 + s * Lay::kTile, p.v, rb, pw, pos);
         }
         tc::cp_async_arrive(&slot_full[s]);
-        if (f.kind != kLead) {
-          if (!att_tc::warp_wait(do_free, (nd & 1) ^ 1, abort_flag)) break;
-          if (mine) gather64(do0, p.dout, f.bh * L, pw, pos);
-          tc::cp_async_arrive(do_full);
-          ++nd;
-        }
         ++F;
         f.advance(p);
       }
       asm volatile("cp.async.wait_all;" ::: "memory");  // never leave with copies in flight
+    } else if (warp == 3) {
+      // ------------------------------------------------------------ dO producer
+      const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
+      FillIt f;
+      f.init(p);
+      uint32_t nd = 0;
+      while (f.valid) {
+        if (f.kind != kLead) {
+          int pos0[2], pos1[2];
+          const bool m0 = fill_rows(p, f, 0, pos0), m1 = fill_rows(p, f, 1, pos1);
+          if (!att_tc::warp_wait(do_free, (nd & 1) ^ 1, abort_flag)) break;
+          if (m0) gather64(do0, p.dout, f.bh * L, 0, pos0);
+          if (m1) gather64(do0, p.dout, f.bh * L, 1, pos1);
+          tc::cp_async_arrive(do_full);
+          ++nd;
+        }
+        f.advance(p);
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == 2) {
       // ------------------------------------------------------------ UMMA issuer
       if (lane == 0) issuer(p, smem, tmem, abort_flag);
@@ -617,23 +631,40 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
     float* xh = reinterpret_cast<float*>(smem + Lay::kXH);
     FillIt f;
     f.init(p);
-    uint32_t F = 0, n = 0, ff = 0;
-    bool ok = true;
-    // one finished chunk: region of owned chunk c, rows [row0, row0 + 64) of slot s, x . dQ partials rbuf
+    uint32_t n = 0, ff = 0;
     // every wait of the epilogue warps ends in one joint decision, so that their named barriers stay matched
     auto epi_wait = [&](uint64_t* bar, uint32_t parity) {
       return bar_and(1, 128, att_tc::warp_wait(bar, parity, abort_flag));
     };
+    float* stage = reinterpret_cast<float*>(smem + Lay::kStage) + q * 32 * 32;  // this warp's [token][feature]
+    // 32 tokens x this warp's 32 features from the staging tile to their rows: 4 tokens per instruction,
+    // 16 bytes per lane; the first round stores, later ones add in L2 (one writer per element and
+    // launch, launches in order: the sums do not depend on timing)
+    auto rows_out = [&](float* base, const int32_t* pm) {
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int t = 4 * it + (lane >> 3), f4 = 4 * (lane & 7);
+        const float4 val = *reinterpret_cast<const float4*>(stage + t * 32 + f4);
+        float* dst = base + (long long)pm[t] * kD + f4;
+        if (p.accumulate)
+          red_add_v4(dst, val);
+        else
+          *reinterpret_cast<float4*>(dst) = val;
+      }
+    };
+    // One finished chunk: TMEM region of owned chunk c, rows [row0, row0 + 64) of fill slot s, x . dQ
+    // partials in r buffer rbuf.
     auto chunk_out = [&](uint32_t c, uint32_t s, int row0, uint32_t rbuf, long long bh) -> bool {
       if (!epi_wait(&hv_done[c % 3], (c / 3) & 1)) return false;
       tc::tc_fence_after();
       const uint32_t reg = tmem + lane_base + kRegCol0 + (c % 3) * kRegCols;
       const uint8_t* xt = smem + Lay::kQK + s * Lay::kTile + (d >> 6) * Lay::kHalf;
       const int dc = (d & 63) >> 3, de = d & 7;
-      float* dq_bh = p.dqk + bh * L * kD + d;
-      float* dv_bh = p.dv + bh * L * kD + d;
-      const int32_t* pm = perm_s + s * kRows + row0;
+      float* dq_w = p.dqk + bh * L * kD + 32 * q;  // this warp's 32 features
+      float* dv_w = p.dv + bh * L * kD + 32 * q;
+#pragma unroll 1
       for (int h = 0; h < 2; ++h) {
+        const int32_t* pm = perm_s + s * kRows + row0 + 32 * h;
         uint32_t hr[32], vr[32];
         tc::tmem_ld32(reg + 32 * h, hr);
         tc::tmem_ld32(reg + 64 + 32 * h, vr);
@@ -643,16 +674,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
           tc::tc_fence_before();
           tc::mbar_arrive(&hv_free[c % 3]);
         }
-        auto xval = [&](int e) {  // x of token row row0 + 32 h + e, feature d
-          return __bfloat162float(
+        float x[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)  // x of token row row0 + 32 h + e, feature d
+          x[e] = __bfloat162float(
               *reinterpret_cast<const __nv_bfloat16*>(xt + swz(row0 + 32 * h + e, dc) + 2 * de));
-        };
         float part;
         {
-          float pr[32];
+          float pr2[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pr[e] = xval(e) * __uint_as_float(hr[e]);
-          part = transpose_reduce(pr, lane);  // token row0 + 32 h + lane, this warp's 32 features
+          for (int e = 0; e < 32; ++e) pr2[e] = x[e] * __uint_as_float(hr[e]);
+          part = transpose_reduce(pr2, lane);  // token 32 h + lane, this warp's 32 features
         }
         xh[q * 32 + lane] = part;
         tc::named_bar_sync(1, 128);
@@ -661,22 +693,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         const float rr = r_s[(rbuf * 2) * kRows + row_l] + r_s[(rbuf * 2 + 1) * kRows + row_l];
         const float coef = (tot - rr) * aux_s[s * kRows + row_l].w;  // (x . G) (||x|| >= 1e-12) / ||x||^2
         tc::named_bar_sync(1, 128);  // xh is reused by the next half
-        // each element of dqk / dv has one writer per launch and the launches run in order, so a
-        // reduction in L2 (no load round trip) adds exactly what a read-modify-write would
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int off = pm[32 * h + e] * kD;
-          const float cf = __shfl_sync(0xffffffffu, coef, e);
-          const float gq = fmaf(-cf, xval(e), __uint_as_float(hr[e]));
-          const float gv = __uint_as_float(vr[e]);
-          if (p.accumulate) {
-            red_add(dq_bh + off, gq);
-            red_add(dv_bh + off, gv);
-          } else {
-            dq_bh[off] = gq;
-            dv_bh[off] = gv;
-          }
-        }
+        for (int e = 0; e < 32; ++e)
+          stage[e * 32 + lane] = fmaf(-__shfl_sync(0xffffffffu, coef, e), x[e], __uint_as_float(hr[e]));
+        __syncwarp();
+        rows_out(dq_w, pm);
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) stage[e * 32 + lane] = __uint_as_float(vr[e]);
+        __syncwarp();
+        rows_out(dv_w, pm);
+        __syncwarp();
       }
       return true;
     };
@@ -684,6 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       tc::named_bar_sync(1, 128);
       if (threadIdx.x == 12 * 32) tc::mbar_arrive(&slot_free[s]);
     };
+    uint32_t F = 0;
     while (f.valid) {
       const uint32_t s = F & 1, sp = (F + 1) & 1;
       if (f.kind == kLead) {
@@ -696,9 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         release(sp);
       }
       if (f.kind == kFull) {
-        ok = epi_wait(&slot_full[s], (F >> 1) & 1);
-        ok = ok && epi_wait(&r_full[ff & 1], (ff >> 1) & 1);
-        if (!ok) break;
+        if (!epi_wait(&slot_full[s], (F >> 1) & 1) || !epi_wait(&r_full[ff & 1], (ff >> 1) & 1)) break;
         if (!chunk_out(n, s, 0, ff & 1, f.bh)) break;
         if (f.t == p.n_fills - 1) {  // segment end: chunk 2t+1 has no later queries
           if (!chunk_out(n + 1, s, 64, ff & 1, f.bh)) break;

@@ -50,10 +50,11 @@
 //
 // Warp roles (512 threads, one CTA per SM; launched at 128 registers, warpgroup
 // 0 gives 56 to the others with setmaxnreg: 72 / 144 / 144 / 152):
-//   warps 0-1   producers: 16-byte cp.async row gathers (X, V, dO) through perm
-//               into 128-byte-swizzled tiles, two fill slots for X and V, one
-//               dO tile, plus each row's LSE, Delta and length terms;
-//   warp 2      TMEM owner; its lane 0 issues every UMMA;
+//   warps 0-1   producers: 16-byte cp.async row gathers (X, V, then dO) through
+//               perm into 128-byte-swizzled tiles, two fill slots for X and V,
+//               one dO tile, plus each row's LSE, Delta and length terms;
+//   warps 2-3   UMMA issuers (lane 0): warp 2 the S and dP of each block, warp 3
+//               the gradient products; warp 2 also owns the TMEM allocation;
 //   warps 4-11  softmax: both warpgroups take every row (TMEM lane), keys
 //               0-31 / 32-63 of each block;
 //   warps 12-15 epilogue.
@@ -279,21 +280,69 @@ __device__ __forceinline__ void issue_sdp(uint32_t tmem, uint32_t xs, uint32_t d
   tc::umma_commit(sp_full);
 }
 
-// Lane 0 of warp 2: every UMMA of the CTA, in fill order (see the kernel's comment).
-__device__ __noinline__ void issuer(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag) {
+// Lane 0 of warp 2: the S and dP UMMAs of every block, in fill order; each waits until the softmax
+// has loaded the previous block's S and dP.
+__device__ __noinline__ void issuer_s(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag) {
   using Lay = Layout;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* slot_full = bars;
   uint64_t* slot_free = bars + 2;
   uint64_t* do_full = bars + 4;
-  uint64_t* do_free = bars + 5;
   uint64_t* sp_full = bars + 6;
   uint64_t* sp_free = bars + 7;
+  const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK), v0 = tc::smem_u32(smem + Lay::kV);
+  const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
+  FillIt f;
+  f.init(p);
+  uint32_t F = 0, nd = 0, kb = 0;  // fills, dO fills, blocks
+  bool ok = true;
+  while (ok && f.valid) {
+    const uint32_t s = F & 1, sp = (F + 1) & 1;
+    if (f.kind == kLead) {
+      ++F;
+      f.advance(p);
+      continue;
+    }
+    const bool full = f.kind == kFull, has_prev = f.has_prev();
+    ok = att_tc::issuer_wait(&slot_full[s], (F >> 1) & 1, abort_flag) &&
+         (!has_prev || att_tc::issuer_wait(&slot_full[sp], ((F - 1) >> 1) & 1, abort_flag)) &&
+         att_tc::issuer_wait(do_full, nd & 1, abort_flag);
+    if (!ok) break;
+    tc::tc_fence_after();
+    if (full && f.t == f.t0 && !has_prev) tc::umma_commit(&slot_free[sp]);  // nothing of the leading fill is read
+    const uint32_t xs = qk0 + s * Lay::kTile, vs = v0 + s * Lay::kTile;
+    const uint32_t xp = qk0 + sp * Lay::kTile, vp = v0 + sp * Lay::kTile;
+    // blocks: 0 = chunk 2t-1 (rows 64.. of the previous slot), 1 = chunk 2t, 2 = chunk 2t+1
+    for (int b = has_prev ? 0 : 1; b <= (full ? 2 : 0); ++b) {
+      ok = att_tc::issuer_wait(sp_free, (kb & 1) ^ 1, abort_flag);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const uint32_t kx = b == 0 ? xp + 64 * 128 : xs + (b == 2 ? 64 * 128 : 0);
+      const uint32_t kv = b == 0 ? vp + 64 * 128 : vs + (b == 2 ? 64 * 128 : 0);
+      issue_sdp(tmem, xs, do0, kx, kv, sp_full);
+      ++kb;
+    }
+    ++nd;
+    ++F;
+    f.advance(p);
+  }
+  uint64_t* done_bar = bars + 18;
+  tc::umma_commit(done_bar);
+  att_tc::drain_wait(done_bar, 0);
+}
+
+// Lane 0 of warp 3: the gradient UMMAs of every block (dK^T, dV^T of its keys, dQ^T of the query
+// chunks that see it), in fill order, each once the softmax has written the block's P~ and Z.
+__device__ __noinline__ void issuer_hv(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag) {
+  using Lay = Layout;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+  uint64_t* slot_free = bars + 2;
+  uint64_t* do_free = bars + 5;
   uint64_t* pz_full = bars + 8;
   uint64_t* pz_free = bars + 9;
   uint64_t* hv_done = bars + 10;
   uint64_t* hv_free = bars + 13;
-  const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK), v0 = tc::smem_u32(smem + Lay::kV);
+  const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK);
   const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
   const uint32_t pt = tc::smem_u32(smem + Lay::kP), zt = tc::smem_u32(smem + Lay::kZ);
   const uint32_t id_kv = tc::idesc_bf16_f32(128, 64, 1, 1);  // dK^T, dV^T: both MN-major
@@ -301,7 +350,7 @@ __device__ __noinline__ void issuer(const Params& p, uint8_t* smem, uint32_t tme
   constexpr uint32_t kRowStep = 16 * 128;                    // 16 tile rows
   FillIt f;
   f.init(p);
-  uint32_t F = 0, nd = 0, kb = 0, n = 0;  // fills, dO fills, blocks, owned chunks
+  uint32_t F = 0, kb = 0, n = 0;  // fills, blocks, owned chunks
   bool ok = true;
   while (ok && f.valid) {
     const uint32_t s = F & 1, sp = (F + 1) & 1;
@@ -312,39 +361,16 @@ __device__ __noinline__ void issuer(const Params& p, uint8_t* smem, uint32_t tme
     }
     const bool full = f.kind == kFull, has_prev = f.has_prev(), owns_prev = f.owns_prev();
     const bool first = full && f.t == f.t0, seg_end = full && f.t == p.n_fills - 1;
-    ok = att_tc::issuer_wait(&slot_full[s], (F >> 1) & 1, abort_flag) &&
-         (!has_prev || att_tc::issuer_wait(&slot_full[sp], ((F - 1) >> 1) & 1, abort_flag)) &&
-         att_tc::issuer_wait(do_full, nd & 1, abort_flag);
-    if (!ok) break;
-    tc::tc_fence_after();
-    const uint32_t xs = qk0 + s * Lay::kTile, vs = v0 + s * Lay::kTile;
-    const uint32_t xp = qk0 + sp * Lay::kTile, vp = v0 + sp * Lay::kTile;
-    if (first && !has_prev) tc::umma_commit(&slot_free[sp]);  // nothing of the leading fill is read
-    // blocks: 0 = chunk 2t-1 (rows 64.. of the previous slot), 1 = chunk 2t, 2 = chunk 2t+1
-    const int b_first = has_prev ? 0 : 1, b_last = full ? 2 : 0;
-    // regions: chunk 2t-1 -> owned chunk n-1, 2t -> n, 2t+1 -> n+1
+    const uint32_t xs = qk0 + s * Lay::kTile, xp = qk0 + sp * Lay::kTile;
+    // regions: chunk 2t-1 -> owned chunk n-1, 2t -> n, 2t+1 -> n+1; the first write into a region
+    // waits until the epilogue has read the chunk three before it
     const uint32_t rp = tmem + kRegCol0 + ((n + 2) % 3) * kRegCols;
     const uint32_t r0 = tmem + kRegCol0 + (n % 3) * kRegCols;
     const uint32_t r1 = tmem + kRegCol0 + ((n + 1) % 3) * kRegCols;
-    for (int b = b_first; b <= b_last; ++b) {
-      if (b == b_first) {
-        ok = att_tc::issuer_wait(sp_free, (kb & 1) ^ 1, abort_flag);
-        if (!ok) break;
-        tc::tc_fence_after();
-      }
-      if (b == b_first)  // S and dP of the first block
-        issue_sdp(tmem, xs, do0, b == 0 ? xp + 64 * 128 : xs, b == 0 ? vp + 64 * 128 : vs, sp_full);
-      if (b < b_last) {  // the next block's S and dP while the softmax works on this one
-        ok = att_tc::issuer_wait(sp_free, kb & 1, abort_flag);
-        if (!ok) break;
-        tc::tc_fence_after();
-        const uint32_t ro = b + 1 == 2 ? 64 * 128 : 0;
-        issue_sdp(tmem, xs, do0, xs + ro, vs + ro, sp_full);
-      }
+    for (int b = has_prev ? 0 : 1; b <= (full ? 2 : 0); ++b) {
       ok = att_tc::issuer_wait(pz_full, kb & 1, abort_flag);
       if (!ok) break;
       tc::tc_fence_after();
-      // first write into a chunk region waits until the epilogue has read the chunk three before it
       if (b == 0) {
         if (owns_prev) {  // key role of chunk 2t-1: queries of chunk 2t (rows 0..63)
           mma_run(rp, mdesc(xs, 0), kRowStep, mdesc(zt, 0), kRowStep, id_kv, 4, true);
@@ -390,10 +416,9 @@ __device__ __noinline__ void issuer(const Params& p, uint8_t* smem, uint32_t tme
       ++kb;
     }
     if (!ok) break;
-    tc::umma_commit(do_free);
+    tc::umma_commit(do_free);  // the fill's last dP was read before its softmax wrote the last block
     if (!full) tc::umma_commit(&slot_free[s]);  // the half fill's slot
     if (full) n += 2;
-    ++nd;
     ++F;
     f.advance(p);
   }
@@ -410,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* slot_full = bars;      // [2] a fill's rows and tables landed (64 producer lanes)
   uint64_t* slot_free = bars + 2;  // [2] a fill slot may be refilled
-  uint64_t* do_full = bars + 4;    // dO rows landed (32 lanes of warp 3)
+  uint64_t* do_full = bars + 4;    // dO rows landed (64 producer lanes)
   uint64_t* do_free = bars + 5;    // dO tile read by the fill's last UMMA
   uint64_t* sp_full = bars + 6;    // S and dP of a block computed
   uint64_t* sp_free = bars + 7;    // S and dP loaded by the softmax (256)
@@ -434,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       tc::mbar_init(&slot_free[i], 1);
       tc::mbar_init(&r_full[i], 256);
     }
-    tc::mbar_init(do_full, 32);
+    tc::mbar_init(do_full, 64);
     tc::mbar_init(do_free, 1);
     tc::mbar_init(sp_full, 1);
     tc::mbar_init(sp_free, 256);
@@ -444,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       tc::mbar_init(&hv_done[i], 1);
       tc::mbar_init(&hv_free[i], 128);
     }
-    tc::mbar_init(done_bar, 1);
+    tc::mbar_init(done_bar, 2);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -463,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK), v0 = tc::smem_u32(smem + Lay::kV);
       FillIt f;
       f.init(p);
-      uint32_t F = 0;
+      uint32_t F = 0, nd = 0;
       while (f.valid) {
         const int s = F & 1;
         int pos[2];
@@ -487,32 +512,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
           if (f.kind != kHalo) gather64(v0 + s * Lay::kTile, p.v, rb, pw, pos);
         }
         tc::cp_async_arrive(&slot_full[s]);
+        if (f.kind != kLead) {  // the fill's dO rows, once the previous fill's UMMAs are done with the tile
+          if (!att_tc::warp_wait(do_free, (nd & 1) ^ 1, abort_flag)) break;
+          if (mine) gather64(tc::smem_u32(smem + Lay::kDO), p.dout, f.bh * L, pw, pos);
+          tc::cp_async_arrive(do_full);
+          ++nd;
+        }
         ++F;
         f.advance(p);
       }
       asm volatile("cp.async.wait_all;" ::: "memory");  // never leave with copies in flight
-    } else if (warp == 3) {
-      // ------------------------------------------------------------ dO producer
-      const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
-      FillIt f;
-      f.init(p);
-      uint32_t nd = 0;
-      while (f.valid) {
-        if (f.kind != kLead) {
-          int pos0[2], pos1[2];
-          const bool m0 = fill_rows(p, f, 0, pos0), m1 = fill_rows(p, f, 1, pos1);
-          if (!att_tc::warp_wait(do_free, (nd & 1) ^ 1, abort_flag)) break;
-          if (m0) gather64(do0, p.dout, f.bh * L, 0, pos0);
-          if (m1) gather64(do0, p.dout, f.bh * L, 1, pos1);
-          tc::cp_async_arrive(do_full);
-          ++nd;
-        }
-        f.advance(p);
+    } else {
+      // ------------------------------------------------------------ UMMA issuers
+      if (lane == 0) {
+        if (warp == 2)
+          issuer_s(p, smem, tmem, abort_flag);
+        else
+          issuer_hv(p, smem, tmem, abort_flag);
       }
-      asm volatile("cp.async.wait_all;" ::: "memory");
-    } else if (warp == 2) {
-      // ------------------------------------------------------------ UMMA issuer
-      if (lane == 0) issuer(p, smem, tmem, abort_flag);
       __syncwarp();
     }
   } else if (warp < 12) {

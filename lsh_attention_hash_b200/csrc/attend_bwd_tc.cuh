@@ -654,15 +654,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       return bar_and(1, 128, att_tc::warp_wait(bar, parity, abort_flag));
     };
     float* stage = reinterpret_cast<float*>(smem + Lay::kStage) + q * 32 * 32;  // this warp's [token][feature]
-    // 32 tokens x this warp's 32 features from the staging tile to their rows: 4 tokens per instruction,
-    // 16 bytes per lane; the first round stores, later ones add in L2 (one writer per element and
-    // launch, launches in order: the sums do not depend on timing)
-    auto rows_out = [&](float* base, const int32_t* pm) {
+    // 32 tokens x this warp's 32 features from the staging tile to their rows (token t's position
+    // in lane t of pos): 4 tokens per instruction, 16 bytes per lane; the first round stores,
+    // later ones add in L2 (one writer per element and launch, launches in order: the sums do not
+    // depend on timing)
+    auto rows_out = [&](float* base, int pos) {
 #pragma unroll
       for (int it = 0; it < 8; ++it) {
         const int t = 4 * it + (lane >> 3), f4 = 4 * (lane & 7);
         const float4 val = *reinterpret_cast<const float4*>(stage + t * 32 + f4);
-        float* dst = base + (long long)pm[t] * kD + f4;
+        float* dst = base + (long long)__shfl_sync(0xffffffffu, pos, t) * kD + f4;
         if (p.accumulate)
           red_add_v4(dst, val);
         else
@@ -670,37 +671,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       }
     };
     // One finished chunk: TMEM region of owned chunk c, rows [row0, row0 + 64) of fill slot s, x . dQ
-    // partials in r buffer rbuf.
-    auto chunk_out = [&](uint32_t c, uint32_t s, int row0, uint32_t rbuf, long long bh) -> bool {
+    // partials in r buffer rbuf.  What it needs from the slot is copied to registers first; a
+    // chunk that is its slot's last reader (`last`) releases the slot before its arithmetic.
+    auto chunk_out = [&](uint32_t c, uint32_t s, int row0, uint32_t rbuf, long long bh, bool last) -> bool {
       if (!epi_wait(&hv_done[c % 3], (c / 3) & 1)) return false;
       tc::tc_fence_after();
+      const uint16_t* xt = reinterpret_cast<const uint16_t*>(smem + Lay::kQK + s * Lay::kTile +
+                                                             (d >> 6) * Lay::kHalf) + (d & 7);
+      const int dc = (d & 63) >> 3;
+      uint32_t xpk[32];  // bf16 x of tokens e (low half) and 32 + e (high half), feature d
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        xpk[e] = (uint32_t)xt[swz(row0 + e, dc) / 2] | ((uint32_t)xt[swz(row0 + 32 + e, dc) / 2] << 16);
+      const int pos_a = perm_s[s * kRows + row0 + lane], pos_b = perm_s[s * kRows + row0 + 32 + lane];
+      const float kc_a = aux_s[s * kRows + row0 + lane].w, kc_b = aux_s[s * kRows + row0 + 32 + lane].w;
+      if (last) {
+        tc::named_bar_sync(1, 128);
+        if (threadIdx.x == 12 * 32) tc::mbar_arrive(&slot_free[s]);
+      }
       const uint32_t reg = tmem + lane_base + kRegCol0 + (c % 3) * kRegCols;
-      const uint8_t* xt = smem + Lay::kQK + s * Lay::kTile + (d >> 6) * Lay::kHalf;
-      const int dc = (d & 63) >> 3, de = d & 7;
       float* dq_w = p.dqk + bh * L * kD + 32 * q;  // this warp's 32 features
       float* dv_w = p.dv + bh * L * kD + 32 * q;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        const int32_t* pm = perm_s + s * kRows + row0 + 32 * h;
-        uint32_t hr[32], vr[32];
+        // x of token 32 h + e, feature d (bf16 -> fp32 is a shift)
+        auto xv = [&](int e) { return __uint_as_float(h ? (xpk[e] & 0xffff0000u) : (xpk[e] << 16)); };
+        uint32_t hr[32];
         tc::tmem_ld32(reg + 32 * h, hr);
-        tc::tmem_ld32(reg + 64 + 32 * h, vr);
         tc::tmem_wait_ld_regs(hr);
-        tc::tmem_wait_ld_regs(vr);
-        if (h == 1) {
-          tc::tc_fence_before();
-          tc::mbar_arrive(&hv_free[c % 3]);
-        }
-        float x[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e)  // x of token row row0 + 32 h + e, feature d
-          x[e] = __bfloat162float(
-              *reinterpret_cast<const __nv_bfloat16*>(xt + swz(row0 + 32 * h + e, dc) + 2 * de));
         float part;
         {
           float pr2[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pr2[e] = x[e] * __uint_as_float(hr[e]);
+          for (int e = 0; e < 32; ++e) pr2[e] = xv(e) * __uint_as_float(hr[e]);
           part = transpose_reduce(pr2, lane);  // token 32 h + lane, this warp's 32 features
         }
         xh[q * 32 + lane] = part;
@@ -708,25 +711,31 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         const int row_l = row0 + 32 * h + lane;
         const float tot = xh[lane] + xh[32 + lane] + xh[64 + lane] + xh[96 + lane];
         const float rr = r_s[(rbuf * 2) * kRows + row_l] + r_s[(rbuf * 2 + 1) * kRows + row_l];
-        const float coef = (tot - rr) * aux_s[s * kRows + row_l].w;  // (x . G) (||x|| >= 1e-12) / ||x||^2
+        const float coef = (tot - rr) * (h ? kc_b : kc_a);  // (x . G) (||x|| >= 1e-12) / ||x||^2
         tc::named_bar_sync(1, 128);  // xh is reused by the next half
+        const int pos_h = h ? pos_b : pos_a;
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          stage[e * 32 + lane] = fmaf(-__shfl_sync(0xffffffffu, coef, e), x[e], __uint_as_float(hr[e]));
+          stage[e * 32 + lane] = fmaf(-__shfl_sync(0xffffffffu, coef, e), xv(e), __uint_as_float(hr[e]));
         __syncwarp();
-        rows_out(dq_w, pm);
+        rows_out(dq_w, pos_h);
         __syncwarp();
+        {
+          uint32_t vr[32];
+          tc::tmem_ld32(reg + 64 + 32 * h, vr);
+          tc::tmem_wait_ld_regs(vr);
+          if (h == 1) {  // the region's last TMEM read
+            tc::tc_fence_before();
+            tc::mbar_arrive(&hv_free[c % 3]);
+          }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) stage[e * 32 + lane] = __uint_as_float(vr[e]);
+          for (int e = 0; e < 32; ++e) stage[e * 32 + lane] = __uint_as_float(vr[e]);
+        }
         __syncwarp();
-        rows_out(dv_w, pm);
+        rows_out(dv_w, pos_h);
         __syncwarp();
       }
       return true;
-    };
-    auto release = [&](uint32_t s) {  // after the slot's last reader in this warp group
-      tc::named_bar_sync(1, 128);
-      if (threadIdx.x == 12 * 32) tc::mbar_arrive(&slot_free[s]);
     };
     uint32_t F = 0;
     while (f.valid) {
@@ -736,17 +745,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         f.advance(p);
         continue;
       }
-      if (f.owns_prev()) {  // chunk 2t-1 (rows 64.. of the previous slot) finished by this fill's first block
-        if (!chunk_out(n - 1, sp, 64, (ff + 1) & 1, f.bh)) break;
-        release(sp);
-      }
+      // chunk 2t-1 (rows 64.. of the previous slot, its last reader) finished by this fill's first block
+      if (f.owns_prev() && !chunk_out(n - 1, sp, 64, (ff + 1) & 1, f.bh, true)) break;
       if (f.kind == kFull) {
         if (!epi_wait(&slot_full[s], (F >> 1) & 1) || !epi_wait(&r_full[ff & 1], (ff >> 1) & 1)) break;
-        if (!chunk_out(n, s, 0, ff & 1, f.bh)) break;
-        if (f.t == p.n_fills - 1) {  // segment end: chunk 2t+1 has no later queries
-          if (!chunk_out(n + 1, s, 64, ff & 1, f.bh)) break;
-          release(s);
-        }
+        if (!chunk_out(n, s, 0, ff & 1, f.bh, false)) break;
+        // segment end: chunk 2t+1 has no later queries
+        if (f.t == p.n_fills - 1 && !chunk_out(n + 1, s, 64, ff & 1, f.bh, true)) break;
         n += 2;
         ++ff;
       }

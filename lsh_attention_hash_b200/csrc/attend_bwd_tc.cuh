@@ -52,7 +52,9 @@
 // 0 gives 56 to the others with setmaxnreg: 72 / 144 / 144 / 152):
 //   warps 0-1   producers: 16-byte cp.async row gathers (X, V, then dO) through
 //               perm into 128-byte-swizzled tiles, two fill slots for X and V,
-//               one dO tile, plus each row's LSE, Delta and length terms;
+//               one dO tile (warp w its rows 64 w .., each half with its own
+//               barriers, so the next fill's rows 0..63 load during block 2),
+//               plus each row's LSE, Delta and length terms;
 //   warps 2-3   UMMA issuers (lane 0): warp 2 the S and dP of each block, warp 3
 //               the gradient products; warp 2 also owns the TMEM allocation;
 //   warps 4-11  softmax: both warpgroups take every row (TMEM lane), keys
@@ -94,8 +96,8 @@ struct Layout {
   static constexpr uint32_t kStage = kXH + 4 * 32 * 4;      // float [4 warps][32 tokens][32 features]
   static constexpr uint32_t kBar = kStage + 4 * 32 * 32 * 4;
   // slot_full[2] slot_free[2] do_full do_free sp_full sp_free pz_full pz_free
-  // hv_done[3] hv_free[3] r_full[2] done
-  static constexpr int kNumBars = 19;
+  // hv_done[3] hv_free[3] r_full[2] done do_full(rows 64..) do_free(rows 64..)
+  static constexpr int kNumBars = 21;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
   static constexpr uint32_t kSmem = kBytes + 1024;        // slack for 1024-byte alignment
@@ -287,7 +289,7 @@ __device__ __noinline__ void issuer_s(const Params& p, uint8_t* smem, uint32_t t
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* slot_full = bars;
   uint64_t* slot_free = bars + 2;
-  uint64_t* do_full = bars + 4;
+  uint64_t* do_full[2] = {bars + 4, bars + 19};  // dO rows 0..63 / 64..127 landed
   uint64_t* sp_full = bars + 6;
   uint64_t* sp_free = bars + 7;
   const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK), v0 = tc::smem_u32(smem + Lay::kV);
@@ -305,17 +307,23 @@ __device__ __noinline__ void issuer_s(const Params& p, uint8_t* smem, uint32_t t
     }
     const bool full = f.kind == kFull, has_prev = f.has_prev();
     ok = att_tc::issuer_wait(&slot_full[s], (F >> 1) & 1, abort_flag) &&
-         (!has_prev || att_tc::issuer_wait(&slot_full[sp], ((F - 1) >> 1) & 1, abort_flag)) &&
-         att_tc::issuer_wait(do_full, nd & 1, abort_flag);
+         (!has_prev || att_tc::issuer_wait(&slot_full[sp], ((F - 1) >> 1) & 1, abort_flag));
     if (!ok) break;
     tc::tc_fence_after();
     if (full && f.t == f.t0 && !has_prev) tc::umma_commit(&slot_free[sp]);  // nothing of the leading fill is read
     const uint32_t xs = qk0 + s * Lay::kTile, vs = v0 + s * Lay::kTile;
     const uint32_t xp = qk0 + sp * Lay::kTile, vp = v0 + sp * Lay::kTile;
     // blocks: 0 = chunk 2t-1 (rows 64.. of the previous slot), 1 = chunk 2t, 2 = chunk 2t+1
+    // the query rows' dO: block 0 needs rows 0..63 (its rows 64.. are not in its window), blocks 1
+    // and 2 all 128
+    bool top = false, bot = false;
     for (int b = has_prev ? 0 : 1; b <= (full ? 2 : 0); ++b) {
-      ok = att_tc::issuer_wait(sp_free, (kb & 1) ^ 1, abort_flag);
+      ok = att_tc::issuer_wait(sp_free, (kb & 1) ^ 1, abort_flag) &&
+           (top || att_tc::issuer_wait(do_full[0], nd & 1, abort_flag)) &&
+           (b == 0 || bot || att_tc::issuer_wait(do_full[1], nd & 1, abort_flag));
       if (!ok) break;
+      top = true;
+      bot = bot || b > 0;
       tc::tc_fence_after();
       const uint32_t kx = b == 0 ? xp + 64 * 128 : xs + (b == 2 ? 64 * 128 : 0);
       const uint32_t kv = b == 0 ? vp + 64 * 128 : vs + (b == 2 ? 64 * 128 : 0);
@@ -337,7 +345,7 @@ __device__ __noinline__ void issuer_hv(const Params& p, uint8_t* smem, uint32_t 
   using Lay = Layout;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* slot_free = bars + 2;
-  uint64_t* do_free = bars + 5;
+  uint64_t* do_free[2] = {bars + 5, bars + 20};  // dO rows 0..63 / 64..127 read by their last UMMA
   uint64_t* pz_full = bars + 8;
   uint64_t* pz_free = bars + 9;
   uint64_t* hv_done = bars + 10;
@@ -404,6 +412,7 @@ __device__ __noinline__ void issuer_hv(const Params& p, uint8_t* smem, uint32_t 
         mma_run(r1, mdesc(xs, 0), kRowStep, kdesc(zt + 64 * 128, 0), 32, id_q, 4, false);
         tc::umma_commit(pz_free);
         tc::umma_commit(&hv_done[n % 3]);
+        tc::umma_commit(do_free[0]);  // dO rows 0..63: no later UMMA of this fill needs them
       } else {
         // key role of chunk 2t+1: queries of chunk 2t+1 (rows 64..127)
         mma_run(r1, mdesc(xs, 64), kRowStep, mdesc(zt, 64), kRowStep, id_kv, 4, true);
@@ -416,7 +425,9 @@ __device__ __noinline__ void issuer_hv(const Params& p, uint8_t* smem, uint32_t 
       ++kb;
     }
     if (!ok) break;
-    tc::umma_commit(do_free);  // the fill's last dP was read before its softmax wrote the last block
+    // (the dP UMMAs read dO too; each finished before the softmax loaded its block)
+    if (!full) tc::umma_commit(do_free[0]);  // a half fill has one block
+    tc::umma_commit(do_free[1]);
     if (!full) tc::umma_commit(&slot_free[s]);  // the half fill's slot
     if (full) n += 2;
     ++F;
@@ -435,8 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* slot_full = bars;      // [2] a fill's rows and tables landed (64 producer lanes)
   uint64_t* slot_free = bars + 2;  // [2] a fill slot may be refilled
-  uint64_t* do_full = bars + 4;    // dO rows landed (64 producer lanes)
-  uint64_t* do_free = bars + 5;    // dO tile read by the fill's last UMMA
+  uint64_t* do_full[2] = {bars + 4, bars + 19};  // dO rows 0..63 / 64..127 landed (one producer warp)
+  uint64_t* do_free[2] = {bars + 5, bars + 20};  // dO rows 0..63 / 64..127 read by their last UMMA
   uint64_t* sp_full = bars + 6;    // S and dP of a block computed
   uint64_t* sp_free = bars + 7;    // S and dP loaded by the softmax (256)
   uint64_t* pz_full = bars + 8;    // P~ and Z of a block written (256)
@@ -459,8 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       tc::mbar_init(&slot_free[i], 1);
       tc::mbar_init(&r_full[i], 256);
     }
-    tc::mbar_init(do_full, 64);
-    tc::mbar_init(do_free, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(do_full[i], 32);
+      tc::mbar_init(do_free[i], 1);
+    }
     tc::mbar_init(sp_full, 1);
     tc::mbar_init(sp_free, 256);
     tc::mbar_init(pz_full, 256);
@@ -513,9 +526,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         }
         tc::cp_async_arrive(&slot_full[s]);
         if (f.kind != kLead) {  // the fill's dO rows, once the previous fill's UMMAs are done with the tile
-          if (!att_tc::warp_wait(do_free, (nd & 1) ^ 1, abort_flag)) break;
+          if (!att_tc::warp_wait(do_free[pw], (nd & 1) ^ 1, abort_flag)) break;
           if (mine) gather64(tc::smem_u32(smem + Lay::kDO), p.dout, f.bh * L, pw, pos);
-          tc::cp_async_arrive(do_full);
+          tc::cp_async_arrive(do_full[pw]);
           ++nd;
         }
         ++F;

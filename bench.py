@@ -510,7 +510,11 @@ def run_ours(args, w, rank, world, local_rank):
             "ms": bwd_ms / bwd_steps, "value": world * w.tokens / (bwd_ms / bwd_steps / 1e3), "unit": UNIT,
             "steps": bwd_steps, "gpu_launches": b_launches,
             "roofline": {"bound": b_bound, "achieved": b_ach, "peak": b_peak, "unit": b_unit,
-                         "frac": b_ach / b_peak, "traffic": None, "peak_source": b_src},
+                         "frac": b_ach / b_peak,
+                         "traffic": (recorded_traffic("backward", args.workload)
+                                     if backward_on_tensor_cores(w, args) else None),
+                         "traffic_note": "DRAM bytes of one round launch (ncu, profiles/traffic.json)",
+                         "peak_source": b_src},
             "note": b_note}
     print(json.dumps(line), flush=True)
 

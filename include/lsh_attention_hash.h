@@ -204,7 +204,10 @@ LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H
  *              number of rounds r' with buckets[r'][i] == buckets[r'][j] (the
  *              article's multi-round union: lsh_combine_rounds then counts each
  *              shared key once).  Every mask runs on the tensor-core path
- *              (UNION there for up to 8 rounds) and on the CUDA-core path
+ *              (UNION there for up to 8 rounds, with a stream-ordered scratch
+ *              buffer of 32 bytes per token, cudaMallocAsync / cudaFreeAsync on
+ *              `stream`, holding each token's buckets in all rounds) and on the
+ *              CUDA-core path
  *   scale      logit scale; <= 0 selects 1/sqrt(D).  logit(s, t) =
  *              scale * qk[perm[s]] . qk[perm[t]] / ||qk[perm[t]]||
  *   out_rounds [B, H, n_rounds, L, D] out_dtype  out: per-round softmax-weighted

@@ -122,7 +122,24 @@ struct Params {
   const uint8_t* qk;     // row sources (qk / v, or their sorted copies)
   const uint8_t* v;
   int out_v8;            // output rows 32-byte aligned: 32-byte stores
+  // union correction: [bh][L][8] each token's bucket in every round of its (b, h) slice (-2: no
+  // such round), 32 bytes per token, so that a row's eight buckets arrive as one sector
+  const int32_t* bk_rows;
 };
+
+// Packs the union correction's per-token rows from buckets [bh][n_rounds][L]: one thread per token.
+__global__ void union_rows_kernel(const int32_t* __restrict__ buckets, long long n_tok, int n_rounds, int L,
+                                  int32_t* __restrict__ rows) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n_tok) return;
+  const long long bh = t / L, pos = t - bh * L;
+  int v[kUnionRounds];
+#pragma unroll
+  for (int r = 0; r < kUnionRounds; ++r) v[r] = r < n_rounds ? buckets[(bh * n_rounds + r) * L + pos] : -2;
+  int4* dst = reinterpret_cast<int4*>(rows + t * kUnionRounds);
+  dst[0] = make_int4(v[0], v[1], v[2], v[3]);
+  dst[1] = make_int4(v[4], v[5], v[6], v[7]);
+}
 
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_inc() {
@@ -319,16 +336,11 @@ __device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, ui
       perm_s[i] = pos[k];
       if (BUCKET)  // the row's bucket lands with the row (same cp.async group, same barrier)
         tc::cp_async4(tc::smem_u32(smem + Lay::kBk) + (slot * kRows + i) * 4, p.buckets + f.seg * p.L + pos[k]);
-      if (UNION) {  // the row's bucket in every round of its (b, h) slice (-2: no such round)
-        const long long seg0 = (f.seg / p.n_rounds) * p.n_rounds;
+      if (UNION) {  // the row's bucket in every round of its (b, h) slice: one 32-byte packed row
         const uint32_t dst = tc::smem_u32(smem + Lay::kBkAll) + ((slot * kRows + i) * kUnionRounds) * 4;
-#pragma unroll
-        for (int rr = 0; rr < kUnionRounds; ++rr) {
-          if (rr < p.n_rounds)
-            tc::cp_async4(dst + rr * 4, p.buckets + (seg0 + rr) * p.L + pos[k]);
-          else
-            reinterpret_cast<int32_t*>(smem + Lay::kBkAll)[(slot * kRows + i) * kUnionRounds + rr] = -2;
-        }
+        const int32_t* src = p.bk_rows + ((f.seg / p.n_rounds) * p.L + pos[k]) * kUnionRounds;
+        tc::cp_async16(dst, src);
+        tc::cp_async16(dst + 16, src + 4);
       }
       grow[k] = p.sorted_input ? f.seg * p.L + chunk * kC + (i & 63) : (f.seg / p.n_rounds) * p.L + pos[k];
     }

@@ -169,6 +169,7 @@ template <int D, typename TO, int MASK>
 lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted, const void* v_sorted,
                             const int32_t* perm, const int32_t* buckets, int B, int H, int L, int n_rounds,
                             int self_mask, float scale, void* out, float* lse, cudaStream_t s, int sms) {
+  constexpr bool kUnion = (MASK & lsh::att_tc::kMaskUnion) != 0;
   using namespace lsh::att_tc;
   const long long segs = (long long)B * H * n_rounds;
   const bool sorted = qk_sorted != nullptr;
@@ -190,13 +191,28 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
   p.qk = (const uint8_t*)(sorted ? qk_sorted : qk);
   p.v = (const uint8_t*)(sorted ? v_sorted : v);
   p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
+  p.bk_rows = nullptr;
+  int32_t* rows = nullptr;
+  if (kUnion) {  // every round's bucket of each token in one 32-byte row (stream-ordered scratch)
+    const long long n_tok = (long long)B * H * L;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&rows), (size_t)n_tok * kUnionRounds * sizeof(int32_t), s) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    union_rows_kernel<<<(unsigned)((n_tok + 255) / 256), 256, 0, s>>>(buckets, n_tok, n_rounds, L, rows);
+    p.bk_rows = rows;
+  }
   const unsigned grid = (unsigned)std::min<long long>(p.n_units, sms);
   auto kfn = attend_tc_kernel<D, TO, MASK>;
   const int smem = (int)Layout<D>::kSmem;
-  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return LSH_ERR_CUDA;
-  kfn<<<grid, kThreads, smem, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
+  lsh_status st = LSH_OK;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    st = LSH_ERR_CUDA;
+  } else {
+    kfn<<<grid, kThreads, smem, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) st = LSH_ERR_CUDA;
+  }
+  if (rows && cudaFreeAsync(rows, s) != cudaSuccess && st == LSH_OK) st = LSH_ERR_CUDA;
+  return st;
 }
 
 // Tensor-core backward (bf16 rows and out / dout, D 128, chunk 64, L % 128 == 0,

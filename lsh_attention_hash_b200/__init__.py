@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     lsh_chunk_attend_backward,
     lsh_get_device_status,
     lsh_attention,
+    lsh_attention_host,
     library_path,
     load_library,
 )

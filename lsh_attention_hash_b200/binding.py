@@ -329,6 +329,85 @@ def lsh_attention(qk, v, R, n_buckets, chunk, *, self_mask=True, causal=False, b
     return out
 
 
+def lsh_attention_host(qk_h, v_h, R, n_buckets, chunk, out_h, *, groups=8, self_mask=True, causal=False,
+                       bucket_mask=False, union=False, scale=None, stream=None, state=None):
+    """The forward pass on host data: ``qk_h``, ``v_h`` [B, H, L, D] in pinned host memory, the
+    merged output written into ``out_h`` (pinned, same shape); ``R`` on the device or pinned host.
+
+    The B*H (b, h) slices are independent problems, processed in ``groups`` contiguous runs.
+    Three CUDA streams overlap the host-to-device copy of run g + 1, the four library calls on
+    run g and the device-to-host copy of run g - 1 (two device buffers per run tensor, so PCIe
+    carries both directions while the kernels run).  The work starts after what is already
+    queued on ``stream`` (default: the current stream) and ``stream`` waits for all of it, so
+    events recorded on ``stream`` around the call time the copies and the kernels together.
+    ``state`` (a dict) keeps the device buffers and streams between calls; each run's results
+    are those of ``lsh_attention`` on its slices.
+    """
+    for t, nm in ((qk_h, "qk_h"), (v_h, "v_h"), (out_h, "out_h")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous pinned host tensor")
+        if t.dtype != qk_h.dtype or t.shape != qk_h.shape:
+            raise ValueError(f"{nm} must match qk_h ({qk_h.dtype}, {tuple(qk_h.shape)})")
+    B, H, L, D = qk_h.shape
+    dev = R.device if R.is_cuda else torch.device("cuda", torch.cuda.current_device())
+    main = stream if stream is not None else torch.cuda.current_stream(dev)
+    n = B * H
+    G = max(1, min(int(groups), n))
+    bounds = [(n * g) // G for g in range(G + 1)]
+    m_max = max(bounds[g + 1] - bounds[g] for g in range(G))
+    st = state if state is not None else {}
+    key = (n, L, D, qk_h.dtype, tuple(R.shape), n_buckets, G, str(dev))
+    if st.get("key") != key:
+        st.clear()
+        st["key"] = key
+        st["qk"] = [torch.empty((1, m_max, L, D), dtype=qk_h.dtype, device=dev) for _ in range(2)]
+        st["v"] = [torch.empty((1, m_max, L, D), dtype=qk_h.dtype, device=dev) for _ in range(2)]
+        st["out"] = [torch.empty((1, m_max, L, D), dtype=qk_h.dtype, device=dev) for _ in range(2)]
+        st["R"] = torch.empty(R.shape, dtype=R.dtype, device=dev)
+        st["bufs"] = alloc_buffers(1, m_max, L, D, R.shape[0], n_buckets, qk_h.dtype, dev)
+        st["streams"] = [torch.cuda.Stream(dev) for _ in range(3)]
+    s_in, s_run, s_out = st["streams"]
+    qf, vf, of = (t.view(1, n, L, D) for t in (qk_h, v_h, out_h))
+    start = torch.cuda.Event()
+    start.record(main)
+    for s_ in (s_in, s_run, s_out):
+        s_.wait_event(start)
+    if R.is_cuda:
+        Rd = R
+    else:
+        with torch.cuda.stream(s_in):
+            st["R"].copy_(R, non_blocking=True)
+        Rd = st["R"]
+    run_done, out_done = [None] * G, [None] * G
+    for g in range(G):
+        a, b = bounds[g], bounds[g + 1]
+        k, m = g % 2, b - a
+        dq, dv, do = st["qk"][k][:, :m], st["v"][k][:, :m], st["out"][k][:, :m]
+        if g >= 2:  # buffer pair k was last read by run g - 2's calls
+            s_in.wait_event(run_done[g - 2])
+        with torch.cuda.stream(s_in):
+            dq.copy_(qf[:, a:b], non_blocking=True)
+            dv.copy_(vf[:, a:b], non_blocking=True)
+        in_done = torch.cuda.Event()
+        in_done.record(s_in)
+        s_run.wait_event(in_done)
+        if g >= 2:  # output buffer k was last read by run g - 2's device-to-host copy
+            s_run.wait_event(out_done[g - 2])
+        bufs = {nm: (t if nm == "workspace" else t[:, :m]) for nm, t in st["bufs"].items()}
+        bufs["out"] = do
+        lsh_attention(dq, dv, Rd, n_buckets, chunk, self_mask=self_mask, causal=causal, bucket_mask=bucket_mask,
+                      union=union, scale=scale, stream=s_run, bufs=bufs)
+        run_done[g] = torch.cuda.Event()
+        run_done[g].record(s_run)
+        s_out.wait_event(run_done[g])
+        with torch.cuda.stream(s_out):
+            of[:, a:b].copy_(do, non_blocking=True)
+        out_done[g] = torch.cuda.Event()
+        out_done[g].record(s_out)
+    main.wait_event(out_done[G - 1])
+    return out_h
+
+
 def alloc_buffers(B, H, L, D, n_rounds, n_buckets, dtype, device, with_near_tie=False):
     """Preallocated buffers for ``lsh_attention`` (device memory through torch)."""
     ws = lsh_sort_workspace_bytes(B, H, L, n_rounds, n_buckets)

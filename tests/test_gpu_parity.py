@@ -384,3 +384,22 @@ def test_hash_streamed_and_narrow_projection(D, n_buckets, L):
     assert lsh.lsh_get_device_status() == 0
     parity.check_hash(qk, R, w.n_buckets, b, nt, 1e-2)
     assert torch.equal(b, b_nf)
+
+
+@pytest.mark.parametrize("groups,kw", [(3, dict()), (1, dict()), (5, dict(bucket_mask=True, union=True)),
+                                       (2, dict(causal=True))])
+def test_host_pipeline_equals_device_call(groups, kw):
+    """lsh_attention_host (host buffers, runs of slices on three streams) gives exactly the
+    device-resident lsh_attention result: each (b, h) slice is an independent problem."""
+    w = synth.small_workload("host_pipe", 2, 3, 2048, 128, "bf16", 64, 64, 3)
+    qk, v, R = synth.make_inputs(w, seed=4)
+    ref = lsh.lsh_attention(qk.cuda(), v.cuda(), R.cuda(), w.n_buckets, w.chunk, **kw)
+    qk_h, v_h, R_h = qk.pin_memory(), v.pin_memory(), R.pin_memory()
+    out_h = torch.empty_like(qk_h).pin_memory()
+    state = {}
+    for _ in range(2):  # the second call reuses the buffers and streams
+        out_h.zero_()
+        lsh.lsh_attention_host(qk_h, v_h, R_h, w.n_buckets, w.chunk, out_h, groups=groups, state=state, **kw)
+        torch.cuda.synchronize()
+        assert lsh.lsh_get_device_status() == 0
+        assert torch.equal(out_h, ref.cpu())

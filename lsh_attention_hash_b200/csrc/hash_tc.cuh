@@ -96,6 +96,7 @@ struct RowState {
   int best_g;       // its group (16 columns) within the round
   float best_raw;   // largest raw value of that group
   float v1, v2;     // exact top-two |p| (near-tie flag only)
+  float best_abs;   // largest exact |p| so far (wide rounds)
 };
 
 // `mask` is 0x7FFFFFF0, passed in at run time: with the mask in a register
@@ -125,7 +126,37 @@ __device__ __forceinline__ void process16(RowState& st, const uint32_t* raw, int
   }
 }
 
-template <int D, int NC, bool FLAG, int SPLIT, int RS>
+// Wide rounds (thousands of columns per row): after the first few dozen groups a group rarely holds
+// a new row maximum, so each group first takes only its exact largest |p| (a 3-input max tree
+// over the absolute values) and the keyed pass above runs, for the whole warp, only when some lane
+// of the warp has a new maximum.  The row's best group is then the one with the largest exact
+// |p|, and within it the keyed pass picks the column, so the result can differ from the keyed pass
+// over every group only where two values agree to 2^-19 relative, inside the near-tie band.
+__device__ __forceinline__ void process16_wide(RowState& st, const uint32_t* raw, int g, uint32_t mask) {
+  float a[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a[j] = fabsf(__uint_as_float(raw[j]));
+  const float gm = max16(a);
+  const bool rec = gm > st.best_abs;
+  if (__any_sync(0xffffffffu, rec)) {
+    float key[16], val[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      val[j] = __uint_as_float(raw[j]);
+      key[j] = __uint_as_float((raw[j] & mask) | (uint32_t)(15 - j));
+    }
+    const float gk = max16(key);
+    const float gr = max16(val);
+    if (rec) {
+      st.best_key = gk;
+      st.best_g = g;
+      st.best_raw = gr;
+      st.best_abs = gm;
+    }
+  }
+}
+
+template <int D, int NC, bool FLAG, int SPLIT, int RS, bool WIDE = false>
 __global__ void __launch_bounds__(threads_for(SPLIT), 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_r,
                const Params p) {
@@ -296,7 +327,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     uint32_t seq = 0, it = 0;
     bool ok = true;
     for (long long tile = first_tile; ok && tile < p.n_tiles; tile += p.per_round, ++it) {
-      RowState st{-1.f, 0, 0.f, -INFINITY, -INFINITY};
+      RowState st{-1.f, 0, 0.f, -INFINITY, -INFINITY, -1.f};
       for (int c = 0; c < p.nchunks; ++c, ++seq) {
         const int b = seq & 1;
         ok = att_tc::warp_wait(&acc_full[b], (seq >> 1) & 1, abort_flag);
@@ -309,8 +340,13 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
           tc::tmem_ld32(lane_base + tmem + b * NC + col, raw);
           tc::tmem_wait_ld();
           const int g = (c * NC + col) >> 4;
-          process16<FLAG>(st, raw, g, p.key_mask);
-          process16<FLAG>(st, raw + 16, g + 1, p.key_mask);
+          if (WIDE) {
+            process16_wide(st, raw, g, p.key_mask);
+            process16_wide(st, raw + 16, g + 1, p.key_mask);
+          } else {
+            process16<FLAG>(st, raw, g, p.key_mask);
+            process16<FLAG>(st, raw + 16, g + 1, p.key_mask);
+          }
         }
         tc::tc_fence_before();
         tc::mbar_arrive(&acc_empty[b]);

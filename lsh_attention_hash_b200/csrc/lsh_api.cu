@@ -110,7 +110,7 @@ inline bool hash_tc_eligible(int dtype, int D, int half, int n_rounds, const Dev
 }
 inline bool hash_tc_streams_r(int D, int half) { return (long long)D * half * 2 > 128 * 1024; }
 
-template <int D, int NC, bool FLAG, int SPLIT, int RS>
+template <int D, int NC, bool FLAG, int SPLIT, int RS, bool WIDE = false>
 lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, int n_rounds, int half,
                           int32_t* buckets, uint8_t* near_tie, cudaStream_t s, int sms) {
   using namespace lsh::hash_tc;
@@ -135,7 +135,7 @@ lsh_status launch_hash_tc(const void* qk, const void* R, int B, int H, int L, in
   p.per_round = (int)std::max<long long>(1, std::min<long long>(sms / n_rounds, p.n_tiles));
   p.key_mask = 0x7FFFFFF0u;
   const unsigned grid = (unsigned)(p.per_round * n_rounds);
-  auto kfn = hash_tc_kernel<D, NC, FLAG, SPLIT, RS>;
+  auto kfn = hash_tc_kernel<D, NC, FLAG, SPLIT, RS, WIDE>;
   const int smem = (int)Layout<D>::smem_bytes(half, NC, RS);
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return LSH_ERR_CUDA;
@@ -152,7 +152,11 @@ lsh_status dispatch_hash_tc(const void* qk, const void* R, int B, int H, int L, 
                                                                      near_tie, s, sms)                     \
              : launch_hash_tc<D, NC, false, (NC >= 128 ? 4 : 2), RS>(qk, R, B, H, L, n_rounds, half, buckets, \
                                                                       near_tie, s, sms)
-  // streamed projection ring: 3 chunks of 32 KB at D 64, 2 of 64 KB at D 128
+  // streamed projection ring: 3 chunks of 32 KB at D 64, 2 of 64 KB at D 128; rounds of 4096 columns
+  // or more without the near-tie flag take the group-maximum fast path
+  if (hash_tc_streams_r(D, half) && !near_tie && half >= 4096)
+    return launch_hash_tc<D, 256, false, 4, D == 64 ? 3 : 2, true>(qk, R, B, H, L, n_rounds, half, buckets, near_tie,
+                                                                    s, sms);
   if (hash_tc_streams_r(D, half)) LSH_HTC(256, D == 64 ? 3 : 2);
   if (half == 32) {  // one epilogue part (32 columns)
     return near_tie ? launch_hash_tc<D, 32, true, 1, 0>(qk, R, B, H, L, n_rounds, half, buckets, near_tie, s, sms)

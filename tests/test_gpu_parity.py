@@ -374,8 +374,10 @@ def test_hash_streamed_and_narrow_projection(D, n_buckets, L):
     in shared memory (D * n_buckets > 128 K elements; R streams in 256-column chunks through a ring
     for every 128-row tile) and 64 buckets (32 columns, copied into a zero-padded 64-column tile,
     one epilogue part).  Buckets bit-exact against the float64 oracle except flagged rows, ragged
-    row counts, several rounds; the flag-free instantiation (the one the bench times) agrees with
-    the flagged one on every row."""
+    row counts, several rounds.  The flag-free instantiation (the one the bench times; for rounds of
+    4096 columns or more it takes the group-maximum fast path) is checked against the oracle the
+    same way, with the flags of the flagged call, and agrees with the flagged call on every row
+    that is not a near tie."""
     w = synth.small_workload("stream", 1, 2, L, D, "bf16", n_buckets, 64 if L % 64 == 0 else 1, 3)
     qk, v, R = synth.make_inputs(w, seed=21)
     qk_d, R_d = qk.to(DEV), R.to(DEV)
@@ -383,7 +385,24 @@ def test_hash_streamed_and_narrow_projection(D, n_buckets, L):
     b_nf, _ = lsh.lsh_hash(qk_d, R_d, w.n_buckets, with_near_tie=False)
     assert lsh.lsh_get_device_status() == 0
     parity.check_hash(qk, R, w.n_buckets, b, nt, 1e-2)
-    assert torch.equal(b, b_nf)
+    parity.check_hash(qk, R, w.n_buckets, b_nf, nt, 1e-2)
+    clear = nt == 0
+    assert torch.equal(b[clear], b_nf[clear])
+
+
+def test_wide_round_hash_fast_path_at_the_1m_shape():
+    """The flag-free hash at the 1M workload's projection (D 64, 16384 buckets: 8192 columns per
+    round, the group-maximum fast path) on 32768 rows of one head: bit-exact against the float64
+    oracle except near ties (flags from the flagged instantiation)."""
+    w = synth.small_workload("wide", 1, 1, 32768, 64, "bf16", 16384, 64, 4)
+    qk, v, R = synth.make_inputs(w, seed=5)
+    qk_d, R_d = qk.to(DEV), R.to(DEV)
+    b, nt = lsh.lsh_hash(qk_d, R_d, w.n_buckets)
+    b_nf, _ = lsh.lsh_hash(qk_d, R_d, w.n_buckets, with_near_tie=False)
+    assert lsh.lsh_get_device_status() == 0
+    parity.check_hash(qk, R, w.n_buckets, b_nf, nt, 1e-2)
+    clear = nt == 0
+    assert torch.equal(b[clear], b_nf[clear])
 
 
 @pytest.mark.parametrize("groups,kw", [(3, dict()), (1, dict()), (5, dict(bucket_mask=True, union=True)),

@@ -366,8 +366,19 @@ def lsh_attention_host(qk_h, v_h, R, n_buckets, chunk, out_h, *, groups=8, self_
         st["R"] = torch.empty(R.shape, dtype=R.dtype, device=dev)
         st["bufs"] = alloc_buffers(1, m_max, L, D, R.shape[0], n_buckets, qk_h.dtype, dev)
         st["streams"] = [torch.cuda.Stream(dev) for _ in range(3)]
-    s_in, s_run, s_out = st["streams"]
     qf, vf, of = (t.view(1, n, L, D) for t in (qk_h, v_h, out_h))
+    if G == 1:  # one run: nothing to overlap, everything in order on the caller's stream
+        with torch.cuda.stream(main):
+            dq, dv, do = st["qk"][0], st["v"][0], st["out"][0]
+            dq.copy_(qf, non_blocking=True)
+            dv.copy_(vf, non_blocking=True)
+            Rd = R if R.is_cuda else st["R"].copy_(R, non_blocking=True)
+            bufs = dict(st["bufs"], out=do)
+            lsh_attention(dq, dv, Rd, n_buckets, chunk, self_mask=self_mask, causal=causal,
+                          bucket_mask=bucket_mask, union=union, scale=scale, stream=main, bufs=bufs)
+            of.copy_(do, non_blocking=True)
+        return out_h
+    s_in, s_run, s_out = st["streams"]
     start = torch.cuda.Event()
     start.record(main)
     for s_ in (s_in, s_run, s_out):

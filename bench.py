@@ -81,10 +81,10 @@ def backward_flops(w):
 
 
 def backward_on_tensor_cores(w, args):
-    """The library's tensor-core backward serves bf16, D 128, chunk 64, L % 128 == 0 and the plain
-    window (with or without the self mask); everything else runs on the CUDA cores."""
+    """The library's tensor-core backward serves bf16, D 128, chunk 64, L % 128 == 0 with every mask
+    (the union correction up to 8 rounds); everything else runs on the CUDA cores."""
     return (w.dtype == "bf16" and w.D == 128 and w.chunk == 64 and w.L % 128 == 0
-            and not args.causal and not args.bucket_mask and not args.union)
+            and not (args.union and w.n_rounds > 8))
 
 
 def measured_sm_max_mhz(default=1965.0):
@@ -515,7 +515,7 @@ def run_ours(args, w, rank, world, local_rank):
             "roofline": {"bound": b_bound, "achieved": b_ach, "peak": b_peak, "unit": b_unit,
                          "frac": b_ach / b_peak,
                          "traffic": (recorded_traffic("backward", args.workload)
-                                     if backward_on_tensor_cores(w, args) else None),
+                                     if backward_on_tensor_cores(w, args) and not mask_config(args) else None),
                          "traffic_note": "DRAM bytes of one round launch (ncu, profiles/traffic.json)",
                          "peak_source": b_src},
             "note": b_note}

@@ -259,13 +259,16 @@ LSH_API lsh_status lsh_combine_rounds(const void* out_rounds, int in_dtype, cons
  *   dqk, dv    [B, H, L, D] float       out: overwritten (zeroed, then accumulated
  *                                       over the rounds in order; deterministic)
  *
- * Every mask runs.  bf16 rows with bf16 out / dout, D = 128, chunk = 64,
- * L % 128 == 0 and the plain window (self mask on or off) run on the tensor
- * cores of sm_100: a per-token pass (LSE, dout . out, key lengths) into a
- * stream-ordered scratch buffer of 16 bytes per token (cudaMallocAsync /
- * cudaFreeAsync on `stream`; LSH_ERR_CUDA if it cannot be had), then one
- * launch per round.  Everything else runs on the CUDA cores (one launch per
- * round after zeroing dqk / dv).  Both keep the rounds in order, so the
+ * Every mask runs.  bf16 rows with bf16 out / dout, D = 128, chunk = 64 and
+ * L % 128 == 0 run on the tensor cores of sm_100 with every mask (the union
+ * correction up to 8 rounds): a per-token pass (LSE, dout . out, key lengths)
+ * into a stream-ordered scratch buffer of 16 bytes per token, with masks a
+ * per-slot pass (bucket, and whether the window leaves the token alone) into
+ * 4 bytes per token and round, with the union correction each token's buckets
+ * in all rounds (32 bytes per token) (cudaMallocAsync / cudaFreeAsync on
+ * `stream`; LSH_ERR_CUDA if they cannot be had), then one launch per round.
+ * Everything else runs on the CUDA cores (one launch per round after zeroing
+ * dqk / dv).  Both keep the rounds in order, so the
  * result is deterministic.  A key row of zero length takes the clamp's linear
  * branch (its gradient is scaled by 1e12).
  * Requires what lsh_chunk_attend requires and B * H <= 65535.

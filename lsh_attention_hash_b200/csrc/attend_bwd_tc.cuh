@@ -94,14 +94,29 @@ struct Layout {
   static constexpr uint32_t kR = kPerm + 2 * kRows * 4;     // float [2][2][128]: x_i . dQ_i partials
   static constexpr uint32_t kXH = kR + 2 * 2 * kRows * 4;   // float [4][32]: epilogue partial sums
   static constexpr uint32_t kStage = kXH + 4 * 32 * 4;      // float [4 warps][32 tokens][32 features]
-  static constexpr uint32_t kBar = kStage + 4 * 32 * 32 * 4;
+  // masks: int32 [2][128]: the row's bucket in this round | (1 << 31) when its window leaves it alone
+  static constexpr uint32_t kMaskRow = kStage + 4 * 32 * 32 * 4;
+  static constexpr uint32_t kLog2 = kMaskRow + 2 * kRows * 4;  // float [16]: log2(n), union correction
+  static constexpr uint32_t kBar = kLog2 + 16 * 4;
   // slot_full[2] slot_free[2] do_full do_free sp_full sp_free pz_full pz_free
   // hv_done[3] hv_free[3] r_full[2] done do_full(rows 64..) do_free(rows 64..)
   static constexpr int kNumBars = 21;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
-  static constexpr uint32_t kSmem = kBytes + 1024;        // slack for 1024-byte alignment
+  // union correction only: int32 [2][128][8], each row's bucket in every round (-2: no such round);
+  // read by 16-byte copies and loads, so 128-byte aligned
+  static constexpr uint32_t kUnion = (kBytes + 127u) & ~127u;
+  static constexpr uint32_t smem(bool with_union) {
+    return (with_union ? kUnion + 2 * kRows * 8 * 4 : kBytes) + 1024;
+  }
 };
+
+// 16-byte copies and vector accesses land on these regions; the whole layout fits one SM
+static_assert(Layout::kAux % 16 == 0 && Layout::kKinv % 16 == 0 && Layout::kStage % 16 == 0 &&
+                  Layout::kUnion % 16 == 0 && Layout::kBar % 8 == 0 && Layout::kP % 1024 == 0 &&
+                  Layout::kZ % 1024 == 0 && Layout::kDO % 1024 == 0,
+              "backward layout alignment");
+static_assert(Layout::smem(true) <= 227 * 1024, "backward layout exceeds the shared memory of an SM");
 
 struct Params {
   const uint8_t* qk;      // bf16 [bh][L][128]
@@ -121,7 +136,14 @@ struct Params {
   int self_mask;
   float scale;
   int accumulate;         // 0: the first round stores, 1: later rounds add
+  // masks (compile-time bits of the instantiation): [bh][n_rounds][L] by original position, the
+  // token's bucket in the round (bucket mask) | (1 << 31) when its window leaves it alone
+  const int32_t* mask_rows;
+  const int32_t* bk_rows;  // union: [bh][L][8] every round's bucket of each token (-2: no such round)
 };
+
+// Compile-time masks of a backward instantiation (as in the forward's attention).
+constexpr int kMaskCausal = att_tc::kMaskCausal, kMaskBucket = att_tc::kMaskBucket, kMaskUnion = att_tc::kMaskUnion;
 
 enum : int { kLead = 0, kFull = 1, kHalo = 2 };
 
@@ -438,7 +460,10 @@ __device__ __noinline__ void issuer_hv(const Params& p, uint8_t* smem, uint32_t 
   att_tc::drain_wait(done_bar, 0);
 }
 
+template <int MASK>
 __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params p) {
+  constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
+  constexpr bool UNION = (MASK & kMaskUnion) != 0;
   using Lay = Layout;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte-aligned base as an offset from the shared array itself (stays a shared-memory pointer)
@@ -486,6 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
+  if (UNION && threadIdx.x < 16)  // log2 of a shared-round count (0: unused)
+    reinterpret_cast<float*>(smem + Lay::kLog2)[threadIdx.x] = threadIdx.x > 1 ? log2f((float)threadIdx.x) : 0.f;
   if (warp == 2) tc::tmem_alloc(tmem_holder, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
@@ -520,6 +547,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
                           p.perm + (f.bh * p.n_rounds + p.round) * L +
                               (f.kind == kLead ? 2 * f.t0 - 1 : 2 * f.t + (f.kind == kFull ? pw : 0)) * kC +
                               32 * k + lane);
+            if (MASK != 0)  // the row's bucket in this round and whether its window leaves it alone
+              tc::cp_async4(tc::smem_u32(smem + Lay::kMaskRow) + (s * kRows + i) * 4,
+                            p.mask_rows + (f.bh * p.n_rounds + p.round) * L + pos[k]);
+            if (MASK & kMaskUnion) {  // every round's bucket of the row: one 32-byte packed row
+              const uint32_t dst = tc::smem_u32(smem + Lay::kUnion) + (s * kRows + i) * 32;
+              const int32_t* src = p.bk_rows + g * 8;
+              tc::cp_async16(dst, src);
+              tc::cp_async16(dst + 16, src + 4);
+            }
           }
           gather64(qk0 + s * Lay::kTile, p.qk, rb, pw, pos);
           if (f.kind != kHalo) gather64(v0 + s * Lay::kTile, p.v, rb, pw, pos);
@@ -571,7 +607,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
            (!has_prev || att_tc::warp_wait(&slot_full[sp], ((F - 1) >> 1) & 1, abort_flag));
       if (!ok) break;
       // LSE log2 e and Delta of the row (a half fill has rows 0..63 only)
-      const float4 qa = (full || q < 2) ? aux_s[s * kRows + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const bool row_here = full || q < 2;
+      const float4 qa = row_here ? aux_s[s * kRows + i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      // masks: the query's position, bucket, whether it is alone in its window, every round's bucket
+      const int32_t* mrow = reinterpret_cast<const int32_t*>(smem + Lay::kMaskRow);
+      const int32_t* urow = reinterpret_cast<const int32_t*>(smem + Lay::kUnion);
+      const float* lg2 = reinterpret_cast<const float*>(smem + Lay::kLog2);
+      const int qpos = (CAUSAL && row_here) ? perm_s[s * kRows + i] : 0;
+      const int qm = (MASK != 0 && row_here) ? mrow[s * kRows + i] : 0;
+      const bool alone = qm < 0;
+      const int qb = qm & 0x7fffffff;
+      int qu[att_tc::kUnionRounds];
+#pragma unroll
+      for (int rr = 0; rr < att_tc::kUnionRounds; ++rr)
+        qu[rr] = (UNION && row_here && rr < p.n_rounds) ? urow[(s * kRows + i) * 8 + rr] : -1;
       float r = 0.f;                            // x_i . dQ_i over this warp group's keys
       int blocks[3], nb = 0;
       if (has_prev) blocks[nb++] = 0;
@@ -597,9 +646,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         uint32_t pw16[16], zw16[16];
         if (active) {
           // keys of the block: slot and first row
-          const float* kin = kinv_s + (b == 0 ? sp * kRows + 64 : s * kRows + (b == 2 ? 64 : 0)) + 32 * wg;
-          // own key: block 1 for rows 0..63, block 2 for rows 64..127, element `lane` of group wg == q % 2
-          const bool self_grp = p.self_mask && b != 0 && (q & 1) == wg && (b == 1) == (q < 2);
+          const int krow0 = (b == 0 ? sp * kRows + 64 : s * kRows + (b == 2 ? 64 : 0)) + 32 * wg;
+          const float* kin = kinv_s + krow0;
+          // own key: block 1 for rows 0..63, block 2 for rows 64..127, element `lane` of group wg == q % 2;
+          // a row that its masks leave alone keeps it
+          const bool self_grp = p.self_mask && !alone && b != 0 && (q & 1) == wg && (b == 1) == (q < 2);
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const float4 k4 = *reinterpret_cast<const float4*>(kin + e);
@@ -608,8 +659,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const float sv = __uint_as_float(sr[e + u]);
-              float pv = tc::ex2_approx(fmaf(sv, kv[u] * c2, -qa.x));
+              float z2 = fmaf(sv, kv[u] * c2, -qa.x);
+              if (UNION) {  // lowered by log2 of the rounds the pair shares
+                const int4 ka = reinterpret_cast<const int4*>(urow + (krow0 + e + u) * 8)[0];
+                const int4 kb2 = reinterpret_cast<const int4*>(urow + (krow0 + e + u) * 8)[1];
+                z2 -= lg2[(ka.x == qu[0]) + (ka.y == qu[1]) + (ka.z == qu[2]) + (ka.w == qu[3]) + (kb2.x == qu[4]) +
+                          (kb2.y == qu[5]) + (kb2.z == qu[6]) + (kb2.w == qu[7])];
+              }
+              float pv = tc::ex2_approx(z2);
               if (self_grp && e + u == lane) pv = 0.f;
+              if (CAUSAL && perm_s[krow0 + e + u] > qpos) pv = 0.f;
+              if (BUCKET && (mrow[krow0 + e + u] & 0x7fffffff) != qb) pv = 0.f;
               const float zv = pv * (__uint_as_float(dr[e + u]) - qa.y) * (kv[u] * p.scale);
               pe[u] = pv;
               ze[u] = zv;
@@ -779,6 +839,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Masked backward, per (b, h, round) segment and sorted slot: the token's bucket in the round (for
+// the bucket mask) and bit 31 set when its window (its own chunk of 64 and the previous one) holds
+// no other key that the masks admit, so that the token keeps its own key (the self rule).  One CTA
+// per pair of chunks with the chunk before it staged in shared memory; L % 128 == 0.
+template <bool CAUSAL, bool BUCKET>
+__global__ void __launch_bounds__(128) bwd_mask_rows_kernel(const int32_t* __restrict__ perm,
+                                                            const int32_t* __restrict__ buckets, int L,
+                                                            int32_t* __restrict__ mask_rows) {
+  __shared__ int pos_s[192], bk_s[192];
+  const int pairs = L / 128;
+  const long long seg = blockIdx.x / pairs;
+  const int base = (int)(blockIdx.x - seg * pairs) * 128;  // first slot of the pair
+  const int32_t* pseg = perm + seg * L;
+  for (int t = threadIdx.x; t < 192; t += 128) {
+    const int slot = base - 64 + t;
+    int pos = -1, bk = 0;
+    if (slot >= 0) {
+      pos = pseg[slot];
+      if (BUCKET) bk = buckets[seg * L + pos];
+    }
+    pos_s[t] = pos;
+    bk_s[t] = bk;
+  }
+  __syncthreads();
+  const int me = 64 + threadIdx.x;              // this slot in the staged window
+  const int w0 = threadIdx.x < 64 ? 0 : 64;     // its window: the previous chunk and its own
+  const int mypos = pos_s[me], mybk = bk_s[me];
+  bool other = false;
+  for (int t = w0; t < w0 + 128 && !other; ++t)
+    other = t != me && pos_s[t] >= 0 && (!CAUSAL || pos_s[t] < mypos) && (!BUCKET || bk_s[t] == mybk);
+  mask_rows[seg * L + mypos] = (BUCKET ? mybk : 0) | (other ? 0 : (int)0x80000000u);
 }
 
 // Per-token terms of the backward: LSE log2 e, Delta = dout . out, 1/max(||x||, 1e-12)

@@ -219,51 +219,71 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
   return st;
 }
 
-// Tensor-core backward (bf16 rows and out / dout, D 128, chunk 64, L % 128 == 0,
-// plain window) on sm_100: per-token terms into a stream-ordered scratch
-// buffer, then one launch per round.
-lsh_status launch_attend_bwd_tc(const void* qk, const void* v, const int32_t* perm, int B, int H, int L,
-                                int n_rounds, int self_mask, float scale, const void* out, const float* lse,
-                                const void* dout, float* dqk, float* dv, cudaStream_t s, int sms) {
+// Tensor-core backward (bf16 rows and out / dout, D 128, chunk 64, L % 128 == 0; the union
+// correction up to 8 rounds) on sm_100: per-token terms (and, with masks, per-slot mask rows and
+// each token's buckets in every round) into stream-ordered scratch buffers, then one launch per round.
+template <int MASK>
+lsh_status launch_attend_bwd_tc(const void* qk, const void* v, const int32_t* perm, const int32_t* buckets, int B,
+                                int H, int L, int n_rounds, int self_mask, float scale, const void* out,
+                                const float* lse, const void* dout, float* dqk, float* dv, cudaStream_t s, int sms) {
   using namespace lsh::bwd_tc;
+  constexpr bool kCausal = (MASK & kMaskCausal) != 0, kBucket = (MASK & kMaskBucket) != 0;
+  constexpr bool kUnion = (MASK & kMaskUnion) != 0;
+  auto kfn = attend_bwd_tc_kernel<MASK>;
   // the setmaxnreg split hands out exactly the registers the launch holds: 512 threads x 128
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, attend_bwd_tc_kernel) != cudaSuccess || fa.numRegs != 128) return LSH_ERR_UNSUPPORTED;
+  if (cudaFuncGetAttributes(&fa, kfn) != cudaSuccess || fa.numRegs != 128) return LSH_ERR_UNSUPPORTED;
   const long long bhs = (long long)B * H, n_tok = bhs * L;
   float4* aux = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&aux), (size_t)n_tok * sizeof(float4), s) != cudaSuccess)
-    return LSH_ERR_CUDA;
-  const int warps = 8;
-  bwd_aux_kernel<<<(unsigned)((n_tok + warps - 1) / warps), warps * 32, 0, s>>>(
-      (const __nv_bfloat16*)qk, (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, aux, n_tok);
-  Params p;
-  p.qk = (const uint8_t*)qk;
-  p.v = (const uint8_t*)v;
-  p.dout = (const uint8_t*)dout;
-  p.perm = perm;
-  p.aux = aux;
-  p.dqk = dqk;
-  p.dv = dv;
-  p.L = L;
-  p.n_rounds = n_rounds;
-  p.n_fills = L / kRows;
-  p.run = 16;
-  p.units_per_seg = (p.n_fills + p.run - 1) / p.run;
-  p.n_units = bhs * p.units_per_seg;
-  p.self_mask = self_mask;
-  p.scale = scale;
-  const unsigned grid = (unsigned)std::min<long long>(p.n_units, sms);
-  const int smem = (int)Layout::kSmem;
+  int32_t* mask_rows = nullptr;
+  int32_t* bk_rows = nullptr;
   lsh_status st = LSH_OK;
-  if (cudaFuncSetAttribute(attend_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (cudaMallocAsync(reinterpret_cast<void**>(&aux), (size_t)n_tok * sizeof(float4), s) != cudaSuccess ||
+      (MASK != 0 && cudaMallocAsync(reinterpret_cast<void**>(&mask_rows), (size_t)n_tok * n_rounds * 4, s) !=
+                        cudaSuccess) ||
+      (kUnion && cudaMallocAsync(reinterpret_cast<void**>(&bk_rows), (size_t)n_tok * 8 * 4, s) != cudaSuccess))
     st = LSH_ERR_CUDA;
-  for (int r = 0; st == LSH_OK && r < n_rounds; ++r) {  // rounds in order: each token has one writer per launch
-    p.round = r;
-    p.accumulate = r > 0 ? 1 : 0;
-    attend_bwd_tc_kernel<<<grid, kThreads, smem, s>>>(p);
-    if (cudaGetLastError() != cudaSuccess) st = LSH_ERR_CUDA;
+  if (st == LSH_OK) {
+    const int warps = 8;
+    bwd_aux_kernel<<<(unsigned)((n_tok + warps - 1) / warps), warps * 32, 0, s>>>(
+        (const __nv_bfloat16*)qk, (const __nv_bfloat16*)out, (const __nv_bfloat16*)dout, lse, aux, n_tok);
+    if (MASK != 0)
+      bwd_mask_rows_kernel<kCausal, kBucket><<<(unsigned)((L / 128) * bhs * n_rounds), 128, 0, s>>>(perm, buckets, L,
+                                                                                                  mask_rows);
+    if (kUnion)
+      lsh::att_tc::union_rows_kernel<<<(unsigned)((n_tok + 255) / 256), 256, 0, s>>>(buckets, n_tok, n_rounds, L,
+                                                                                    bk_rows);
+    Params p;
+    p.qk = (const uint8_t*)qk;
+    p.v = (const uint8_t*)v;
+    p.dout = (const uint8_t*)dout;
+    p.perm = perm;
+    p.aux = aux;
+    p.dqk = dqk;
+    p.dv = dv;
+    p.L = L;
+    p.n_rounds = n_rounds;
+    p.n_fills = L / kRows;
+    p.run = 16;
+    p.units_per_seg = (p.n_fills + p.run - 1) / p.run;
+    p.n_units = bhs * p.units_per_seg;
+    p.self_mask = self_mask;
+    p.scale = scale;
+    p.mask_rows = mask_rows;
+    p.bk_rows = bk_rows;
+    const unsigned grid = (unsigned)std::min<long long>(p.n_units, sms);
+    const int smem = (int)Layout::smem(kUnion);
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      st = LSH_ERR_CUDA;
+    for (int r = 0; st == LSH_OK && r < n_rounds; ++r) {  // rounds in order: each token has one writer per launch
+      p.round = r;
+      p.accumulate = r > 0 ? 1 : 0;
+      kfn<<<grid, kThreads, smem, s>>>(p);
+      if (cudaGetLastError() != cudaSuccess) st = LSH_ERR_CUDA;
+    }
   }
-  if (cudaFreeAsync(aux, s) != cudaSuccess && st == LSH_OK) st = LSH_ERR_CUDA;
+  for (void* ptr : {static_cast<void*>(aux), static_cast<void*>(mask_rows), static_cast<void*>(bk_rows)})
+    if (ptr && cudaFreeAsync(ptr, s) != cudaSuccess && st == LSH_OK) st = LSH_ERR_CUDA;
   return st;
 }
 
@@ -578,9 +598,21 @@ lsh_status lsh_chunk_attend_backward(const void* qk, const void* v, int dtype, i
   cudaStream_t s = as_stream(stream);
   const DevInfo di = dev_info();
   if (di.major == 10 && dtype == LSH_BF16 && out_dtype == LSH_BF16 && D == 128 && chunk == 64 && L % 128 == 0 &&
-      !causal && !bucket_mask)
-    return launch_attend_bwd_tc(qk, v, perm, B, H, L, n_rounds, self_mask, scale, out, lse, dout, dqk, dv, s,
-                                di.sms);
+      (!union_count || n_rounds <= lsh::att_tc::kUnionRounds)) {
+    using lsh::bwd_tc::kMaskBucket;
+    using lsh::bwd_tc::kMaskCausal;
+    using lsh::bwd_tc::kMaskUnion;
+#define LSH_BWD_TC(MM)                                                                                         \
+  return launch_attend_bwd_tc<MM>(qk, v, perm, buckets, B, H, L, n_rounds, self_mask, scale, out, lse, dout, dqk, \
+                                  dv, s, di.sms)
+    if (union_count && causal) LSH_BWD_TC(kMaskCausal | kMaskBucket | kMaskUnion);
+    if (union_count) LSH_BWD_TC(kMaskBucket | kMaskUnion);
+    if (causal && bucket_mask) LSH_BWD_TC(kMaskCausal | kMaskBucket);
+    if (causal) LSH_BWD_TC(kMaskCausal);
+    if (bucket_mask) LSH_BWD_TC(kMaskBucket);
+    LSH_BWD_TC(0);
+#undef LSH_BWD_TC
+  }
   const size_t grad_bytes = (size_t)bhs * L * D * sizeof(float);
   if (cudaMemsetAsync(dqk, 0, grad_bytes, s) != cudaSuccess || cudaMemsetAsync(dv, 0, grad_bytes, s) != cudaSuccess)
     return LSH_ERR_CUDA;

@@ -97,6 +97,23 @@ def test_tensor_core_backward_matches_oracle(name, shape, kw):
     _check(qk, v, dout, res, dqk, dv, w.chunk, w.torch_dtype, **kw)
 
 
+# The masks on the tensor-core backward: positions, buckets and (union) every round's bucket land with
+# each row; queries that their masks leave alone keep their own key.
+@pytest.mark.parametrize("name,shape,kw", [
+    ("bwd_tc_causal", (1, 2, 1024, 128, "bf16", 16, 64, 2), dict(causal=True)),
+    ("bwd_tc_bucket", (1, 2, 1024, 128, "bf16", 32, 64, 2), dict(bucket_mask=True)),
+    ("bwd_tc_bucket_union", (1, 2, 1024, 128, "bf16", 16, 64, 3), dict(bucket_mask=True, union=True)),
+    ("bwd_tc_causal_bucket_union", (1, 1, 4096, 128, "bf16", 64, 64, 4),
+     dict(causal=True, bucket_mask=True, union=True)),
+    ("bwd_tc_causal_bucket_noself", (1, 1, 2560, 128, "bf16", 32, 64, 2),
+     dict(causal=True, bucket_mask=True, self_mask=False)),
+])
+def test_tensor_core_backward_masks_match_oracle(name, shape, kw):
+    w = synth.small_workload(name, *shape)
+    qk, v, dout, res, dqk, dv = _run(w, zlib.crc32(name.encode()) % 1000, **kw)
+    _check(qk, v, dout, res, dqk, dv, w.chunk, w.torch_dtype, **kw)
+
+
 def test_tensor_core_backward_more_units_than_sms():
     """160 one-fill units: every persistent CTA walks several (b, h) slices."""
     w = synth.small_workload("bwd_tc_many", 10, 16, 128, 128, "bf16", 16, 64, 2)

@@ -75,7 +75,28 @@ constexpr int kRows = 128;
 constexpr int kD = 128;
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol = 0, kPCol = 64, kRegCol0 = 128, kRegCols = 128;
+// TMEM: two S/dP buffers of 128 columns (S 64, dP 64), then two chunk regions of H (64) and dv (64)
+constexpr uint32_t kSPCols = 128, kPOff = 64, kRegCol0 = 256, kRegCols = 128;
+
+// mbarrier indices
+struct Bars {
+  static constexpr int kSlotFull = 0;   // [2] a fill's rows and tables landed (64 producer lanes)
+  static constexpr int kSlotFree = 2;   // [2] a fill slot may be refilled
+  static constexpr int kDoFull = 4;     // dO rows 0..63 landed (producer warp 0)
+  static constexpr int kDoFree = 5;     // dO rows 0..63 read by their last UMMA
+  static constexpr int kSpFull = 6;     // [2] S and dP of a block computed (buffer kb % 2)
+  static constexpr int kSpFree = 8;     // [2] S and dP loaded by the softmax (256)
+  static constexpr int kPzFull = 10;    // P~ and Z of a block written (256)
+  static constexpr int kPzFree = 11;    // P~ and Z read by the block's UMMAs
+  static constexpr int kHvDone = 12;    // [2] a chunk region finished
+  static constexpr int kHvHFree = 14;   // [2][2] a region's H columns 0..31 / 32..63 read by the epilogue (128)
+  static constexpr int kHvVFree = 18;   // [2] a region's dv columns read by the epilogue (128)
+  static constexpr int kRFull = 20;     // [2] x . dQ partials of a fill written (256)
+  static constexpr int kDone = 22;      // every UMMA retired (both issuers)
+  static constexpr int kDoFull1 = 23;   // dO rows 64..127 landed (producer warp 1)
+  static constexpr int kDoFree1 = 24;   // dO rows 64..127 read by their last UMMA
+  static constexpr int kCount = 25;
+};
 // registers per thread after the launch's 128: 72 (producers, issuer), 144 (softmax), 152 (epilogue);
 // 128 x (72 + 2 x 144 + 152) = 65536
 constexpr uint32_t kLowRegs = 72, kSoftRegs = 144, kEpiRegs = 152;
@@ -98,9 +119,7 @@ struct Layout {
   static constexpr uint32_t kMaskRow = kStage + 4 * 32 * 32 * 4;
   static constexpr uint32_t kLog2 = kMaskRow + 2 * kRows * 4;  // float [16]: log2(n), union correction
   static constexpr uint32_t kBar = kLog2 + 16 * 4;
-  // slot_full[2] slot_free[2] do_full do_free sp_full sp_free pz_full pz_free
-  // hv_done[3] hv_free[3] r_full[2] done do_full(rows 64..) do_free(rows 64..)
-  static constexpr int kNumBars = 21;
+  static constexpr int kNumBars = Bars::kCount;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
   // union correction only: int32 [2][128][8], each row's bucket in every round (-2: no such round);
@@ -293,32 +312,33 @@ __device__ __forceinline__ void mma_run(uint32_t d, uint64_t a, uint32_t a_step,
 }
 
 // S = X_fill X_b^T and dP = dO_fill V_b^T of one 64-key block (rows kx / kv of the X / V tiles)
-__device__ __forceinline__ void issue_sdp(uint32_t tmem, uint32_t xs, uint32_t do0, uint32_t kx, uint32_t kv,
+// into the S/dP buffer at TMEM column sp
+__device__ __forceinline__ void issue_sdp(uint32_t sp, uint32_t xs, uint32_t do0, uint32_t kx, uint32_t kv,
                                           uint64_t* sp_full) {
   const uint32_t id_s = tc::idesc_bf16_f32(128, 64, 0, 0);  // both K-major
 #pragma unroll 1
   for (int kk = 0; kk < kD / 16; ++kk) {
-    tc::umma_ss(tmem + kSCol, kdesc(xs, kk), kdesc(kx, kk), id_s, kk > 0);
-    tc::umma_ss(tmem + kPCol, kdesc(do0, kk), kdesc(kv, kk), id_s, kk > 0);
+    tc::umma_ss(sp, kdesc(xs, kk), kdesc(kx, kk), id_s, kk > 0);
+    tc::umma_ss(sp + kPOff, kdesc(do0, kk), kdesc(kv, kk), id_s, kk > 0);
   }
   tc::umma_commit(sp_full);
 }
 
-// Lane 0 of warp 2: the S and dP UMMAs of every block, in fill order; each waits until the softmax
-// has loaded the previous block's S and dP.
+// Lane 0 of warp 2: the S and dP UMMAs of every block, in fill order, into two alternating TMEM
+// buffers; each waits until the softmax has loaded the block two before it from the same buffer.
 __device__ __noinline__ void issuer_s(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag) {
   using Lay = Layout;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
-  uint64_t* slot_full = bars;
-  uint64_t* slot_free = bars + 2;
-  uint64_t* do_full[2] = {bars + 4, bars + 19};  // dO rows 0..63 / 64..127 landed
-  uint64_t* sp_full = bars + 6;
-  uint64_t* sp_free = bars + 7;
+  uint64_t* slot_full = bars + Bars::kSlotFull;
+  uint64_t* slot_free = bars + Bars::kSlotFree;
+  uint64_t* do_full[2] = {bars + Bars::kDoFull, bars + Bars::kDoFull1};  // dO rows 0..63 / 64..127 landed
+  uint64_t* sp_full = bars + Bars::kSpFull;
+  uint64_t* sp_free = bars + Bars::kSpFree;
   const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK), v0 = tc::smem_u32(smem + Lay::kV);
   const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
   FillIt f;
   f.init(p);
-  uint32_t F = 0, nd = 0, kb = 0;  // fills, dO fills, blocks
+  uint32_t F = 0, nd = 0, nf = 0, kb = 0;  // fills, fills with dO rows 0..63, full fills, blocks
   bool ok = true;
   while (ok && f.valid) {
     const uint32_t s = F & 1, sp = (F + 1) & 1;
@@ -337,26 +357,28 @@ __device__ __noinline__ void issuer_s(const Params& p, uint8_t* smem, uint32_t t
     const uint32_t xp = qk0 + sp * Lay::kTile, vp = v0 + sp * Lay::kTile;
     // blocks: 0 = chunk 2t-1 (rows 64.. of the previous slot), 1 = chunk 2t, 2 = chunk 2t+1
     // the query rows' dO: block 0 needs rows 0..63 (its rows 64.. are not in its window), blocks 1
-    // and 2 all 128
+    // and 2 (full fills only) all 128.  Rows 64.. are handed over once per full fill and rows 0..63
+    // once per fill, so that neither barrier can run two phases ahead of its waiter.
     bool top = false, bot = false;
     for (int b = has_prev ? 0 : 1; b <= (full ? 2 : 0); ++b) {
-      ok = att_tc::issuer_wait(sp_free, (kb & 1) ^ 1, abort_flag) &&
+      ok = att_tc::issuer_wait(&sp_free[kb & 1], ((kb >> 1) & 1) ^ 1, abort_flag) &&
            (top || att_tc::issuer_wait(do_full[0], nd & 1, abort_flag)) &&
-           (b == 0 || bot || att_tc::issuer_wait(do_full[1], nd & 1, abort_flag));
+           (b == 0 || bot || att_tc::issuer_wait(do_full[1], nf & 1, abort_flag));
       if (!ok) break;
       top = true;
       bot = bot || b > 0;
       tc::tc_fence_after();
       const uint32_t kx = b == 0 ? xp + 64 * 128 : xs + (b == 2 ? 64 * 128 : 0);
       const uint32_t kv = b == 0 ? vp + 64 * 128 : vs + (b == 2 ? 64 * 128 : 0);
-      issue_sdp(tmem, xs, do0, kx, kv, sp_full);
+      issue_sdp(tmem + (kb & 1) * kSPCols, xs, do0, kx, kv, &sp_full[kb & 1]);
       ++kb;
     }
     ++nd;
+    if (full) ++nf;
     ++F;
     f.advance(p);
   }
-  uint64_t* done_bar = bars + 18;
+  uint64_t* done_bar = bars + Bars::kDone;
   tc::umma_commit(done_bar);
   att_tc::drain_wait(done_bar, 0);
 }
@@ -366,17 +388,19 @@ __device__ __noinline__ void issuer_s(const Params& p, uint8_t* smem, uint32_t t
 __device__ __noinline__ void issuer_hv(const Params& p, uint8_t* smem, uint32_t tmem, volatile int* abort_flag) {
   using Lay = Layout;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
-  uint64_t* slot_free = bars + 2;
-  uint64_t* do_free[2] = {bars + 5, bars + 20};  // dO rows 0..63 / 64..127 read by their last UMMA
-  uint64_t* pz_full = bars + 8;
-  uint64_t* pz_free = bars + 9;
-  uint64_t* hv_done = bars + 10;
-  uint64_t* hv_free = bars + 13;
+  uint64_t* slot_free = bars + Bars::kSlotFree;
+  uint64_t* do_free[2] = {bars + Bars::kDoFree, bars + Bars::kDoFree1};  // dO rows 0..63 / 64..127 read
+  uint64_t* pz_full = bars + Bars::kPzFull;
+  uint64_t* pz_free = bars + Bars::kPzFree;
+  uint64_t* hv_done = bars + Bars::kHvDone;
+  uint64_t* hvh_free = bars + Bars::kHvHFree;
+  uint64_t* hvv_free = bars + Bars::kHvVFree;
   const uint32_t qk0 = tc::smem_u32(smem + Lay::kQK);
   const uint32_t do0 = tc::smem_u32(smem + Lay::kDO);
   const uint32_t pt = tc::smem_u32(smem + Lay::kP), zt = tc::smem_u32(smem + Lay::kZ);
   const uint32_t id_kv = tc::idesc_bf16_f32(128, 64, 1, 1);  // dK^T, dV^T: both MN-major
   const uint32_t id_q = tc::idesc_bf16_f32(128, 64, 1, 0);   // dQ^T: A MN-major, B K-major
+  const uint32_t id_q32 = tc::idesc_bf16_f32(128, 32, 1, 0); // dQ^T for 32 queries
   constexpr uint32_t kRowStep = 16 * 128;                    // 16 tile rows
   FillIt f;
   f.init(p);
@@ -392,70 +416,85 @@ __device__ __noinline__ void issuer_hv(const Params& p, uint8_t* smem, uint32_t 
     const bool full = f.kind == kFull, has_prev = f.has_prev(), owns_prev = f.owns_prev();
     const bool first = full && f.t == f.t0, seg_end = full && f.t == p.n_fills - 1;
     const uint32_t xs = qk0 + s * Lay::kTile, xp = qk0 + sp * Lay::kTile;
-    // regions: chunk 2t-1 -> owned chunk n-1, 2t -> n, 2t+1 -> n+1; the first write into a region
-    // waits until the epilogue has read the chunk three before it
-    const uint32_t rp = tmem + kRegCol0 + ((n + 2) % 3) * kRegCols;
-    const uint32_t r0 = tmem + kRegCol0 + (n % 3) * kRegCols;
-    const uint32_t r1 = tmem + kRegCol0 + ((n + 1) % 3) * kRegCols;
+    // regions: chunk 2t-1 -> owned chunk n-1, 2t -> n, 2t+1 -> n+1, in a ring of two (chunk 2t+1 takes
+    // the region of chunk 2t-1).  Before chunk c first writes H (or dv) the epilogue must have read
+    // the H (dv) columns of chunk c-2: hvh_free / hvv_free[c % 2], parity ((c / 2) & 1) ^ 1.
+    const uint32_t r0 = tmem + kRegCol0 + (n & 1) * kRegCols;        // chunk 2t
+    const uint32_t r1 = tmem + kRegCol0 + ((n + 1) & 1) * kRegCols;  // chunk 2t+1, and chunk 2t-1 before it
+    auto free_wait = [&](uint64_t* bar, uint32_t c) {  // dv columns of chunk c's region
+      if (!att_tc::issuer_wait(&bar[c & 1], ((c >> 1) & 1) ^ 1, abort_flag)) return false;
+      tc::tc_fence_after();
+      return true;
+    };
+    auto free_wait_h = [&](uint32_t c, int half) {  // H columns 32 half .. of chunk c's region
+      if (!att_tc::issuer_wait(&hvh_free[(c & 1) * 2 + half], ((c >> 1) & 1) ^ 1, abort_flag)) return false;
+      tc::tc_fence_after();
+      return true;
+    };
     for (int b = has_prev ? 0 : 1; b <= (full ? 2 : 0); ++b) {
       ok = att_tc::issuer_wait(pz_full, kb & 1, abort_flag);
       if (!ok) break;
       tc::tc_fence_after();
       if (b == 0) {
         if (owns_prev) {  // key role of chunk 2t-1: queries of chunk 2t (rows 0..63)
-          mma_run(rp, mdesc(xs, 0), kRowStep, mdesc(zt, 0), kRowStep, id_kv, 4, true);
-          mma_run(rp + 64, mdesc(do0, 0), kRowStep, mdesc(pt, 0), kRowStep, id_kv, 4, true);
+          mma_run(r1, mdesc(xs, 0), kRowStep, mdesc(zt, 0), kRowStep, id_kv, 4, true);
+          mma_run(r1 + 64, mdesc(do0, 0), kRowStep, mdesc(pt, 0), kRowStep, id_kv, 4, true);
         }
         if (full) {
-          ok = att_tc::issuer_wait(&hv_free[n % 3], ((n / 3) & 1) ^ 1, abort_flag);
+          ok = free_wait_h(n, 0) && free_wait_h(n, 1);
           if (!ok) break;
-          tc::tc_fence_after();
           // dQ^T of chunk 2t from the keys of chunk 2t-1
           mma_run(r0, mdesc(xp + 64 * 128, 0), kRowStep, kdesc(zt, 0), 32, id_q, 4, false);
         }
         tc::umma_commit(pz_free);
-        if (owns_prev) tc::umma_commit(&hv_done[(n + 2) % 3]);
+        if (owns_prev) tc::umma_commit(&hv_done[(n + 1) & 1]);
         if (first) tc::umma_commit(&slot_free[sp]);  // the leading fill's slot (full fills: the epilogue)
       } else if (b == 1) {
         if (!has_prev) {
-          ok = att_tc::issuer_wait(&hv_free[n % 3], ((n / 3) & 1) ^ 1, abort_flag);
+          ok = free_wait_h(n, 0) && free_wait_h(n, 1);
           if (!ok) break;
-          tc::tc_fence_after();
         }
         // key role of chunk 2t: all 128 queries
         mma_run(r0, mdesc(xs, 0), kRowStep, mdesc(zt, 0), kRowStep, id_kv, 8, has_prev);
+        ok = free_wait(hvv_free, n);
+        if (!ok) break;
         mma_run(r0 + 64, mdesc(do0, 0), kRowStep, mdesc(pt, 0), kRowStep, id_kv, 8, false);
         // dQ^T of chunk 2t from the keys of chunk 2t
         mma_run(r0, mdesc(xs, 0), kRowStep, kdesc(zt, 0), 32, id_q, 4, true);
-        ok = att_tc::issuer_wait(&hv_free[(n + 1) % 3], (((n + 1) / 3) & 1) ^ 1, abort_flag);
+        // dQ^T of chunk 2t+1 from the keys of chunk 2t, in two 32-query halves, each as soon as the
+        // epilogue has read the same H columns of chunk 2t-1
+        ok = free_wait_h(n + 1, 0);
         if (!ok) break;
-        tc::tc_fence_after();
-        // dQ^T of chunk 2t+1 from the keys of chunk 2t
-        mma_run(r1, mdesc(xs, 0), kRowStep, kdesc(zt + 64 * 128, 0), 32, id_q, 4, false);
+        mma_run(r1, mdesc(xs, 0), kRowStep, kdesc(zt + 64 * 128, 0), 32, id_q32, 4, false);
+        ok = free_wait_h(n + 1, 1);
+        if (!ok) break;
+        mma_run(r1 + 32, mdesc(xs, 0), kRowStep, kdesc(zt + 96 * 128, 0), 32, id_q32, 4, false);
         tc::umma_commit(pz_free);
-        tc::umma_commit(&hv_done[n % 3]);
+        tc::umma_commit(&hv_done[n & 1]);
         tc::umma_commit(do_free[0]);  // dO rows 0..63: no later UMMA of this fill needs them
       } else {
         // key role of chunk 2t+1: queries of chunk 2t+1 (rows 64..127)
         mma_run(r1, mdesc(xs, 64), kRowStep, mdesc(zt, 64), kRowStep, id_kv, 4, true);
+        ok = free_wait(hvv_free, n + 1);  // chunk 2t-1's dv columns read
+        if (!ok) break;
         mma_run(r1 + 64, mdesc(do0, 64), kRowStep, mdesc(pt, 64), kRowStep, id_kv, 4, false);
         // dQ^T of chunk 2t+1 from the keys of chunk 2t+1
         mma_run(r1, mdesc(xs, 64), kRowStep, kdesc(zt + 64 * 128, 0), 32, id_q, 4, true);
         tc::umma_commit(pz_free);
-        if (seg_end) tc::umma_commit(&hv_done[(n + 1) % 3]);
+        if (seg_end) tc::umma_commit(&hv_done[(n + 1) & 1]);
       }
       ++kb;
     }
     if (!ok) break;
     // (the dP UMMAs read dO too; each finished before the softmax loaded its block)
     if (!full) tc::umma_commit(do_free[0]);  // a half fill has one block
-    tc::umma_commit(do_free[1]);
+    else tc::umma_commit(do_free[1]);        // rows 64..: full fills only
     if (!full) tc::umma_commit(&slot_free[s]);  // the half fill's slot
     if (full) n += 2;
     ++F;
     f.advance(p);
   }
-  uint64_t* done_bar = bars + 18;
+  uint64_t* done_bar = bars + Bars::kDone;
   tc::umma_commit(done_bar);
   att_tc::drain_wait(done_bar, 0);
 }
@@ -469,18 +508,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
   // 1024-byte-aligned base as an offset from the shared array itself (stays a shared-memory pointer)
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
-  uint64_t* slot_full = bars;      // [2] a fill's rows and tables landed (64 producer lanes)
-  uint64_t* slot_free = bars + 2;  // [2] a fill slot may be refilled
-  uint64_t* do_full[2] = {bars + 4, bars + 19};  // dO rows 0..63 / 64..127 landed (one producer warp)
-  uint64_t* do_free[2] = {bars + 5, bars + 20};  // dO rows 0..63 / 64..127 read by their last UMMA
-  uint64_t* sp_full = bars + 6;    // S and dP of a block computed
-  uint64_t* sp_free = bars + 7;    // S and dP loaded by the softmax (256)
-  uint64_t* pz_full = bars + 8;    // P~ and Z of a block written (256)
-  uint64_t* pz_free = bars + 9;    // P~ and Z read by the block's UMMAs
-  uint64_t* hv_done = bars + 10;   // [3] a chunk region finished
-  uint64_t* hv_free = bars + 13;   // [3] a chunk region read by the epilogue (128)
-  uint64_t* r_full = bars + 16;    // [2] x . dQ partials of a fill written (256)
-  uint64_t* done_bar = bars + 18;  // every UMMA retired
+  uint64_t* slot_full = bars + Bars::kSlotFull;
+  uint64_t* slot_free = bars + Bars::kSlotFree;
+  uint64_t* do_full[2] = {bars + Bars::kDoFull, bars + Bars::kDoFull1};
+  uint64_t* do_free[2] = {bars + Bars::kDoFree, bars + Bars::kDoFree1};
+  uint64_t* sp_full = bars + Bars::kSpFull;
+  uint64_t* sp_free = bars + Bars::kSpFree;
+  uint64_t* pz_full = bars + Bars::kPzFull;
+  uint64_t* pz_free = bars + Bars::kPzFree;
+  uint64_t* hv_done = bars + Bars::kHvDone;
+  uint64_t* hvh_free = bars + Bars::kHvHFree;
+  uint64_t* hvv_free = bars + Bars::kHvVFree;
+  uint64_t* r_full = bars + Bars::kRFull;
+  uint64_t* done_bar = bars + Bars::kDone;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
   const float4* aux_s = reinterpret_cast<const float4*>(smem + Lay::kAux);
@@ -499,13 +539,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       tc::mbar_init(do_full[i], 32);
       tc::mbar_init(do_free[i], 1);
     }
-    tc::mbar_init(sp_full, 1);
-    tc::mbar_init(sp_free, 256);
     tc::mbar_init(pz_full, 256);
     tc::mbar_init(pz_free, 1);
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&sp_full[i], 1);
+      tc::mbar_init(&sp_free[i], 256);
       tc::mbar_init(&hv_done[i], 1);
-      tc::mbar_init(&hv_free[i], 128);
+      tc::mbar_init(&hvh_free[2 * i], 128);
+      tc::mbar_init(&hvh_free[2 * i + 1], 128);
+      tc::mbar_init(&hvv_free[i], 128);
     }
     tc::mbar_init(done_bar, 2);
     *abort_flag = 0;
@@ -561,7 +603,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
           if (f.kind != kHalo) gather64(v0 + s * Lay::kTile, p.v, rb, pw, pos);
         }
         tc::cp_async_arrive(&slot_full[s]);
-        if (f.kind != kLead) {  // the fill's dO rows, once the previous fill's UMMAs are done with the tile
+        // the fill's dO rows, once the UMMAs of the previous fill that read them are done: rows 0..63
+        // for every fill with queries, rows 64.. for full fills (a half fill has none)
+        if (f.kind != kLead && (pw == 0 || f.kind == kFull)) {
           if (!att_tc::warp_wait(do_free[pw], (nd & 1) ^ 1, abort_flag)) break;
           if (mine) gather64(tc::smem_u32(smem + Lay::kDO), p.dout, f.bh * L, pw, pos);
           tc::cp_async_arrive(do_full[pw]);
@@ -631,18 +675,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       for (int bi = 0; bi < nb; ++bi) {
         const int b = blocks[bi];
         const bool active = b == 1 || (b == 0 ? q < 2 : q >= 2);  // the block is in the row's window
-        ok = att_tc::warp_wait(sp_full, kb & 1, abort_flag);
+        ok = att_tc::warp_wait(&sp_full[kb & 1], (kb >> 1) & 1, abort_flag);
         if (!ok) break;
         tc::tc_fence_after();
         uint32_t sr[32], dr[32];
         if (active) {
-          tc::tmem_ld32(tmem + lane_base + kSCol + 32 * wg, sr);
-          tc::tmem_ld32(tmem + lane_base + kPCol + 32 * wg, dr);
+          const uint32_t spb = tmem + lane_base + (kb & 1) * kSPCols + 32 * wg;
+          tc::tmem_ld32(spb, sr);
+          tc::tmem_ld32(spb + kPOff, dr);
           tc::tmem_wait_ld_regs(sr);
           tc::tmem_wait_ld_regs(dr);
         }
         tc::tc_fence_before();
-        tc::mbar_arrive(sp_free);
+        tc::mbar_arrive(&sp_free[kb & 1]);
         uint32_t pw16[16], zw16[16];
         if (active) {
           // keys of the block: slot and first row
@@ -747,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
     // partials in r buffer rbuf.  What it needs from the slot is copied to registers first; a
     // chunk that is its slot's last reader (`last`) releases the slot before its arithmetic.
     auto chunk_out = [&](uint32_t c, uint32_t s, int row0, uint32_t rbuf, long long bh, bool last) -> bool {
-      if (!epi_wait(&hv_done[c % 3], (c / 3) & 1)) return false;
+      if (!epi_wait(&hv_done[c & 1], (c >> 1) & 1)) return false;
       tc::tc_fence_after();
       const uint16_t* xt = reinterpret_cast<const uint16_t*>(smem + Lay::kQK + s * Lay::kTile +
                                                              (d >> 6) * Lay::kHalf) + (d & 7);
@@ -762,16 +807,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         tc::named_bar_sync(1, 128);
         if (threadIdx.x == 12 * 32) tc::mbar_arrive(&slot_free[s]);
       }
-      const uint32_t reg = tmem + lane_base + kRegCol0 + (c % 3) * kRegCols;
+      const uint32_t reg = tmem + lane_base + kRegCol0 + (c & 1) * kRegCols;
       float* dq_w = p.dqk + bh * L * kD + 32 * q;  // this warp's 32 features
       float* dv_w = p.dv + bh * L * kD + 32 * q;
+      // per 32-token half: its H columns (released once in registers: the next chunk of this region
+      // writes them first), the key-normalisation term, the dqk rows; then the dv columns
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        // x of token 32 h + e, feature d (bf16 -> fp32 is a shift)
         auto xv = [&](int e) { return __uint_as_float(h ? (xpk[e] & 0xffff0000u) : (xpk[e] << 16)); };
         uint32_t hr[32];
         tc::tmem_ld32(reg + 32 * h, hr);
         tc::tmem_wait_ld_regs(hr);
+        tc::tc_fence_before();
+        tc::mbar_arrive(&hvh_free[(c & 1) * 2 + h]);
         float part;
         {
           float pr2[32];
@@ -786,26 +834,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
         const float rr = r_s[(rbuf * 2) * kRows + row_l] + r_s[(rbuf * 2 + 1) * kRows + row_l];
         const float coef = (tot - rr) * (h ? kc_b : kc_a);  // (x . G) (||x|| >= 1e-12) / ||x||^2
         tc::named_bar_sync(1, 128);  // xh is reused by the next half
-        const int pos_h = h ? pos_b : pos_a;
 #pragma unroll
         for (int e = 0; e < 32; ++e)
           stage[e * 32 + lane] = fmaf(-__shfl_sync(0xffffffffu, coef, e), xv(e), __uint_as_float(hr[e]));
         __syncwarp();
-        rows_out(dq_w, pos_h);
+        rows_out(dq_w, h ? pos_b : pos_a);
         __syncwarp();
-        {
-          uint32_t vr[32];
-          tc::tmem_ld32(reg + 64 + 32 * h, vr);
-          tc::tmem_wait_ld_regs(vr);
-          if (h == 1) {  // the region's last TMEM read
-            tc::tc_fence_before();
-            tc::mbar_arrive(&hv_free[c % 3]);
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) stage[e * 32 + lane] = __uint_as_float(vr[e]);
+      }
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t vr[32];
+        tc::tmem_ld32(reg + 64 + 32 * h, vr);
+        tc::tmem_wait_ld_regs(vr);
+        if (h == 1) {  // the region's last TMEM read
+          tc::tc_fence_before();
+          tc::mbar_arrive(&hvv_free[c & 1]);
         }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) stage[e * 32 + lane] = __uint_as_float(vr[e]);
         __syncwarp();
-        rows_out(dv_w, pos_h);
+        rows_out(dv_w, h ? pos_b : pos_a);
         __syncwarp();
       }
       return true;

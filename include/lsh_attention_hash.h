@@ -205,9 +205,11 @@ LSH_API lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H
  *              article's multi-round union: lsh_combine_rounds then counts each
  *              shared key once).  Every mask runs on the tensor-core path
  *              (UNION there for up to 8 rounds, with a stream-ordered scratch
- *              buffer of 32 bytes per token, cudaMallocAsync / cudaFreeAsync on
- *              `stream`, holding each token's buckets in all rounds) and on the
- *              CUDA-core path
+ *              buffer of 16 bytes per token, cudaMallocAsync / cudaFreeAsync on
+ *              `stream`, holding each token's buckets in all rounds as fp16
+ *              codes; a bucket id outside [0, 30720) has no code and records
+ *              LSH_ERR_UNSUPPORTED in the device status word, its pairs then
+ *              counting no shared round) and on the CUDA-core path
  *   scale      logit scale; <= 0 selects 1/sqrt(D).  logit(s, t) =
  *              scale * qk[perm[s]] . qk[perm[t]] / ||qk[perm[t]]||
  *   out_rounds [B, H, n_rounds, L, D] out_dtype  out: per-round softmax-weighted
@@ -265,7 +267,8 @@ LSH_API lsh_status lsh_combine_rounds(const void* out_rounds, int in_dtype, cons
  * into a stream-ordered scratch buffer of 16 bytes per token, with masks a
  * per-slot pass (bucket, and whether the window leaves the token alone) into
  * 4 bytes per token and round, with the union correction each token's buckets
- * in all rounds (32 bytes per token) (cudaMallocAsync / cudaFreeAsync on
+ * in all rounds (16 bytes per token; bucket ids below 30720, as for
+ * lsh_chunk_attend) (cudaMallocAsync / cudaFreeAsync on
  * `stream`; LSH_ERR_CUDA if they cannot be had), then one launch per round.
  * Everything else runs on the CUDA cores (one launch per round after zeroing
  * dqk / dv).  Both keep the rounds in order, so the

@@ -117,16 +117,15 @@ struct Layout {
   static constexpr uint32_t kStage = kXH + 4 * 32 * 4;      // float [4 warps][32 tokens][32 features]
   // masks: int32 [2][128]: the row's bucket in this round | (1 << 31) when its window leaves it alone
   static constexpr uint32_t kMaskRow = kStage + 4 * 32 * 32 * 4;
-  static constexpr uint32_t kLog2 = kMaskRow + 2 * kRows * 4;  // float [16]: log2(n), union correction
-  static constexpr uint32_t kBar = kLog2 + 16 * 4;
+  static constexpr uint32_t kBar = kMaskRow + 2 * kRows * 4;
   static constexpr int kNumBars = Bars::kCount;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;  // tmem base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
-  // union correction only: int32 [2][128][8], each row's bucket in every round (-2: no such round);
-  // read by 16-byte copies and loads, so 128-byte aligned
+  // union correction only: uint4 [2][128], each row's bucket in every round as 8 fp16 codes (as in
+  // the forward's union rows); read by 16-byte copies and loads, so 128-byte aligned
   static constexpr uint32_t kUnion = (kBytes + 127u) & ~127u;
   static constexpr uint32_t smem(bool with_union) {
-    return (with_union ? kUnion + 2 * kRows * 8 * 4 : kBytes) + 1024;
+    return (with_union ? kUnion + 2 * kRows * 16 : kBytes) + 1024;
   }
 };
 
@@ -158,7 +157,7 @@ struct Params {
   // masks (compile-time bits of the instantiation): [bh][n_rounds][L] by original position, the
   // token's bucket in the round (bucket mask) | (1 << 31) when its window leaves it alone
   const int32_t* mask_rows;
-  const int32_t* bk_rows;  // union: [bh][L][8] every round's bucket of each token (-2: no such round)
+  const uint4* bk_rows;    // union: [bh][L] every round's bucket of each token as 8 fp16 codes
 };
 
 // Compile-time masks of a backward instantiation (as in the forward's attention).
@@ -553,8 +552,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (UNION && threadIdx.x < 16)  // log2 of a shared-round count (0: unused)
-    reinterpret_cast<float*>(smem + Lay::kLog2)[threadIdx.x] = threadIdx.x > 1 ? log2f((float)threadIdx.x) : 0.f;
   if (warp == 2) tc::tmem_alloc(tmem_holder, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
@@ -592,12 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
             if (MASK != 0)  // the row's bucket in this round and whether its window leaves it alone
               tc::cp_async4(tc::smem_u32(smem + Lay::kMaskRow) + (s * kRows + i) * 4,
                             p.mask_rows + (f.bh * p.n_rounds + p.round) * L + pos[k]);
-            if (MASK & kMaskUnion) {  // every round's bucket of the row: one 32-byte packed row
-              const uint32_t dst = tc::smem_u32(smem + Lay::kUnion) + (s * kRows + i) * 32;
-              const int32_t* src = p.bk_rows + g * 8;
-              tc::cp_async16(dst, src);
-              tc::cp_async16(dst + 16, src + 4);
-            }
+            if (MASK & kMaskUnion)  // every round's bucket of the row: one 16-byte packed row
+              tc::cp_async16(tc::smem_u32(smem + Lay::kUnion) + (s * kRows + i) * 16, p.bk_rows + g);
           }
           gather64(qk0 + s * Lay::kTile, p.qk, rb, pw, pos);
           if (f.kind != kHalo) gather64(v0 + s * Lay::kTile, p.v, rb, pw, pos);
@@ -655,16 +648,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
       const float4 qa = row_here ? aux_s[s * kRows + i] : make_float4(0.f, 0.f, 0.f, 0.f);
       // masks: the query's position, bucket, whether it is alone in its window, every round's bucket
       const int32_t* mrow = reinterpret_cast<const int32_t*>(smem + Lay::kMaskRow);
-      const int32_t* urow = reinterpret_cast<const int32_t*>(smem + Lay::kUnion);
-      const float* lg2 = reinterpret_cast<const float*>(smem + Lay::kLog2);
+      const uint4* urow = reinterpret_cast<const uint4*>(smem + Lay::kUnion);
       const int qpos = (CAUSAL && row_here) ? perm_s[s * kRows + i] : 0;
       const int qm = (MASK != 0 && row_here) ? mrow[s * kRows + i] : 0;
       const bool alone = qm < 0;
       const int qb = qm & 0x7fffffff;
-      int qu[att_tc::kUnionRounds];
-#pragma unroll
-      for (int rr = 0; rr < att_tc::kUnionRounds; ++rr)
-        qu[rr] = (UNION && row_here && rr < p.n_rounds) ? urow[(s * kRows + i) * 8 + rr] : -1;
+      __half2 qu[4];
+      att_tc::union_query((UNION && row_here) ? urow[s * kRows + i] : make_uint4(0u, 0u, 0u, 0u), p.n_rounds, qu);
       float r = 0.f;                            // x_i . dQ_i over this warp group's keys
       int blocks[3], nb = 0;
       if (has_prev) blocks[nb++] = 0;
@@ -705,12 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_bwd_tc_kernel(const Params
             for (int u = 0; u < 4; ++u) {
               const float sv = __uint_as_float(sr[e + u]);
               float z2 = fmaf(sv, kv[u] * c2, -qa.x);
-              if (UNION) {  // lowered by log2 of the rounds the pair shares
-                const int4 ka = reinterpret_cast<const int4*>(urow + (krow0 + e + u) * 8)[0];
-                const int4 kb2 = reinterpret_cast<const int4*>(urow + (krow0 + e + u) * 8)[1];
-                z2 -= lg2[(ka.x == qu[0]) + (ka.y == qu[1]) + (ka.z == qu[2]) + (ka.w == qu[3]) + (kb2.x == qu[4]) +
-                          (kb2.y == qu[5]) + (kb2.z == qu[6]) + (kb2.w == qu[7])];
-              }
+              if (UNION) z2 -= att_tc::union_log2(urow + krow0 + e + u, qu);  // log2 of the rounds shared
               float pv = tc::ex2_approx(z2);
               if (self_grp && e + u == lane) pv = 0.f;
               if (CAUSAL && perm_s[krow0 + e + u] > qpos) pv = 0.f;

@@ -56,6 +56,8 @@
 // Every wait is bounded; a timeout unwinds the CTA cleanly.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "tc_common.cuh"
 
 namespace lsh {
@@ -81,6 +83,13 @@ constexpr int kMaskBucket = 2;  // a key in another bucket than the query's is n
 // rounds (at most kUnionRounds) whose hash puts query and key in one bucket
 constexpr int kMaskUnion = 4;
 constexpr int kUnionRounds = 8;
+// Union rows code bucket b of a round as the fp16 bit pattern 0x0400 + b: a normal, positive,
+// finite half, and distinct buckets give distinct values, so an fp16 compare is an exact bucket
+// compare and no subnormal flushing can merge two buckets.  Buckets from kUnionMaxBucket up have no
+// code; rounds that do not exist are -1.0 in a key's row and -2.0 in a query's, so they never agree.
+constexpr int kUnionMaxBucket = 0x7C00 - 0x0400;  // 30720: 0x7C00 is +inf
+constexpr uint16_t kUnionKeyNone = 0xBC00;        // -1.0
+constexpr uint16_t kUnionQueryNone = 0xC000;      // -2.0
 
 template <int D>
 struct Layout {
@@ -93,10 +102,9 @@ struct Layout {
   static constexpr uint32_t kPerm = kOnes + 16 * 128;               // int32 [kSlots][128]
   static constexpr uint32_t kColMul = kPerm + kSlots * kRows * 4;   // float [kSlots][128]
   static constexpr uint32_t kBk = kColMul + kSlots * kRows * 4;     // int32 [kSlots][128] (bucket mask)
-  // int32 [kSlots][128][8]: every round's bucket of each row (union correction)
+  // uint4 [kSlots][128]: every round's bucket of each row as 8 fp16 codes (union correction)
   static constexpr uint32_t kBkAll = kBk + kSlots * kRows * 4;
-  static constexpr uint32_t kLog2 = kBkAll + kSlots * kRows * kUnionRounds * 4;  // float [16]: log2(n)
-  static constexpr uint32_t kBar = kLog2 + 16 * 4;
+  static constexpr uint32_t kBar = kBkAll + kSlots * kRows * 16;
   // full[3] empty[3] cm_full[3] s_full[2] p_ready[2] o_full[2] buf_empty[2] done
   static constexpr int kNumBars = 18;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;   // tmem base, abort flag
@@ -122,23 +130,35 @@ struct Params {
   const uint8_t* qk;     // row sources (qk / v, or their sorted copies)
   const uint8_t* v;
   int out_v8;            // output rows 32-byte aligned: 32-byte stores
-  // union correction: [bh][L][8] each token's bucket in every round of its (b, h) slice (-2: no
-  // such round), 32 bytes per token, so that a row's eight buckets arrive as one sector
-  const int32_t* bk_rows;
+  // union correction: [bh][L] each token's bucket in every round of its (b, h) slice as 8 fp16 codes
+  // (see kUnionMaxBucket), 16 bytes per token, one copy per row
+  const uint4* bk_rows;
 };
 
-// Packs the union correction's per-token rows from buckets [bh][n_rounds][L]: one thread per token.
+// Packs the union correction's per-token rows from buckets [bh][n_rounds][L]: one thread per token,
+// 8 fp16 codes (round r in halfword r).  A bucket outside [0, kUnionMaxBucket) records
+// LSH_ERR_UNSUPPORTED in the device status word and is coded as a NaN, which agrees with nothing.
 __global__ void union_rows_kernel(const int32_t* __restrict__ buckets, long long n_tok, int n_rounds, int L,
-                                  int32_t* __restrict__ rows) {
+                                  uint4* __restrict__ rows) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= n_tok) return;
   const long long bh = t / L, pos = t - bh * L;
-  int v[kUnionRounds];
+  uint32_t code[kUnionRounds];
 #pragma unroll
-  for (int r = 0; r < kUnionRounds; ++r) v[r] = r < n_rounds ? buckets[(bh * n_rounds + r) * L + pos] : -2;
-  int4* dst = reinterpret_cast<int4*>(rows + t * kUnionRounds);
-  dst[0] = make_int4(v[0], v[1], v[2], v[3]);
-  dst[1] = make_int4(v[4], v[5], v[6], v[7]);
+  for (int r = 0; r < kUnionRounds; ++r) {
+    code[r] = kUnionKeyNone;
+    if (r < n_rounds) {
+      const int b = buckets[(bh * n_rounds + r) * L + pos];
+      if (b >= 0 && b < kUnionMaxBucket) {
+        code[r] = 0x0400u + (uint32_t)b;
+      } else {
+        record_error(LSH_ERR_UNSUPPORTED);
+        code[r] = 0x7E00u;
+      }
+    }
+  }
+  rows[t] = make_uint4(code[0] | (code[1] << 16), code[2] | (code[3] << 16), code[4] | (code[5] << 16),
+                       code[6] | (code[7] << 16));
 }
 
 template <uint32_t N>
@@ -336,12 +356,9 @@ __device__ __forceinline__ void producer_fill(const Params& p, uint8_t* smem, ui
       perm_s[i] = pos[k];
       if (BUCKET)  // the row's bucket lands with the row (same cp.async group, same barrier)
         tc::cp_async4(tc::smem_u32(smem + Lay::kBk) + (slot * kRows + i) * 4, p.buckets + f.seg * p.L + pos[k]);
-      if (UNION) {  // the row's bucket in every round of its (b, h) slice: one 32-byte packed row
-        const uint32_t dst = tc::smem_u32(smem + Lay::kBkAll) + ((slot * kRows + i) * kUnionRounds) * 4;
-        const int32_t* src = p.bk_rows + ((f.seg / p.n_rounds) * p.L + pos[k]) * kUnionRounds;
-        tc::cp_async16(dst, src);
-        tc::cp_async16(dst + 16, src + 4);
-      }
+      if (UNION)  // the row's bucket in every round of its (b, h) slice: one 16-byte packed row
+        tc::cp_async16(tc::smem_u32(smem + Lay::kBkAll) + (slot * kRows + i) * 16,
+                       p.bk_rows + (f.seg / p.n_rounds) * p.L + pos[k]);
       grow[k] = p.sorted_input ? f.seg * p.L + chunk * kC + (i & 63) : (f.seg / p.n_rounds) * p.L + pos[k];
     }
     const uint32_t qk_dst = tc::smem_u32(smem + Lay::kQK + slot * Lay::kSlotBytes);
@@ -380,22 +397,44 @@ __device__ __forceinline__ float row_colmul(const uint8_t* qk_slot, int r, float
   return colscale / fmaxf(sqrtf(ss), 1e-12f);
 }
 
-// The union correction of one key: log2 of the number of rounds whose buckets
-// of query and key agree (`ku`: the key's kUnionRounds buckets, `qu`: the
-// query's, -1 for rounds that do not exist; `lg2`: log2 of 0..8, 0 at 0).
-__device__ __forceinline__ float union_log2(const int32_t* ku, const int (&qu)[kUnionRounds], const float* lg2) {
-  const int4 a = reinterpret_cast<const int4*>(ku)[0], b = reinterpret_cast<const int4*>(ku)[1];
-  const int n = (a.x == qu[0]) + (a.y == qu[1]) + (a.z == qu[2]) + (a.w == qu[3]) + (b.x == qu[4]) +
-                (b.y == qu[5]) + (b.z == qu[6]) + (b.w == qu[7]);
-  return lg2[n];
+// Reinterprets two packed fp16 codes.
+__device__ __forceinline__ __half2 u32_half2(uint32_t w) {
+  __half2 h;
+  memcpy(&h, &w, 4);
+  return h;
+}
+
+// The union correction of one key: log2 of the number of rounds whose buckets of query and key
+// agree (`ku`: the key's row of 8 fp16 codes, `qu`: the query's, with the query-side code for
+// rounds that do not exist).  Four packed compares give 1.0 per agreeing round; a key that shares
+// no round is masked by the bucket test, and its count is taken as 1.
+__device__ __forceinline__ float union_log2(const uint4* ku, const __half2 (&qu)[4]) {
+  const uint4 a = *ku;
+  __half2 c = __heq2(u32_half2(a.x), qu[0]);
+  c = __hadd2(c, __heq2(u32_half2(a.y), qu[1]));
+  c = __hadd2(c, __heq2(u32_half2(a.z), qu[2]));
+  c = __hadd2(c, __heq2(u32_half2(a.w), qu[3]));
+  const float n = __half2float(__hadd(__low2half(c), __high2half(c)));
+  return __log2f(fmaxf(n, 1.f));
+}
+
+// A query row's codes for union_log2: its own row, rounds from n_rounds on replaced by the query-side
+// code.
+__device__ __forceinline__ void union_query(const uint4 row, int n_rounds, __half2 (&qu)[4]) {
+  const uint32_t w[4] = {row.x, row.y, row.z, row.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t lo = 2 * k < n_rounds ? (w[k] & 0xffffu) : kUnionQueryNone;
+    const uint32_t hi = 2 * k + 1 < n_rounds ? (w[k] >> 16) : kUnionQueryNone;
+    qu[k] = u32_half2(lo | (hi << 16));
+  }
 }
 
 template <int D, int MASK>
 __device__ __forceinline__ void softmax_group(uint32_t sbuf, uint32_t pcol, int g, const uint32_t (&cur)[32],
                                               const float* cm, const int32_t* kp, const int32_t* kb, bool dead,
                                               bool self_grp, int lane, float m, float& l, int qpos, int qb,
-                                              int& others, const int32_t* ku, const int (&qu)[kUnionRounds],
-                                              const float* lg2) {
+                                              int& others, const uint4* ku, const __half2 (&qu)[4]) {
   constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
   constexpr bool UNION = (MASK & kMaskUnion) != 0;
   // key multipliers (and positions, buckets) as 16-byte loads: each group's 32 values start on a
@@ -431,8 +470,8 @@ __device__ __forceinline__ void softmax_group(uint32_t sbuf, uint32_t pcol, int 
       if (!dead) others += (int)c0 + (int)c1;
     }
     if (UNION) {  // lower each logit by log2 of the rounds the pair shares
-      v0 -= union_log2(ku + e * kUnionRounds, qu, lg2);
-      v1 -= union_log2(ku + (e + 1) * kUnionRounds, qu, lg2);
+      v0 -= union_log2(ku + e, qu);
+      v1 -= union_log2(ku + e + 1, qu);
     }
     if (self_grp) {
       if (e == lane) v0 = -INFINITY;
@@ -459,8 +498,8 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
                                              const float* cm_hi, int g_first, int g_self, int lane, int self_mask,
                                              float m, float& l, const int32_t* kp_lo, const int32_t* kp_hi,
                                              int qpos, const int32_t* kb_lo, const int32_t* kb_hi, int qb,
-                                             int& others, const int32_t* ku_lo, const int32_t* ku_hi,
-                                             const int (&qu)[kUnionRounds], const float* lg2) {
+                                             int& others, const uint4* ku_lo, const uint4* ku_hi,
+                                             const __half2 (&qu)[4]) {
   uint32_t ra[32], rb[32];
   tc::tmem_ld32(sbuf + scol, ra);
   tc::tmem_wait_ld_regs(ra);
@@ -469,16 +508,16 @@ __device__ __forceinline__ void softmax_pass(uint32_t sbuf, uint32_t scol, uint3
     const float* cm = h ? cm_hi : cm_lo;
     const int32_t* kp = h ? kp_hi : kp_lo;
     const int32_t* kb = h ? kb_hi : kb_lo;
-    const int32_t* ku = h ? ku_hi : ku_lo;
+    const uint4* ku = h ? ku_hi : ku_lo;
     const bool dead = 2 * h < g_first;  // g_first is 0 or 2: both groups of the first half
     tc::tmem_ld32(sbuf + scol + 64 * h + 32, rb);
     softmax_group<D, MASK>(sbuf, pcol, 2 * h, ra, cm, kp, kb, dead, self_mask && 2 * h == g_self, lane, m, l,
-                           qpos, qb, others, ku, qu, lg2);
+                           qpos, qb, others, ku, qu);
     tc::tmem_wait_ld_regs(rb);
     if (h == 0) tc::tmem_ld32(sbuf + scol + 64, ra);
     softmax_group<D, MASK>(sbuf, pcol, 2 * h + 1, rb, cm + 32, kp + 32, kb + 32, dead,
                            self_mask && 2 * h + 1 == g_self, lane, m, l, qpos, qb, others,
-                           ku + 32 * kUnionRounds, qu, lg2);
+                           ku + 32, qu);
     if (h == 0) tc::tmem_wait_ld_regs(ra);
   }
 }
@@ -513,8 +552,8 @@ __device__ __noinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const 
                                                int g_first, int g_self, int lane, int self_mask,
                                                const int32_t* kp_lo, const int32_t* kp_hi, int qpos,
                                                const int32_t* kb_lo, const int32_t* kb_hi, int qb,
-                                               const int32_t* ku_lo, const int32_t* ku_hi,
-                                               const int (&qu)[kUnionRounds], const float* lg2) {
+                                               const uint4* ku_lo, const uint4* ku_hi,
+                                               const __half2 (&qu)[4]) {
   constexpr bool CAUSAL = (MASK & kMaskCausal) != 0, BUCKET = (MASK & kMaskBucket) != 0;
   constexpr bool UNION = (MASK & kMaskUnion) != 0;
   float m = -INFINITY;
@@ -527,11 +566,11 @@ __device__ __noinline__ float exact_row_max(uint32_t sbuf, uint32_t scol, const 
     const float* cm = g < 2 ? cm_lo + 32 * g : cm_hi + 32 * (g - 2);
     const int32_t* kp = g < 2 ? kp_lo + 32 * g : kp_hi + 32 * (g - 2);
     const int32_t* kb = g < 2 ? kb_lo + 32 * g : kb_hi + 32 * (g - 2);
-    const int32_t* ku = g < 2 ? ku_lo + 32 * g * kUnionRounds : ku_hi + 32 * (g - 2) * kUnionRounds;
+    const uint4* ku = g < 2 ? ku_lo + 32 * g : ku_hi + 32 * (g - 2);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       float v = __uint_as_float(raw[e]) * cm[e];
-      if (UNION) v -= union_log2(ku + e * kUnionRounds, qu, lg2);
+      if (UNION) v -= union_log2(ku + e, qu);
       if (CAUSAL && kp[e] > qpos) v = -INFINITY;
       if (BUCKET && kb[e] != qb) v = -INFINITY;
       if (g == g_self && self_mask && e == lane) v = -INFINITY;
@@ -669,8 +708,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
   {
     uint32_t* ones = reinterpret_cast<uint32_t*>(smem + Lay::kOnes);
     for (int i = threadIdx.x; i < 16 * 128 / 4; i += kThreads) ones[i] = 0x3F803F80u;  // two bf16 1.0
-    if (threadIdx.x < 16)  // log2 of a shared-round count (0: unused, the key is masked)
-      reinterpret_cast<float*>(smem + Lay::kLog2)[threadIdx.x] = threadIdx.x > 1 ? log2f((float)threadIdx.x) : 0.f;
     tc::fence_proxy_async_smem();
   }
   if (warp == 2) tc::tmem_alloc(tmem_holder, kTmemCols);
@@ -864,14 +901,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
       const int32_t* kb_hi = low ? bk_s + sc * kRows : bk_s + sc * kRows + 64;
       const int qb = (MASK & kMaskBucket) ? bk_s[sc * kRows + r] : 0;
       // union correction: every round's bucket of the keys (per fill row) and of the query
-      const int32_t* bku = reinterpret_cast<const int32_t*>(smem + Lay::kBkAll);
-      const int32_t* ku_lo = low ? bku + (sp * kRows + 64) * kUnionRounds : bku + (sc * kRows) * kUnionRounds;
-      const int32_t* ku_hi = low ? bku + (sc * kRows) * kUnionRounds : bku + (sc * kRows + 64) * kUnionRounds;
-      const float* lg2 = reinterpret_cast<const float*>(smem + Lay::kLog2);
-      int qu[kUnionRounds];
-#pragma unroll
-      for (int rr = 0; rr < kUnionRounds; ++rr)
-        qu[rr] = ((MASK & kMaskUnion) && rr < p.n_rounds) ? bku[(sc * kRows + r) * kUnionRounds + rr] : -1;
+      const uint4* bku = reinterpret_cast<const uint4*>(smem + Lay::kBkAll);
+      const uint4* ku_lo = low ? bku + sp * kRows + 64 : bku + sc * kRows;
+      const uint4* ku_hi = low ? bku + sc * kRows : bku + sc * kRows + 64;
+      __half2 qu[4];
+      union_query((MASK & kMaskUnion) ? bku[sc * kRows + r] : make_uint4(0u, 0u, 0u, 0u), p.n_rounds, qu);
       const float self_weight = (MASK & kMaskUnion) ? 1.f / (float)p.n_rounds : 1.f;
       int others = 0;
       const int g_first = (low && it.j == 0) ? 2 : 0;  // chunk 0 has no previous chunk
@@ -885,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
         l = 0.f;
         others = 0;
         softmax_pass<D, MASK>(sbuf, scol, pcol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, m, l, kp_lo,
-                              kp_hi, pos, kb_lo, kb_hi, qb, others, ku_lo, ku_hi, qu, lg2);
+                              kp_hi, pos, kb_lo, kb_hi, qb, others, ku_lo, ku_hi, qu);
         if (MASKED) self_only_fixup<MASK>(sbuf, pcol, g_self, lane, others, l, self_weight);
         if (attempt > 0 || !__any_sync(0xffffffffu, !(l > 1e-30f))) break;
         // the bound was too loose for some row of the warp (long query rows): S is
@@ -893,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Params p) 
         // it) and the warp's rows are redone with their exact maxima
         restore_s<D>(smem, sbuf, scol, sp, sc, r, low);
         m = exact_row_max<MASK>(sbuf, scol, cm_lo, cm_hi, g_first, g_self, lane, p.self_mask, kp_lo, kp_hi, pos,
-                                kb_lo, kb_hi, qb, ku_lo, ku_hi, qu, lg2);
+                                kb_lo, kb_hi, qb, ku_lo, ku_hi, qu);
         if (MASKED && m == -INFINITY) m = m_cs;  // self-only row: its own logit is the shift
       }
       {

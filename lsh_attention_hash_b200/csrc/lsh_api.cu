@@ -196,11 +196,10 @@ lsh_status launch_attend_tc(const void* qk, const void* v, const void* qk_sorted
   p.v = (const uint8_t*)(sorted ? v_sorted : v);
   p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   p.bk_rows = nullptr;
-  int32_t* rows = nullptr;
-  if (kUnion) {  // every round's bucket of each token in one 32-byte row (stream-ordered scratch)
+  uint4* rows = nullptr;
+  if (kUnion) {  // every round's bucket of each token in one 16-byte row (stream-ordered scratch)
     const long long n_tok = (long long)B * H * L;
-    if (cudaMallocAsync(reinterpret_cast<void**>(&rows), (size_t)n_tok * kUnionRounds * sizeof(int32_t), s) !=
-        cudaSuccess)
+    if (cudaMallocAsync(reinterpret_cast<void**>(&rows), (size_t)n_tok * sizeof(uint4), s) != cudaSuccess)
       return LSH_ERR_CUDA;
     union_rows_kernel<<<(unsigned)((n_tok + 255) / 256), 256, 0, s>>>(buckets, n_tok, n_rounds, L, rows);
     p.bk_rows = rows;
@@ -236,12 +235,12 @@ lsh_status launch_attend_bwd_tc(const void* qk, const void* v, const int32_t* pe
   const long long bhs = (long long)B * H, n_tok = bhs * L;
   float4* aux = nullptr;
   int32_t* mask_rows = nullptr;
-  int32_t* bk_rows = nullptr;
+  uint4* bk_rows = nullptr;
   lsh_status st = LSH_OK;
   if (cudaMallocAsync(reinterpret_cast<void**>(&aux), (size_t)n_tok * sizeof(float4), s) != cudaSuccess ||
       (MASK != 0 && cudaMallocAsync(reinterpret_cast<void**>(&mask_rows), (size_t)n_tok * n_rounds * 4, s) !=
                         cudaSuccess) ||
-      (kUnion && cudaMallocAsync(reinterpret_cast<void**>(&bk_rows), (size_t)n_tok * 8 * 4, s) != cudaSuccess))
+      (kUnion && cudaMallocAsync(reinterpret_cast<void**>(&bk_rows), (size_t)n_tok * sizeof(uint4), s) != cudaSuccess))
     st = LSH_ERR_CUDA;
   if (st == LSH_OK) {
     const int warps = 8;

@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(threads_for(SPLIT), 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_r,
                const Params p) {
   using Lay = Layout<D>;
+  constexpr uint32_t kRS = RS > 0 ? RS : 1;  // ring stages as a divisor (the resident layout has none)
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte-aligned base as an offset from the shared array itself (not an integer
   // cast), so that every access through it stays a shared-memory access
@@ -244,8 +245,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                           (int)(tile * kRows));
         if (RS > 0) {  // the tile's pass over R[round], chunk by chunk
           for (int c = 0; ok && c < p.nchunks; ++c, ++rq) {
-            const int sr = rq % RS;
-            ok = tc::mbar_wait(&rs_empty[sr], ((rq / RS) & 1) ^ 1, abort_flag);
+            const int sr = rq % kRS;
+            ok = tc::mbar_wait(&rs_empty[sr], ((rq / kRS) & 1) ^ 1, abort_flag);
             if (!ok) break;
             tc::mbar_arrive_expect_tx(&rs_full[sr], (uint32_t)D * NC * 2);
 #pragma unroll
@@ -269,7 +270,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
       }
       for (uint32_t k = (rq > (uint32_t)RS ? rq - RS : 0); k < rq; ++k) {
         const unsigned long long t0 = tc::globaltimer();
-        while (!tc::mbar_try_wait(&rs_full[k % RS], (k / RS) & 1))
+        while (!tc::mbar_try_wait(&rs_full[k % kRS], (k / kRS) & 1))
           if (tc::globaltimer() - t0 > tc::kWaitNs / 16) break;
       }
     }
@@ -287,9 +288,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         if (!ok) break;
         for (int c = 0; c < p.nchunks; ++c, ++seq) {
           const int b = seq & 1;
-          const int sr = RS > 0 ? (int)(rq % RS) : 0;
+          const int sr = RS > 0 ? (int)(rq % kRS) : 0;
           if (RS > 0) {
-            ok = tc::mbar_wait(&rs_full[sr], (rq / RS) & 1, abort_flag);
+            ok = tc::mbar_wait(&rs_full[sr], (rq / kRS) & 1, abort_flag);
             if (!ok) break;
           }
           ok = tc::mbar_wait(&acc_empty[b], ((seq >> 1) & 1) ^ 1, abort_flag);

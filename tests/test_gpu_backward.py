@@ -83,8 +83,9 @@ def test_backward_is_deterministic():
     assert torch.equal(dqk, dqk2) and torch.equal(dv, dv2)
 
 
-# The tensor-core backward serves bf16, D 128, chunk 64, L % 128 == 0 and the plain window: work units of
-# 16 fills (2048 tokens), so L > 2048 has leading and half fills between units.
+# The tensor-core backward serves bf16, D 128, chunk 64, L % 128 == 0 and every mask (the union
+# correction up to 8 rounds): work units of 16 fills (2048 tokens), so L > 2048 has leading and half
+# fills between units.
 @pytest.mark.parametrize("name,shape,kw", [
     ("bwd_tc_one_fill", (1, 1, 128, 128, "bf16", 16, 64, 1), dict()),
     ("bwd_tc_units", (1, 2, 4096, 128, "bf16", 64, 64, 2), dict()),
@@ -114,18 +115,22 @@ def test_tensor_core_backward_masks_match_oracle(name, shape, kw):
     _check(qk, v, dout, res, dqk, dv, w.chunk, w.torch_dtype, **kw)
 
 
-def test_tensor_core_backward_more_units_than_sms():
-    """160 one-fill units: every persistent CTA walks several (b, h) slices."""
+@pytest.mark.parametrize("kw", [dict(), dict(causal=True), dict(bucket_mask=True, union=True)],
+                         ids=["plain", "causal", "bucket_union"])
+def test_tensor_core_backward_more_units_than_sms(kw):
+    """160 one-fill units: every persistent CTA walks several (b, h) slices, with each mask's per-row
+    tables landing in slots that earlier units used."""
     w = synth.small_workload("bwd_tc_many", 10, 16, 128, 128, "bf16", 16, 64, 2)
-    qk, v, dout, res, dqk, dv = _run(w, 11)
-    _check(qk, v, dout, res, dqk, dv, w.chunk, w.torch_dtype, slices=[(0, 0), (3, 7), (9, 15), (5, 0)])
+    qk, v, dout, res, dqk, dv = _run(w, 11, **kw)
+    _check(qk, v, dout, res, dqk, dv, w.chunk, w.torch_dtype, slices=[(0, 0), (3, 7), (9, 15), (5, 0)], **kw)
 
 
-def test_tensor_core_backward_is_deterministic():
+@pytest.mark.parametrize("kw", [dict(), dict(causal=True, bucket_mask=True, union=True)], ids=["plain", "all_masks"])
+def test_tensor_core_backward_is_deterministic(kw):
     w = synth.small_workload("bwd_tc_det", 1, 2, 4096, 128, "bf16", 64, 64, 2)
-    qk, v, dout, res, dqk, dv = _run(w, 5)
+    qk, v, dout, res, dqk, dv = _run(w, 5, **kw)
     dqk2, dv2 = lsh.lsh_chunk_attend_backward(qk.to(DEV), v.to(DEV), res["perm"], w.chunk, res["out"], res["lse"],
-                                              dout.to(DEV))
+                                              dout.to(DEV), buckets=res["buckets"] if kw else None, **kw)
     torch.cuda.synchronize()
     assert torch.equal(dqk, dqk2) and torch.equal(dv, dv2)
 

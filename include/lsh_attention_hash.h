@@ -155,11 +155,13 @@ LSH_API lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L,
  *
  * Shapes with L <= 65536 and n_buckets <= 1024 (the 64K workload among them)
  * are sorted by one CTA per segment entirely in shared memory and touch the
- * array not at all.  Larger shapes run the count-scan-scatter sort, whose
- * counters take B*H*n_rounds * n_buckets * ceil(L / max(4096, n_buckets))
- * uint32 words of the array; the call returns LSH_ERR_WORKSPACE, before any
- * launch, when that exceeds the array's 4 Mi words (16 MiB).  All other
- * argument rules and errors are those of lsh_sort_permute.
+ * array not at all.  Larger shapes run the radix sort (one counting pass per
+ * 8-bit digit of the bucket id), which takes, with S = B*H*n_rounds segments,
+ * S * 256 * ceil(L / 4096) counter words, at most S * 64 + S + 3 more, and, when
+ * n_buckets > 256, 2 * S * L words for the first pass's ids and positions; the
+ * call returns LSH_ERR_WORKSPACE, before any launch, when that exceeds the
+ * array's 4 Mi words (16 MiB).  All other argument rules and errors are those
+ * of lsh_sort_permute.
  *
  * The first call on a device that needs the array looks up its device
  * address (with that device current) and keeps it for the life of the

@@ -21,7 +21,6 @@
 
 namespace {
 
-using lsh::kSortSmemBuckets;
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -339,6 +338,45 @@ lsh_status lsh_hash(const void* qk, int dtype, int B, int H, int L, int D, const
   return launch_status();
 }
 
+// Radix sort of segs segments of L positions (longer than one CTA sorts, or with more buckets), in
+// the workspace ws (lsh::radix_ws words).
+static lsh_status launch_radix_sort(const int32_t* buckets, long long segs, int L, int n_buckets, int32_t* perm,
+                                    int32_t* inv, uint32_t* ws, cudaStream_t s) {
+  const lsh::RadixWs w = lsh::radix_ws(segs, L, n_buckets);
+  const int nt = lsh::radix_tiles(L);
+  const long long n = (long long)lsh::kRadixDigits * nt;
+  const int nch = lsh::sort_scan_chunks(segs, n);
+  const long long C = (n + nch - 1) / nch;
+  uint32_t* cnt = ws + w.cnt;
+  uint32_t* sums = ws + w.sums;
+  uint32_t* valid = ws + w.valid;
+  int32_t* keys1 = reinterpret_cast<int32_t*>(ws + w.keys);
+  int32_t* pos1 = reinterpret_cast<int32_t*>(ws + w.pos);
+  const dim3 grid((unsigned)segs, nt), scan_grid((unsigned)segs, nch);
+  const int threads = lsh::kRadixWarps * 32;
+  const bool two = lsh::radix_passes(n_buckets) > 1;
+  // pass 1: the low digit of the bucket ids
+  lsh::radix_count_kernel<true><<<grid, threads, 0, s>>>(buckets, L, n_buckets, 0, nullptr, cnt);
+  lsh::sort_chunk_sum_kernel<<<scan_grid, 1024, 0, s>>>(cnt, n, C, sums);
+  lsh::sort_scan_kernel<<<scan_grid, 1024, 0, s>>>(cnt, n, C, sums, valid);
+  if (two)
+    lsh::radix_scatter_kernel<true, false><<<grid, threads, 0, s>>>(buckets, nullptr, L, n_buckets, 0, nullptr, cnt,
+                                                                    keys1, pos1, nullptr);
+  else
+    lsh::radix_scatter_kernel<true, true><<<grid, threads, 0, s>>>(buckets, nullptr, L, n_buckets, 0, nullptr, cnt,
+                                                                   nullptr, perm, inv);
+  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+  if (!two) return LSH_OK;
+  // pass 2: the high digit, over the valid ids in the first pass's order
+  const int shift = lsh::kRadixBits;
+  lsh::radix_count_kernel<false><<<grid, threads, 0, s>>>(keys1, L, n_buckets, shift, valid, cnt);
+  lsh::sort_chunk_sum_kernel<<<scan_grid, 1024, 0, s>>>(cnt, n, C, sums);
+  lsh::sort_scan_kernel<<<scan_grid, 1024, 0, s>>>(cnt, n, C, sums, nullptr);
+  lsh::radix_scatter_kernel<false, true><<<grid, threads, 0, s>>>(keys1, pos1, L, n_buckets, shift, valid, cnt,
+                                                                  nullptr, perm, inv);
+  return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
+}
+
 // Shapes sorted by one CTA per segment (no workspace).
 static inline bool sort_by_segment(int L, int n_buckets) {
   return L <= lsh::kSegMaxL && n_buckets <= lsh::kSegMaxBuckets;
@@ -347,7 +385,7 @@ static inline bool sort_by_segment(int L, int n_buckets) {
 size_t lsh_sort_workspace_bytes(int B, int H, int L, int n_rounds, int n_buckets) {
   if (B <= 0 || H <= 0 || L <= 0 || n_rounds <= 0 || n_buckets < 2) return 0;
   if (sort_by_segment(L, n_buckets)) return 0;
-  return lsh::sort_ws_elems((long long)B * H * n_rounds, L, n_buckets) * sizeof(uint32_t);
+  return (size_t)lsh::radix_ws((long long)B * H * n_rounds, L, n_buckets).words * sizeof(uint32_t);
 }
 
 lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L, int n_rounds,
@@ -384,23 +422,8 @@ lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L, int n_r
     lsh::sort_segment_kernel<<<(unsigned)segs, lsh::kSegWarps * 32, smem, s>>>(buckets, L, n_buckets, perm, inv);
     if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
   } else {
-    const int T = lsh::sort_tile(n_buckets);
-    const int nt = (L + T - 1) / T;
-    uint32_t* cnt = (uint32_t*)workspace;
-    const bool in_smem = n_buckets <= kSortSmemBuckets;
-    const size_t hist_smem = in_smem ? (size_t)n_buckets * sizeof(uint32_t) : 0;
-    if (!in_smem && cudaMemsetAsync(cnt, 0, need, s) != cudaSuccess) return LSH_ERR_CUDA;
-    if (hist_smem > 48 * 1024) {
-      cudaFuncSetAttribute(lsh::sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
-      cudaFuncSetAttribute(lsh::sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
-  }
-    dim3 grid((unsigned)segs, nt);
-    lsh::sort_count_kernel<<<grid, 256, hist_smem, s>>>(buckets, L, n_buckets, T, cnt);
-    if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
-    lsh::sort_scan_kernel<<<(unsigned)segs, 1024, 0, s>>>(cnt, (long long)n_buckets * nt);
-    if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
-    lsh::sort_scatter_kernel<<<grid, 32, hist_smem, s>>>(buckets, L, n_buckets, T, cnt, perm, inv);
-    if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
+    const lsh_status st = launch_radix_sort(buckets, segs, L, n_buckets, perm, inv, (uint32_t*)workspace, s);
+    if (st != LSH_OK) return st;
   }
   if (gather) {
     const int row_bytes = D * (int)elt_size(dtype);
@@ -420,7 +443,8 @@ lsh_status lsh_sort_permute(const int32_t* buckets, int B, int H, int L, int n_r
 namespace {
 
 // Scratch of lsh_sort_permute_noalloc: static device memory of this library,
-// 16 MiB of uint32 counters on every device that loads it.
+// 16 MiB of 32-bit words (the radix sort's counters and, with two passes, the
+// first pass's ids and positions) on every device that loads it.
 constexpr size_t kNoallocScratchWords = (size_t)4 << 20;
 __device__ __align__(256) uint32_t g_noalloc_scratch[kNoallocScratchWords];
 
@@ -464,27 +488,12 @@ lsh_status lsh_sort_permute_noalloc(const int32_t* buckets, int B, int H, int L,
     lsh::sort_segment_kernel<<<(unsigned)segs, lsh::kSegWarps * 32, smem, s>>>(buckets, L, n_buckets, perm, inv);
     return launch_status();
   }
-  const size_t words = lsh::sort_ws_elems(segs, L, n_buckets);
+  const size_t words = (size_t)lsh::radix_ws(segs, L, n_buckets).words;
   if (words > kNoallocScratchWords) return LSH_ERR_WORKSPACE;
-  uint32_t* cnt = noalloc_scratch_ptr();
-  if (!cnt) return LSH_ERR_CUDA;
-
-  const int T = lsh::sort_tile(n_buckets);
-  const int nt = (L + T - 1) / T;
-  const bool in_smem = n_buckets <= kSortSmemBuckets;
-  const size_t hist_smem = in_smem ? (size_t)n_buckets * sizeof(uint32_t) : 0;
-  // with global-memory counters the previous call's counts must not leak in
-  if (!in_smem && cudaMemsetAsync(cnt, 0, words * sizeof(uint32_t), s) != cudaSuccess) return LSH_ERR_CUDA;
-  if (hist_smem > 48 * 1024) {
-    cudaFuncSetAttribute(lsh::sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
-    cudaFuncSetAttribute(lsh::sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem);
-  }
-  dim3 grid((unsigned)segs, nt);
-  lsh::sort_count_kernel<<<grid, 256, hist_smem, s>>>(buckets, L, n_buckets, T, cnt);
-  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
-  lsh::sort_scan_kernel<<<(unsigned)segs, 1024, 0, s>>>(cnt, (long long)n_buckets * nt);
-  if (cudaGetLastError() != cudaSuccess) return LSH_ERR_CUDA;
-  lsh::sort_scatter_kernel<<<grid, 32, hist_smem, s>>>(buckets, L, n_buckets, T, cnt, perm, inv);
+  uint32_t* ws = noalloc_scratch_ptr();
+  if (!ws) return LSH_ERR_CUDA;
+  const lsh_status st = launch_radix_sort(buckets, segs, L, n_buckets, perm, inv, ws, s);
+  if (st != LSH_OK) return st;
   return launch_status();
 }
 

@@ -192,8 +192,11 @@ def test_sort_workspace_formula_bounds(lib):
     # whole segments in one CTA need none
     for (B, H, L, nr, nb) in [(8, 8, 65536, 8, 1024), (1, 1, 1024, 1, 16), (8, 8, 16384, 4, 256)]:
         assert lib.lsh_sort_workspace_bytes(B, H, L, nr, nb) == 0
-    # bucket-major per-tile counters: at most 4 bytes per element plus 4 per bucket per segment
+    # radix sort: digit-major counters per 4096-element tile, the scan chunks' sums and the valid
+    # counts, and with two passes (more than 256 buckets) the first pass's ids and positions
     for (B, H, L, nr, nb) in [(1, 8, 1 << 20, 4, 16384), (1, 1, 1024, 1, 2048), (2, 2, 70000, 2, 64)]:
         ws = lib.lsh_sort_workspace_bytes(B, H, L, nr, nb)
         segs = B * H * nr
-        assert 0 < ws <= 4 * segs * (L + nb) + 4 * segs * nb
+        counters = segs * 256 * ((L + 4095) // 4096)
+        pairs = 2 * segs * L if nb > 256 else 0
+        assert 4 * (counters + pairs) < ws <= 4 * (counters + pairs + 66 * segs + 3)
